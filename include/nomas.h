@@ -1,0 +1,223 @@
+/*
+ * nomas.h -- C ABI of libnomas: action-aware segment-causal attention over an
+ * INT8 key/value cache with a sliding history window, for one NVIDIA B200
+ * (sm_100a).
+ *
+ * The operations follow the Hy-Nomas pages (no API is given there; these
+ * signatures are this library's statement of the problem):
+ *   - fluxbbs.com "Hy-Nomas 拆解", section 架构: segment-causal attention
+ *     (bidirectional inside a segment, a segment sees only itself and earlier
+ *     segments, text and video K/V cached for the next segment) and the
+ *     action-aware mask (one description head per segment visible across
+ *     segments, action tails visible only in their own segment and time
+ *     window);
+ *   - same page, section 单卡 4090 怎么做到的: K/V stored as INT8 with float
+ *     scale factors and dequantised to BF16 for compute; retained history
+ *     limited to 18 latent frames; block-sparse attention keeping 25 % of the
+ *     candidate video blocks after the first two denoising steps;
+ *   - hyphentech.top, config table: at most 18 history latent frames on the
+ *     GPU in the single-GPU setting, full history in the standard one.
+ *
+ * Conventions shared by every call
+ *   - Ownership: the caller allocates every device buffer (sizes come from the
+ *     *_bytes / *_layout queries).  The library allocates no device memory
+ *     and never synchronises a stream, except nomas_device_status.
+ *   - Pointers: device pointers, 16-byte aligned; bf16 tensors are
+ *     [tokens][heads][head_dim] with a token stride and a head stride given in
+ *     elements (both multiples of 8, head_dim contiguous).
+ *   - Errors: argument, shape and capacity errors are returned before any work
+ *     is enqueued and leave every state unchanged.  Errors found on the device
+ *     (a bounded wait that ran out, an inconsistent mask buffer) are written to
+ *     the cache's device error word and read by nomas_device_status.
+ *   - Streams: nomas_stream is the CUDA runtime's cudaStream_t; NULL means the
+ *     legacy default stream.  All work of one call goes to that stream.
+ *   - Supported head_dim: 64 and 128.  Supported query rows: video tokens of
+ *     the current segment.
+ */
+#ifndef NOMAS_H
+#define NOMAS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *nomas_stream;
+
+typedef enum {
+    NOMAS_OK = 0,
+    NOMAS_EINVAL = -1,        /* bad argument, shape, stride or alignment */
+    NOMAS_ECAPACITY = -2,     /* ring or head store would overflow */
+    NOMAS_ECUDA = -3,         /* a CUDA runtime / driver call failed */
+    NOMAS_ETIMEOUT = -4,      /* a bounded device wait ran out (device error word) */
+    NOMAS_EDEVICE = -5,       /* inconsistent device data, e.g. a stale mask buffer */
+    NOMAS_EUNSUPPORTED = -6,  /* head_dim or size not supported */
+    NOMAS_ESTATE = -7         /* call order or cache state does not allow the call */
+} nomas_status;
+
+/* Device buffers of a cache, all caller-owned; sizes from nomas_kv_cache_bytes.
+ * Let C = capacity_frames, T = tokens_per_frame, H = heads, D = head_dim, S = head_store_tokens.
+ *   K8, V8   int8  [H][C*T][D]   ring of latent-frame slots; frame g lives in slot g mod C
+ *   KS, VS   fp32  [H][C*T]      one scale per (token, head): value = code * scale
+ *   HK8, HV8 int8  [H][S][D]     description heads of appended segments, in append order
+ *   HKS, HVS fp32  [H][S]
+ *   ERR      int32 [4]           device error word (first error wins) + diagnostics
+ */
+enum {
+    NOMAS_BUF_K8 = 0, NOMAS_BUF_V8, NOMAS_BUF_KS, NOMAS_BUF_VS,
+    NOMAS_BUF_HK8, NOMAS_BUF_HV8, NOMAS_BUF_HKS, NOMAS_BUF_HVS,
+    NOMAS_BUF_ERR, NOMAS_NBUF
+};
+
+typedef struct {
+    int32_t heads;             /* H, >= 1 */
+    int32_t head_dim;          /* D, 64 or 128 */
+    int32_t tokens_per_frame;  /* T, tokens of one latent frame (880 at 1280x704) */
+    int32_t window_frames;     /* W, retained history frames; 0 = keep full history */
+    int32_t capacity_frames;   /* C, ring slots; >= W when W > 0 */
+    int32_t head_store_tokens; /* S, capacity of the description-head store */
+} nomas_cache_dims;
+
+/* One action tail: `len` text tokens visible to query latent frames f0 <= t < f1
+ * (segment-local frames) of its own segment only. */
+typedef struct { int32_t len, f0, f1; } nomas_tail;
+
+/* Text layout of the current segment: head_len description-head tokens followed
+ * by the tails in order.  n_frames latent frames of T video tokens each. */
+typedef struct {
+    int32_t n_frames;
+    int32_t head_len;
+    int32_t n_tails;           /* <= NOMAS_MAX_TAILS */
+    const nomas_tail *tails;   /* host pointer */
+} nomas_segment_text;
+
+#define NOMAS_MAX_TAILS 64
+
+/* Host-mirrored ring state (deterministic from the append sequence). */
+typedef struct {
+    int64_t frames_appended;   /* global latent frames appended so far */
+    int32_t retained_frames;   /* frames visible as history to the next segment */
+    int32_t first_slot;        /* ring slot of the oldest retained frame */
+    int64_t history_tokens;    /* retained_frames * T */
+    int64_t head_tokens;       /* description-head tokens in the store */
+    int32_t segments;          /* successful appends */
+    int32_t _pad;
+} nomas_cache_state;
+
+typedef struct nomas_kv_cache nomas_kv_cache;
+
+/* Total bytes of the cache's device buffers; out_sizes (nullable) receives each
+ * buffer's size.  Returns 0 on invalid dims. */
+size_t nomas_kv_cache_bytes(const nomas_cache_dims *dims, size_t out_sizes[NOMAS_NBUF]);
+
+/* Create a host handle over caller-owned device buffers (bufs[i] sized by
+ * nomas_kv_cache_bytes, 16-byte aligned).  Clears the device error word on
+ * `stream`.  The cache starts empty. */
+int nomas_kv_cache_init(nomas_kv_cache **out, const nomas_cache_dims *dims, void *const bufs[NOMAS_NBUF],
+                        nomas_stream stream);
+
+/* Free the host handle only; the device buffers stay the caller's. */
+int nomas_kv_cache_destroy(nomas_kv_cache *cache);
+
+int nomas_kv_cache_state(const nomas_kv_cache *cache, nomas_cache_state *out);
+
+/* Quantise a finished segment's K/V and write them into the ring (fluxbbs.com
+ * 单卡 4090 怎么做到的, first and second techniques; 架构 for the cache).
+ *   k, v      bf16 [n_frames*T][H][D], strides tok_stride / head_stride (elements)
+ *   head_k/v  bf16 [head_len][H][D], same strides; may be NULL when head_len == 0
+ * Per (token, head): a = max|x|, s = a/127 (fp32, round to nearest), code =
+ * clamp(rint(x/s), -127, 127) with fp32 division and round-half-even; a == 0
+ * gives s = 0 and codes 0.  Frame f of the segment gets global index
+ * g = frames_appended + f and ring slot g mod C; with a window W only frames
+ * f >= n_frames - W are written (older ones would leave the window at once).
+ * The description head is appended to the head store; action tails are never
+ * cached.  Errors: NOMAS_ECAPACITY if the head store would overflow or, with
+ * W == 0, the ring would; the cache is then unchanged. */
+int nomas_kv_append(nomas_kv_cache *cache, const void *k, const void *v, int64_t tok_stride,
+                    int64_t head_stride, int32_t n_frames, const void *head_k, const void *head_v,
+                    int32_t head_len, nomas_stream stream);
+
+#define NOMAS_MODE_DENSE 0
+#define NOMAS_MODE_SPARSE 1
+
+/* Where mask_build puts its results inside the caller's mask buffer.
+ * Key order for tiles and classes: retained history (age order), description
+ * heads of earlier segments, current video, current text (head then tails);
+ * every region is cut into 128-key tiles from its first key.  Query blocks are
+ * 128 current-video rows. */
+typedef struct {
+    int32_t mode, head_dim, heads, n_qblocks;
+    int32_t n_tiles;           /* KV tiles over all four regions */
+    int32_t n_hist_tiles, n_head_tiles, n_cur_tiles, n_text_tiles;
+    int32_t n_cand;            /* sparse candidates: history tiles then current tiles */
+    int32_t keep;              /* kept candidates per (head, query block); 0 in dense mode */
+    int32_t n_lists, list_cap; /* per-CTA tile lists used by nomas_attn_fwd */
+    int32_t _pad;
+    int64_t history_tokens, head_tokens, n_query, text_tokens;
+    size_t off_class;          /* int8  [n_qblocks][n_tiles]: 0 SKIP, 1 FULL, 2 PARTIAL */
+    size_t off_sel;            /* int32 [H][n_qblocks][keep]: kept candidates, score desc then index asc */
+    size_t off_score;          /* fp32  [H][n_qblocks][n_cand] */
+    size_t off_qmean;          /* fp32  [H][n_qblocks][D]   (scratch) */
+    size_t off_kmean;          /* fp32  [H][n_cand][D]      (scratch) */
+    size_t off_txtwin;         /* int32 [text_tokens][2]: visible frame window [lo, hi) per text key */
+    size_t off_count;          /* int32 [n_lists] */
+    size_t off_list;           /* int32x4 [n_lists][list_cap] */
+    size_t total_bytes;
+} nomas_mask_layout;
+
+/* Fill `out` for the current cache state and segment text.  keep_frac in (0, 1]
+ * (sparse only): keep = clamp(ceil(n_cand * keep_frac), 1, n_cand), ceil taken in
+ * double precision of the float value. */
+int nomas_mask_layout_query(const nomas_kv_cache *cache, const nomas_segment_text *seg, int mode,
+                            float keep_frac, nomas_mask_layout *out);
+
+/* Bytes of the mask buffer (0 on invalid arguments). */
+size_t nomas_mask_bytes(const nomas_kv_cache *cache, const nomas_segment_text *seg, int mode, float keep_frac);
+
+/* Build the visibility classes and per-CTA tile lists (fluxbbs.com 架构) and,
+ * in sparse mode, the kept candidate blocks (same page, fourth technique of
+ * 单卡 4090 怎么做到的; the ranking rule is this library's own: per head and
+ * query block, score = fmaf chain over channels of the fp32 mean of the block's
+ * queries and the fp32 mean of the candidate's keys, history keys taken as
+ * float(code) * scale, sums in ascending token order, mean = sum / n_valid).
+ *   q, kcur   bf16 [n_frames*T][H][D] (sparse mode only; NULL allowed in dense)
+ *   mask_buf  device buffer of nomas_mask_bytes bytes, 16-byte aligned
+ * The result is valid for this cache state; an append in between makes
+ * nomas_attn_fwd report NOMAS_EDEVICE through the error word. */
+int nomas_mask_build(const nomas_kv_cache *cache, const nomas_segment_text *seg, int mode, float keep_frac,
+                     const void *q, const void *kcur, int64_t tok_stride, int64_t head_stride, void *mask_buf,
+                     nomas_stream stream);
+
+/* Masked (or block-sparse) attention of the current segment's video queries
+ * over the retained INT8 history, earlier description heads (INT8), the current
+ * segment's video (bf16) and its text (bf16), with the visibility of
+ * nomas_mask_build.  Per head h and query row i:
+ *     O[i,h] = sum_j softmax_j(softmax_scale * q_i . k^_j) v^_j   over visible j
+ * with k^ = code * scale for cached keys (exactly; the key scale is applied to
+ * the fp32 score) and v^ = bf16(code * scale) for cached values.
+ *   q, kcur, vcur  bf16 [n_frames*T][H][D];  ktxt, vtxt bf16 [text_tokens][H][D]
+ *                  (NULL allowed when the segment has no text)
+ *   out            fp32 [n_frames*T][H][D], contiguous
+ *   lse            fp32 [H][n_frames*T] natural-log sum of exp of the scaled
+ *                  scores, nullable */
+int nomas_attn_fwd(const nomas_kv_cache *cache, const nomas_segment_text *seg, int mode, float keep_frac,
+                   const void *mask_buf, const void *q, const void *kcur, const void *vcur, const void *ktxt,
+                   const void *vtxt, int64_t tok_stride, int64_t head_stride, float softmax_scale, float *out,
+                   float *lse, nomas_stream stream);
+
+/* Diagnostic: retained history in age order, dequantised as fp32 code * scale.
+ *   k_out, v_out  fp32 [history_tokens][H][D] */
+int nomas_kv_dequant(const nomas_kv_cache *cache, float *k_out, float *v_out, nomas_stream stream);
+
+/* Synchronise `stream`, read and clear the device error word.  Returns NOMAS_OK
+ * or the first device-side error recorded since the last call. */
+int nomas_device_status(const nomas_kv_cache *cache, nomas_stream stream);
+
+const char *nomas_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NOMAS_H */

@@ -1,0 +1,112 @@
+"""GPU parity of nomas_kv_append (bit-exact INT8 codes, scales and ring placement) and nomas_kv_dequant."""
+import numpy as np
+import pytest
+import torch
+
+from int8_kv_cache_action_b200.workloads import CONFIGS, make_inputs, small_config
+from tests.helpers import f32, gpu_cache, oracle_cache
+
+pytestmark = pytest.mark.gpu
+
+
+def _compare_cache(gc, oc):
+    st = gc.state()
+    assert st["frames_appended"] == oc.frames_appended
+    assert st["head_tokens"] == oc.head_used
+    assert st["history_tokens"] == oc.history_tokens()
+    T = oc.T
+    k8, v8 = gc.ring_k8().cpu().numpy(), gc.ring_v8().cpu().numpy()
+    ks, vs = gc.ring_ks().cpu().numpy(), gc.ring_vs().cpu().numpy()
+    for g in oc.retained_frames():
+        s = slice((g % oc.C) * T, (g % oc.C + 1) * T)
+        assert np.array_equal(k8[:, s], oc.k8[:, s]), f"K codes of frame {g}"
+        assert np.array_equal(v8[:, s], oc.v8[:, s]), f"V codes of frame {g}"
+        assert np.array_equal(ks[:, s].view(np.uint32), oc.ks[:, s].view(np.uint32)), f"K scales of frame {g}"
+        assert np.array_equal(vs[:, s].view(np.uint32), oc.vs[:, s].view(np.uint32)), f"V scales of frame {g}"
+    u = oc.head_used
+    if u:
+        assert np.array_equal(gc.head_k8()[:, :u].cpu().numpy(), oc.hk8[:, :u])
+        assert np.array_equal(gc.head_v8()[:, :u].cpu().numpy(), oc.hv8[:, :u])
+        assert np.array_equal(gc.head_ks()[:, :u].cpu().numpy().view(np.uint32), oc.hks[:, :u].view(np.uint32))
+        assert np.array_equal(gc.head_vs()[:, :u].cpu().numpy().view(np.uint32), oc.hvs[:, :u].view(np.uint32))
+
+
+SMALL = [CONFIGS["C0"], CONFIGS["C0w3"], small_config(),
+         small_config(window=0, prior_frames=(2, 1, 3), head_dim=64, heads=3),
+         small_config(window=3, prior_frames=(5, 1, 4), tokens_per_frame=37)]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name + f"_w{c.window_frames}_d{c.head_dim}")
+def test_append_bit_exact_after_every_segment(cfg):
+    from int8_kv_cache_action_b200.runtime import KVCache
+    from oracle.ring import OracleCache
+    inp = make_inputs(cfg)
+    gc = KVCache.for_config(cfg)
+    oc = OracleCache(cfg.heads, cfg.head_dim, cfg.tokens_per_frame, cfg.window_frames, cfg.capacity_frames,
+                     cfg.head_store_tokens)
+    for seg, kv in zip(cfg.prior, inp.prior):
+        gc.append(kv.k.cuda(), kv.v.cuda(), seg.n_frames,
+                  None if kv.head_k is None else kv.head_k.cuda(), None if kv.head_v is None else kv.head_v.cuda())
+        oc.append(f32(kv.k), f32(kv.v), seg.n_frames, f32(kv.head_k), f32(kv.head_v))
+        _compare_cache(gc, oc)
+    # and the current segment, as the step after its generation would append it
+    if cfg.window_frames or oc.frames_appended + cfg.current.n_frames <= cfg.capacity_frames:
+        hl = cfg.current.head_len
+        if oc.head_used + hl <= cfg.head_store_tokens:
+            hk, hv = inp.k_txt[:hl], inp.v_txt[:hl]
+            gc.append(inp.k_cur.cuda(), inp.v_cur.cuda(), cfg.current.n_frames,
+                      hk.cuda() if hl else None, hv.cuda() if hl else None)
+            oc.append(f32(inp.k_cur), f32(inp.v_cur), cfg.current.n_frames, f32(hk) if hl else None,
+                      f32(hv) if hl else None)
+            _compare_cache(gc, oc)
+    assert gc.status() == 0
+
+
+@pytest.mark.parametrize("name", ["C1", "C2", "C4"])
+def test_append_full_size(name):
+    cfg = CONFIGS[name]
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    oc = oracle_cache(cfg, inp)
+    _compare_cache(gc, oc)
+    assert gc.status() == 0
+
+
+def test_strided_head_major_input_and_dequant():
+    cfg = small_config(window=4, prior_frames=(3, 3))
+    inp = make_inputs(cfg)
+    from int8_kv_cache_action_b200.runtime import KVCache
+    gc = KVCache.for_config(cfg)
+    for seg, kv in zip(cfg.prior, inp.prior):
+        # [H, S, D] storage viewed as [S, H, D]: token stride D, head stride S*D
+        k = kv.k.transpose(0, 1).contiguous().cuda().transpose(0, 1)
+        v = kv.v.transpose(0, 1).contiguous().cuda().transpose(0, 1)
+        hk = kv.head_k.transpose(0, 1).contiguous().cuda().transpose(0, 1)
+        hv = kv.head_v.transpose(0, 1).contiguous().cuda().transpose(0, 1)
+        gc.append(k, v, seg.n_frames, hk, hv)
+    oc = oracle_cache(cfg, inp)
+    _compare_cache(gc, oc)
+    kd, vd = gc.dequant()
+    hk8, hks, hv8, hvs = oc.history()
+    want_k = (hk8.astype(np.float32) * hks[..., None]).transpose(1, 0, 2)
+    want_v = (hv8.astype(np.float32) * hvs[..., None]).transpose(1, 0, 2)
+    assert np.array_equal(kd.cpu().numpy(), want_k) and np.array_equal(vd.cpu().numpy(), want_v)
+
+
+def test_capacity_and_argument_errors_leave_cache_unchanged():
+    from int8_kv_cache_action_b200 import _nomas as N
+    from int8_kv_cache_action_b200.runtime import KVCache
+    gc = KVCache(2, 128, 10, 0, 3, 8)
+    k = torch.randn(20, 2, 128, device="cuda").bfloat16()
+    gc.append(k, k, 2)
+    with pytest.raises(N.NomasError) as e:
+        gc.append(k, k, 2)
+    assert e.value.status == N.NOMAS_ECAPACITY
+    h = torch.randn(9, 2, 128, device="cuda").bfloat16()
+    with pytest.raises(N.NomasError) as e:
+        gc.append(k[:10], k[:10], 1, h, h)
+    assert e.value.status == N.NOMAS_ECAPACITY
+    rc = N.nomas_kv_append(gc.handle, k.data_ptr() + 2, k.data_ptr(), 256, 128, 1, 0, 0, 0)
+    assert rc == N.NOMAS_EINVAL
+    st = gc.state()
+    assert st["frames_appended"] == 2 and st["head_tokens"] == 0 and st["segments"] == 1

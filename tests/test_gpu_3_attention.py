@@ -1,0 +1,139 @@
+"""GPU parity of nomas_attn_fwd against the fp64 oracle: max-abs 1e-2 and mean-relative 2e-3 on the
+output, plus invariants the visibility rule implies (masked keys contribute exactly nothing)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from int8_kv_cache_action_b200.workloads import CONFIGS, make_inputs, small_config
+from tests.helpers import (TOL_MAX_ABS, TOL_MEAN_REL, attention_errors, f32, gpu_cache, oracle_cache,
+                           sample_rows, to_device)
+
+pytestmark = pytest.mark.gpu
+
+LSE_TOL = 2e-3
+
+
+def _run(cfg, inp, gc, mode=0, keep=None):
+    from int8_kv_cache_action_b200.runtime import segment_text_of
+    seg = segment_text_of(cfg.current)
+    d = to_device(inp)
+    keep = cfg.keep_frac if keep is None else keep
+    buf, lay = gc.build_mask(seg, mode, keep, d["q"], d["k_cur"])
+    out, lse = gc.attention(seg, buf, d["q"], d["k_cur"], d["v_cur"], d["k_txt"], d["v_txt"],
+                            mode=mode, keep_frac=keep, want_lse=True)
+    torch.cuda.synchronize()
+    return out, lse, buf, lay
+
+
+def _oracle(cfg, inp, oc, rows, mode=0, keep=None):
+    from oracle import attention as att
+    from oracle import select as sel
+    s = None
+    if mode:
+        hk8, hks, _, _ = oc.history()
+        s, _ = sel.select(f32(inp.q), hk8, hks, f32(inp.k_cur), cfg.keep_frac if keep is None else keep)
+    return att.attention(oc, f32(inp.q), f32(inp.k_cur), f32(inp.v_cur), f32(inp.k_txt), f32(inp.v_txt),
+                         cfg.current, 1.0 / math.sqrt(cfg.head_dim), rows=rows, sel=s)
+
+
+def _check(cfg, mode=0, rows=None, keep=None):
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    oc = oracle_cache(cfg, inp)
+    out, lse, _, _ = _run(cfg, inp, gc, mode, keep)
+    assert gc.status() == 0
+    rows = np.arange(cfg.n_query) if rows is None else rows
+    ref, ref_lse = _oracle(cfg, inp, oc, rows, mode, keep)
+    got = out.cpu().numpy()[rows]
+    mx, mr = attention_errors(got, ref)
+    assert np.isfinite(got).all()
+    assert mx <= TOL_MAX_ABS and mr <= TOL_MEAN_REL, (mx, mr)
+    gl = lse.cpu().numpy()[:, rows]
+    assert np.abs(gl - ref_lse).max() <= LSE_TOL
+    return mx, mr
+
+
+SMALL_DENSE = [
+    CONFIGS["C0"], CONFIGS["C0w3"],
+    small_config(),                                                    # 2 heads x 128, ragged everywhere
+    small_config(heads=3, head_dim=64, tokens_per_frame=57, n_frames=4, window=3, prior_frames=(2, 2, 2)),
+    small_config(tokens_per_frame=33, n_frames=7, window=0, prior_frames=(2, 5), tails=()),   # no text tails
+    small_config(tokens_per_frame=70, n_frames=5, tails=((64, 0, 1), (100, 1, 4), (5, 4, 5), (130, 2, 3))),
+    small_config(prior_frames=(), prior_head=0, head_len=0, tails=(), window=0, n_frames=2),   # no history, no text
+    small_config(tokens_per_frame=128, n_frames=2, prior_frames=(1,), tails=((128, 0, 1), (128, 1, 2))),  # aligned
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL_DENSE, ids=lambda c: f"{c.name}_d{c.head_dim}_T{c.tokens_per_frame}_F{c.current.n_frames}")
+def test_dense_small_all_rows(cfg):
+    _check(cfg)
+
+
+SMALL_SPARSE = [small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), window=4),
+                small_config(tokens_per_frame=97, n_frames=5, prior_frames=(4, 4), window=5, head_dim=64)]
+
+
+@pytest.mark.parametrize("cfg", SMALL_SPARSE, ids=lambda c: f"{c.name}_d{c.head_dim}_T{c.tokens_per_frame}")
+def test_sparse_small_all_rows(cfg):
+    _check(cfg, mode=1)
+
+
+def test_sparse_full_keep_equals_dense_bitwise():
+    cfg = small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), window=4)
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    dense, dl, _, _ = _run(cfg, inp, gc, 0)
+    full, fl, _, _ = _run(cfg, inp, gc, 1, keep=1.0)
+    assert torch.equal(dense, full) and torch.equal(dl, fl)
+
+
+def test_masked_tail_keys_contribute_exactly_nothing():
+    # rows outside a tail's window must not change at all when that tail's K/V change
+    cfg = small_config(tokens_per_frame=70, n_frames=5, tails=((64, 0, 1), (100, 1, 4), (5, 4, 5), (130, 2, 3)))
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    base, _, _, _ = _run(cfg, inp, gc)
+    a0 = cfg.current.head_len + 64          # tail 1 covers frames [1, 4)
+    inp.k_txt[a0:a0 + 100] *= -3
+    inp.v_txt[a0:a0 + 100] += 5
+    pert, _, _, _ = _run(cfg, inp, gc)
+    frames = torch.arange(cfg.n_query, device="cuda") // cfg.tokens_per_frame
+    outside = (frames < 1) | (frames >= 4)
+    assert torch.equal(base[outside], pert[outside])
+    assert (base[~outside] - pert[~outside]).abs().max() > 1e-3
+
+
+def test_deterministic():
+    cfg = small_config()
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    a, la, _, _ = _run(cfg, inp, gc)
+    b, lb, _, _ = _run(cfg, inp, gc)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_stale_mask_is_reported():
+    from int8_kv_cache_action_b200 import _nomas as N
+    from int8_kv_cache_action_b200.runtime import segment_text_of
+    cfg = small_config()
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    d = to_device(inp)
+    seg = segment_text_of(cfg.current)
+    buf, _ = gc.build_mask(seg)
+    gc.append(d["k_cur"][:cfg.tokens_per_frame], d["v_cur"][:cfg.tokens_per_frame], 1)
+    gc.attention(seg, buf, d["q"], d["k_cur"], d["v_cur"], d["k_txt"], d["v_txt"])
+    assert gc.status() == N.NOMAS_EDEVICE
+    assert gc.status() == 0   # the error word is cleared by the read
+
+
+@pytest.mark.parametrize("name,mode,n_random", [("C1", 0, 300), ("C3r", 1, 300), ("C2", 0, 120), ("C3", 1, 120),
+                                                ("C4", 0, 40)])
+def test_full_size_sampled_rows(name, mode, n_random):
+    cfg = CONFIGS[name]
+    rows = sample_rows(cfg, n_random=n_random)
+    if name == "C4":
+        rows = rows[::3]
+    _check(cfg, mode=mode, rows=rows)

@@ -1,0 +1,395 @@
+"""Benchmark of the INT8-KV segment-causal attention hot path on B200 (one JSON line on stdout).
+
+One step = one pass of the whole path on the production shape (1280x704 -> 880 tokens per latent
+frame, 30-frame segment, 16 heads x 128, 18-frame INT8 history, 768-token description head + 8 action
+tails of 64):
+  a1  nomas_kv_append   quantise-append the finished previous segment (26400 tokens, 18 frames kept)
+  a2  nomas_mask_build  dense visibility classes and tile lists
+  a4  nomas_attn_fwd    dense masked attention (steps 1-2 of a segment's denoising)
+  a3  nomas_mask_build  sparse selection (25 % of candidate video blocks)
+  a4' nomas_attn_fwd    block-sparse attention (steps 3-8)
+`value` = algorithmic attention FLOPs of the step (visible / selected keys only) / step time, on the
+device, inputs resident in HBM.  Inputs (324 MB of bf16 q/k/v per step) exceed the 126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "C2"
+METRIC = "masked attention TFLOP/s (dense + 25% block-sparse step, INT8 KV history) on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def visible_key_sum(cfg, hist_tokens, head_tokens):
+    """Sum over query rows of visible keys (dense): closed form per latent frame."""
+    T, F = cfg.tokens_per_frame, cfg.current.n_frames
+    base = hist_tokens + head_tokens + cfg.n_query + cfg.current.head_len
+    tot = 0
+    for t in range(F):
+        tot += T * (base + sum(a.len for a in cfg.current.tails if a.f0 <= t < a.f1))
+    return tot
+
+
+def sparse_key_sum(sel, cfg, hist_tokens, head_tokens):
+    """Sum over heads and query rows of kept keys: kept candidate video blocks of the row's query block
+    (their valid tokens), every earlier description head, and the row's visible current text."""
+    nq, T = cfg.n_query, cfg.tokens_per_frame
+    nh = (hist_tokens + 127) // 128
+    sel = sel.cpu().numpy()
+    H, nqb, keep = sel.shape
+    def cand_len(c):
+        if c < nh:
+            return min(128, hist_tokens - 128 * c)
+        c -= nh
+        return min(128, nq - 128 * c)
+    lens = {}
+    tot = 0
+    for b in range(nqb):
+        rows = range(128 * b, min(128 * b + 128, nq))
+        text = sum(cfg.current.head_len + sum(a.len for a in cfg.current.tails if a.f0 <= r // T < a.f1)
+                   for r in rows)
+        for h in range(H):
+            vid = 0
+            for c in sel[h, b]:
+                c = int(c)
+                if c not in lens:
+                    lens[c] = cand_len(c)
+                vid += lens[c]
+            tot += len(rows) * (vid + head_tokens) + text
+    return tot
+
+
+class Clock:
+    """Samples nvidia-smi clocks / throttle reasons in the background during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from int8_kv_cache_action_b200 import _nomas as N
+    from int8_kv_cache_action_b200.runtime import KVCache, mask_views, segment_text_of
+    from int8_kv_cache_action_b200.workloads import CONFIGS, make_inputs, APPEND_BYTES_PER_TOKEN_HEAD
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = CONFIGS[WORKLOAD]
+    inp = make_inputs(cfg, seed_offset=rank)
+    q, kc, vc, kt, vt = (getattr(inp, n).to(dev) for n in ("q", "k_cur", "v_cur", "k_txt", "v_txt"))
+    prev = inp.prior[-1]
+    pk, pv = prev.k.to(dev), prev.v.to(dev)
+    cache = KVCache.for_config(cfg, dev)
+    for seg, kv in zip(cfg.prior, inp.prior):
+        cache.append(kv.k.to(dev), kv.v.to(dev), seg.n_frames)
+    seg = segment_text_of(cfg.current)
+    st = torch.cuda.current_stream()
+    s = st.cuda_stream
+    lay_d = cache.mask_layout(seg, N.NOMAS_MODE_DENSE)
+    lay_s = cache.mask_layout(seg, N.NOMAS_MODE_SPARSE, 0.25)
+    mbuf_d = torch.empty(lay_d["total_bytes"], dtype=torch.uint8, device=dev)
+    mbuf_s = torch.empty(lay_s["total_bytes"], dtype=torch.uint8, device=dev)
+    out_d = torch.empty((cfg.n_query, cfg.heads, cfg.head_dim), dtype=torch.float32, device=dev)
+    out_s = torch.empty_like(out_d)
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    ts, hs = q.stride(0), q.stride(1)
+    n_frames_prev = cfg.prior[-1].n_frames
+
+    def check(rc, what):
+        if rc != 0:
+            raise N.NomasError(rc, what)
+
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+
+    def step(record=None):
+        if record is not None:
+            ev[0].record(st)
+        check(N.nomas_kv_append(cache.handle, pk.data_ptr(), pv.data_ptr(), pk.stride(0), pk.stride(1),
+                                n_frames_prev, 0, 0, 0, s), "append")
+        if record is not None:
+            ev[1].record(st)
+        check(N.nomas_mask_build(cache.handle, seg, 0, 0.25, 0, 0, ts, hs, mbuf_d.data_ptr(), s), "mask dense")
+        if record is not None:
+            ev[2].record(st)
+        check(N.nomas_attn_fwd(cache.handle, seg, 0, 0.25, mbuf_d.data_ptr(), q.data_ptr(), kc.data_ptr(),
+                               vc.data_ptr(), kt.data_ptr(), vt.data_ptr(), ts, hs, scale, out_d.data_ptr(), 0, s),
+              "attn dense")
+        if record is not None:
+            ev[3].record(st)
+        check(N.nomas_mask_build(cache.handle, seg, 1, 0.25, q.data_ptr(), kc.data_ptr(), ts, hs,
+                                 mbuf_s.data_ptr(), s), "mask sparse")
+        if record is not None:
+            ev[4].record(st)
+        check(N.nomas_attn_fwd(cache.handle, seg, 1, 0.25, mbuf_s.data_ptr(), q.data_ptr(), kc.data_ptr(),
+                               vc.data_ptr(), kt.data_ptr(), vt.data_ptr(), ts, hs, scale, out_s.data_ptr(), 0, s),
+              "attn sparse")
+        if record is not None:
+            ev[5].record(st)
+            torch.cuda.synchronize()
+            for i in range(5):
+                record[i].append(ev[i].elapsed_time(ev[i + 1]))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if cache.status() != 0:
+        raise RuntimeError("device error during warm-up")
+    st_now = cache.state()
+    flops_dense = 4.0 * cfg.head_dim * cfg.heads * visible_key_sum(cfg, st_now["history_tokens"], st_now["head_tokens"])
+    mv = mask_views(mbuf_s, lay_s)
+    flops_sparse = 4.0 * cfg.head_dim * sparse_key_sum(mv["sel"], cfg, st_now["history_tokens"],
+                                                       st_now["head_tokens"])
+    append_bytes = (cfg.window_frames * cfg.tokens_per_frame) * cfg.heads * APPEND_BYTES_PER_TOKEN_HEAD(cfg.head_dim)
+
+    # timed region: K steps back to back, events on the launching stream
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with Clock(local_rank) as clk:
+        t0.record(st)
+        for _ in range(args.steps):
+            step()
+        t1.record(st)
+        torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        tm = torch.tensor([ms], device=dev)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ms = float(tm.item())
+    if cache.status() != 0:
+        raise RuntimeError("device error in the timed region")
+    # per-phase breakdown (separate pass with events between the phases)
+    rec = [[] for _ in range(5)]
+    for _ in range(max(3, min(args.steps, 10))):
+        step(rec)
+    ph = [statistics.mean(r) for r in rec]
+
+    # end to end: pinned host inputs -> device, the same C-ABI calls, device -> host of the outputs
+    e2e = None
+    if rank == 0 or world > 1:
+        host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("kc", kc), ("vc", vc), ("kt", kt), ("vt", vt),
+                                                     ("pk", pk), ("pv", pv))}
+        hout = torch.empty(out_d.shape, dtype=torch.float32).pin_memory()
+        hout2 = torch.empty(out_s.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = 2 * hout.numel() * 4
+        dst = {"q": q, "kc": kc, "vc": vc, "kt": kt, "vt": vt, "pk": pk, "pv": pv}
+        n_e2e = max(2, min(args.steps, 5))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(st)
+        for _ in range(n_e2e):
+            for n, t in host.items():
+                dst[n].copy_(t, non_blocking=True)
+            step()
+            hout.copy_(out_d, non_blocking=True)
+            hout2.copy_(out_s, non_blocking=True)
+        e1.record(st)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1) / n_e2e
+        e2e = {"value": (flops_dense + flops_sparse) / (ems * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+    return dict(ms=ms, phases=ph, flops_dense=flops_dense, flops_sparse=flops_sparse, append_bytes=append_bytes,
+                clocks=clk.summary(), e2e=e2e, cfg=cfg)
+
+
+def cpu_oracle_sample(seconds_budget=15.0, rows_per_head_start=16):
+    """Time the CPU oracle (as it stands) on a bounded sample of the same workload's dense attention."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from int8_kv_cache_action_b200.workloads import CONFIGS, make_inputs
+    from oracle import attention as att
+    from oracle.ring import OracleCache
+
+    cfg = CONFIGS[WORKLOAD]
+    inp = make_inputs(cfg)
+    f = lambda t: t.float().numpy()
+    oc = OracleCache(cfg.heads, cfg.head_dim, cfg.tokens_per_frame, cfg.window_frames, cfg.capacity_frames,
+                     cfg.head_store_tokens)
+    for seg, kv in zip(cfg.prior, inp.prior):
+        oc.append(f(kv.k), f(kv.v), seg.n_frames)
+    qf, kcf, vcf, ktf, vtf = f(inp.q), f(inp.k_cur), f(inp.v_cur), f(inp.k_txt), f(inp.v_txt)
+    rng = np.random.default_rng(0)
+    n = rows_per_head_start
+    while True:
+        rows = np.sort(rng.choice(cfg.n_query, n, replace=False))
+        t0 = time.perf_counter()
+        att.attention(oc, qf, kcf, vcf, ktf, vtf, cfg.current, 1.0 / math.sqrt(cfg.head_dim), rows=rows)
+        dt = time.perf_counter() - t0
+        if dt > seconds_budget / 4 or n >= cfg.n_query:
+            break
+        n = min(cfg.n_query, n * 4)
+    vis = 15840 + 26400 + 768
+    T = cfg.tokens_per_frame
+    flops = 0.0
+    for r in rows:
+        t = r // T
+        flops += 4.0 * cfg.head_dim * cfg.heads * (vis + sum(a.len for a in cfg.current.tails if a.f0 <= t < a.f1))
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"dense attention of {len(rows)} random query rows x 16 heads of the production shape "
+                      f"(fp64 numpy oracle, {dt:.1f} s)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    pk, pk_kind = peaks()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        vals = []
+        for i in range(args.warmup + args.steps):
+            r = cpu_oracle_sample(seconds_budget=6.0)
+            if i >= args.warmup:
+                vals.append(r)
+        v = statistics.mean(x["value"] for x in vals)
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": "production_1280x704 dense attention (sampled rows)"},
+                "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": vals[0]["cores"], "kind": "oracle",
+                                 "sample": vals[0]["sample"]},
+                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = cpu_oracle_sample()
+    r = run_ours(args, rank, world, local_rank)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    cfg = r["cfg"]
+    ms_step = r["ms"] / args.steps
+    flops = r["flops_dense"] + r["flops_sparse"]
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    ph = r["phases"]
+    dense_tflops = r["flops_dense"] / (ph[2] * 1e-3) / 1e12
+    sparse_tflops = r["flops_sparse"] / (ph[4] * 1e-3) / 1e12
+    append_gbs = r["append_bytes"] / (ph[0] * 1e-3) / 1e9
+    peak_t = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "attn_dense_production_traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            traffic = json.load(f).get("bytes_per_launch")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "production_1280x704: 16x128, 30-frame segment (26400 queries), 18-frame INT8 "
+                               "history (15840 keys), 768 head + 8 tails x 64; step = append + dense mask + "
+                               "dense attention + sparse selection (25%) + sparse attention",
+                   "seq_len": cfg.n_query, "heads": cfg.heads, "head_dim": cfg.head_dim,
+                   "l2": "inputs larger than L2 (324 MB bf16 q/k/v per step)", "parallelism": f"replica x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128> dense", "achieved": dense_tflops,
+                     "peak": peak_t, "unit": "TFLOP/s", "frac": dense_tflops / peak_t,
+                     "peak_kind": f"bf16 dense, sustained ({pk_kind})", "frac_of_burst": dense_tflops / peak_burst,
+                     "traffic": traffic},
+        "roofline_append": {"bound": "hbm", "kernel": "quant_append_kernel<128>", "achieved": append_gbs,
+                            "peak": hbm, "unit": "GB/s", "frac": append_gbs / hbm, "traffic": None},
+        "breakdown_ms": {"append": ph[0], "mask_dense": ph[1], "attn_dense": ph[2], "mask_sparse": ph[3],
+                         "attn_sparse": ph[4]},
+        "attn_dense_tflops": dense_tflops, "attn_sparse_tflops": sparse_tflops,
+        "flops_per_step": {"dense": r["flops_dense"], "sparse": r["flops_sparse"]},
+        "kv_tokens_per_s_append": (cfg.window_frames * cfg.tokens_per_frame) * cfg.heads / (ph[0] * 1e-3),
+        "cpu_baseline": cpu_base,
+        "e2e": r["e2e"],
+        "gpu_launches": 13 * args.steps,
+        "clocks": r["clocks"],
+    }
+    print(json.dumps(line))
+
+
+if __name__ == "__main__":
+    main()

@@ -195,8 +195,9 @@ int nomas_mask_build(const nomas_kv_cache *cache, const nomas_segment_text *seg,
  * segment's video (bf16) and its text (bf16), with the visibility of
  * nomas_mask_build.  Per head h and query row i:
  *     O[i,h] = sum_j softmax_j(softmax_scale * q_i . k^_j) v^_j   over visible j
- * with k^ = code * scale for cached keys (exactly; the key scale is applied to
- * the fp32 score) and v^ = bf16(code * scale) for cached values.
+ * with k^ = code * scale for cached keys (exactly: bf16 codes in the QK^T product,
+ * the key scale applied to the fp32 score) and v^ = fp16(code * scale) for cached
+ * values; the P V product runs in fp16 with fp32 accumulation.
  *   q, kcur, vcur  bf16 [n_frames*T][H][D];  ktxt, vtxt bf16 [text_tokens][H][D]
  *                  (NULL allowed when the segment has no text)
  *   out            fp32 [n_frames*T][H][D], contiguous
@@ -216,6 +217,10 @@ int nomas_kv_dequant(const nomas_kv_cache *cache, float *k_out, float *v_out, no
 int nomas_device_status(const nomas_kv_cache *cache, nomas_stream stream);
 
 const char *nomas_status_string(int status);
+
+/* Diagnostic text of the last NOMAS_ECUDA returned on the calling thread: the CUDA call that
+ * failed and its error string ("" if none).  Valid until the next failing call on this thread. */
+const char *nomas_last_error(void);
 
 #ifdef __cplusplus
 }

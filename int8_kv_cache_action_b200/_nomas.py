@@ -24,7 +24,8 @@ NOMAS_MAX_TAILS = 64
 
 EXPORTED = ["nomas_kv_cache_bytes", "nomas_kv_cache_init", "nomas_kv_cache_destroy", "nomas_kv_cache_state",
             "nomas_kv_append", "nomas_mask_layout_query", "nomas_mask_bytes", "nomas_mask_build",
-            "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string"]
+            "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string",
+            "nomas_last_error"]
 
 
 class nomas_cache_dims(ctypes.Structure):
@@ -76,6 +77,7 @@ _sigs = {
     "nomas_kv_dequant": (ctypes.c_int, [_p, _p, _p, _p]),
     "nomas_device_status": (ctypes.c_int, [_p, _p]),
     "nomas_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "nomas_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(lib, _name)
@@ -86,7 +88,8 @@ for _name, (_res, _args) in _sigs.items():
 class NomasError(RuntimeError):
     def __init__(self, status: int, what: str = ""):
         self.status = status
-        super().__init__(f"{what}: {nomas_status_string(status)} ({status})")
+        extra = f" [{nomas_last_error()}]" if status == NOMAS_ECUDA else ""
+        super().__init__(f"{what}: {nomas_status_string(status)} ({status}){extra}")
 
 
 def _check(rc: int, what: str) -> None:
@@ -96,6 +99,10 @@ def _check(rc: int, what: str) -> None:
 
 def nomas_status_string(status: int) -> str:
     return lib.nomas_status_string(status).decode()
+
+
+def nomas_last_error() -> str:
+    return lib.nomas_last_error().decode()
 
 
 def make_dims(heads, head_dim, tokens_per_frame, window_frames, capacity_frames, head_store_tokens):

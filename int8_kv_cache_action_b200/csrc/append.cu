@@ -163,7 +163,7 @@ static int launch_append(const AppendArgs &a, int D, cudaStream_t st) {
     if (blocks > 148 * 32) blocks = 148 * 32;
     if (D == 128) quant_append_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(a);
     else quant_append_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(a);
-    return cudaGetLastError() == cudaSuccess ? NOMAS_OK : NOMAS_ECUDA;
+    return check_launch("quant_append_kernel launch");
 }
 
 }  // namespace nomas
@@ -257,5 +257,5 @@ extern "C" int nomas_kv_dequant(const nomas_kv_cache *c, float *k_out, float *v_
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (c->d.head_dim == 128) dequant_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(a);
     else dequant_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(a);
-    return cudaGetLastError() == cudaSuccess ? NOMAS_OK : NOMAS_ECUDA;
+    return check_launch("dequant_kernel launch");
 }

@@ -4,12 +4,18 @@
 // One CTA = one head x two 128-row query tiles (Q0, Q1) that share every K/V tile of their list.
 //   warps 0-3   softmax for Q0   (TMEM lanes 0-127 of S0 / O0; one thread per query row)
 //   warps 4-7   softmax for Q1
-//   warps 8-11  loader: TMA for bf16 tiles; INT8 -> BF16 conversion into the same 128B-swizzled
-//               layout for cached tiles (keys exact, values times their scale); per-column key
-//               scale and visibility window for the softmax
-//   warp 12     tcgen05.mma issuer (one thread) and TMEM owner
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D); P_q (bf16) overwrites
+//   warps 8-11  loader: TMA for bf16 key tiles; INT8 keys -> bf16 codes and INT8 values x scale ->
+//               fp16, bf16 values -> fp16, all written in the 128B-swizzled UMMA layout;
+//               per-column key scale and visibility window for the softmax
+//   warp 12     tcgen05.mma issuer (one thread) and TMEM owner; warps 13-15 idle
+// The register file is split per SM sub-partition (one warp of each warpgroup on each), so the
+// kernel launches at 128 registers per thread and moves them with setmaxnreg: softmax 168 each,
+// loader 112, MMA warpgroup 64 -- 2*168 + 112 + 64 = 512 = 4 x 128, the launch's own total.
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D); P_q (fp16) overwrites
 // the first 64 columns of S_q and feeds the PV MMA as its A operand.
+// Precision: Q K^T runs in bf16 with the INT8 key codes exact and the key scale applied to the fp32
+// score; P V runs in fp16 (P <= 2^8 and the values fit its range), which keeps 3 more significand
+// bits than bf16 for the weights and the dequantised values (fp32 accumulation in both).
 // Per KV tile j the MMA thread issues S_q = Q_q K_j^T when K_j has landed and PV_q(j-1) has been
 // issued, and O_q += P_q V_j when softmax q has published P_q; both query tiles are interleaved so
 // that the tensor core works on one tile while the other tile's softmax runs.
@@ -18,12 +24,17 @@
 // S_q(j) implies completion of every earlier MMA of this thread (tcgen05.commit tracks all prior
 // operations), so O_q is idle whenever softmax q holds a fresh S_q.
 #include <cmath>
+#include <cstdio>
+
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
 namespace nomas {
 
-constexpr int kAttnThreads = 416;
+constexpr int kAttnThreads = 512;
+constexpr int kRegSoftmax = 168, kRegLoader = 112, kRegMma = 64;
+static_assert(2 * kRegSoftmax + kRegLoader + kRegMma == 4 * 128, "register split must equal the launch total");
 constexpr int kNCI = 4;                     // column-info ring depth
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
@@ -52,6 +63,9 @@ struct AttnParams {
     const int8_t *hk8, *hv8;
     const float *hks, *hvs;
     int64_t ring_tokens, first_tok, head_rows;
+    // current-segment and text values (bf16), staged to fp16 by the loader
+    const __nv_bfloat16 *vcur, *vtxt;
+    int64_t tok_stride, head_stride;
     // mask buffer
     const uint8_t *mask;
     const int4 *lists;
@@ -76,6 +90,15 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -88,28 +111,50 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// 8 bf16 (16 bytes) from 8 int8, optionally times a scale; returned as 4 packed words.
-__device__ __forceinline__ uint4 cvt8(uint32_t lo, uint32_t hi, float s, bool scaled) {
-    uint32_t w[2] = {lo, hi};
+// 8 int8 codes -> 8 bf16 (exact: |code| <= 127), packed in 16 bytes.
+__device__ __forceinline__ uint4 cvt_i8x8_bf16(uint32_t lo, uint32_t hi) {
+    const uint32_t w[2] = {lo, hi};
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t src = w[i >> 1];
         const int sh = (i & 1) * 16;
-        float a = (float)(int8_t)((src >> sh) & 0xFF);
-        float b = (float)(int8_t)((src >> (sh + 8)) & 0xFF);
-        if (scaled) {
-            a *= s;
-            b *= s;
-        }
-        __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
+        __nv_bfloat162 pr = __floats2bfloat162_rn((float)(int8_t)((src >> sh) & 0xFF),
+                                                  (float)(int8_t)((src >> (sh + 8)) & 0xFF));
+        o[i] = *reinterpret_cast<uint32_t *>(&pr);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// 8 int8 codes times their row scale -> 8 fp16 (round to nearest), packed in 16 bytes.
+__device__ __forceinline__ uint4 cvt_i8x8_f16(uint32_t lo, uint32_t hi, float s) {
+    const uint32_t w[2] = {lo, hi};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t src = w[i >> 1];
+        const int sh = (i & 1) * 16;
+        __half2 pr = __floats2half2_rn((float)(int8_t)((src >> sh) & 0xFF) * s,
+                                       (float)(int8_t)((src >> (sh + 8)) & 0xFF) * s);
+        o[i] = *reinterpret_cast<uint32_t *>(&pr);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// 8 bf16 -> 8 fp16 (exact for |x| >= 2^-14; below that fp16 keeps 2^-24 absolute resolution).
+__device__ __forceinline__ uint4 cvt_bf16x8_f16(const uint4 &v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __half2 pr = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
         o[i] = *reinterpret_cast<uint32_t *>(&pr);
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 template <int D>
-__global__ void __maxnreg__(152)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
                     const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kt,
                     const __grid_constant__ CUtensorMap tm_vt, const AttnParams p) {
@@ -169,6 +214,7 @@ __global__ void __maxnreg__(152)
             mbar_init(&o_final[q], 1);
         }
         misc[1] = 0;
+        for (int i = 0; i < C::NS; ++i) misc[8 + i] = 0;
         fence_mbar_init();
     }
     if (warp == 12) {
@@ -185,6 +231,7 @@ __global__ void __maxnreg__(152)
 
     if (warp >= 8 && warp < 12) {
         // ------------------------------------------------------------------ loader warpgroup
+        setmaxnreg_dec<kRegLoader>();
         // Every wait is followed by a named barrier over the 128 loader threads and a read of the
         // shared abort flag, so all loader threads leave the loop together.
         wd.where = 3;
@@ -193,7 +240,6 @@ __global__ void __maxnreg__(152)
         if (t == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_kc);
-            prefetch_tmap(&tm_vc);
             mbar_arrive_expect_tx(bar_q, 2 * C::QB);
 #pragma unroll
             for (int q = 0; q < 2; ++q)
@@ -203,12 +249,18 @@ __global__ void __maxnreg__(152)
                                 (int)(qrow0 + q * kTile));
         }
         constexpr int CPR = D / 16;          // 16-byte int8 chunks per row
-        constexpr int RSTEP = 128 / CPR;     // rows covered by the 128 threads in one pass
-        constexpr int NR = 128 / RSTEP;      // rows per thread
+        constexpr int RSTEP = 128 / CPR;     // int8 rows covered by the 128 threads in one pass
+        constexpr int NR = 128 / RSTEP;      // int8 rows per thread
+        constexpr int CPRB = D / 8;          // 16-byte bf16 chunks per row
+        constexpr int RSTEPB = 128 / CPRB;
+        constexpr int NRB = 128 / RSTEPB;    // bf16 rows per thread
+        constexpr int NRAW = (2 * NR > NRB) ? 2 * NR : NRB;
         const int my_chunk = t % CPR;
         const int my_row0 = t / CPR;
         const int hh_mine = my_chunk / 4;
         const int c0_mine = (my_chunk % 4) * 2;
+        const int my_chunkb = t % CPRB;
+        const int my_row0b = t / CPRB;
         for (int j = 0; j < n_tiles; ++j) {
             const int4 e = list[j];
             const int kind = e.x & 3;
@@ -225,19 +277,32 @@ __global__ void __maxnreg__(152)
                 const int64_t a = start + r;
                 return head_base + (hist ? (p.first_tok + a) % p.ring_tokens : a);
             };
-            // raw INT8 loads of K and V issued first so their latency overlaps the slot waits
-            uint4 rk[NR], rv[NR];
+            // raw loads issued first so their latency overlaps the slot waits:
+            //   cached tile: raw[0, NR) = K codes, raw[NR, 2 NR) = V codes (16 int8 per chunk)
+            //   bf16 tile:   raw[0, NRB) = V values (8 bf16 per chunk); K arrives by TMA
+            uint4 raw[NRAW];
             float svv[NR];
 #pragma unroll
-            for (int i = 0; i < NR; ++i) {
-                const int r = my_row0 + i * RSTEP;
-                rk[i] = rv[i] = make_uint4(0, 0, 0, 0);
-                svv[i] = 0.0f;
-                if (cached && r < count) {
-                    const int64_t gr = cache_row(r);
-                    rk[i] = __ldg(reinterpret_cast<const uint4 *>(src_k + gr * D) + my_chunk);
-                    rv[i] = __ldg(reinterpret_cast<const uint4 *>(src_v + gr * D) + my_chunk);
-                    svv[i] = __ldg(src_vs + gr);
+            for (int i = 0; i < NRAW; ++i) raw[i] = make_uint4(0, 0, 0, 0);
+            if (cached) {
+#pragma unroll
+                for (int i = 0; i < NR; ++i) {
+                    const int r = my_row0 + i * RSTEP;
+                    svv[i] = 0.0f;
+                    if (r < count) {
+                        const int64_t gr = cache_row(r);
+                        raw[i] = __ldg(reinterpret_cast<const uint4 *>(src_k + gr * D) + my_chunk);
+                        raw[NR + i] = __ldg(reinterpret_cast<const uint4 *>(src_v + gr * D) + my_chunk);
+                        svv[i] = __ldg(src_vs + gr);
+                    }
+                }
+            } else {
+                const __nv_bfloat16 *vb = (kind == kKindCur ? p.vcur : p.vtxt) + (int64_t)h * p.head_stride;
+#pragma unroll
+                for (int i = 0; i < NRB; ++i) {
+                    const int r = my_row0b + i * RSTEPB;
+                    if (r < count)
+                        raw[i] = __ldg(reinterpret_cast<const uint4 *>(vb + (start + r) * p.tok_stride) + my_chunkb);
                 }
             }
             float cs = 0.0f;
@@ -271,8 +336,8 @@ __global__ void __maxnreg__(152)
                 for (int i = 0; i < NR; ++i) {
                     const int r = my_row0 + i * RSTEP;
                     uint8_t *base = dK + hh_mine * (kTile * 128);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = cvt8(rk[i].x, rk[i].y, 1.0f, false);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = cvt8(rk[i].z, rk[i].w, 1.0f, false);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = cvt_i8x8_bf16(raw[i].x, raw[i].y);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = cvt_i8x8_bf16(raw[i].z, raw[i].w);
                 }
                 fence_proxy_async_smem();
                 tma_pending &= ~(1u << sk);
@@ -285,30 +350,28 @@ __global__ void __maxnreg__(152)
             mbar_wait(&kv_empty[sv], (((2 * j + 1) / C::NS) & 1) ^ 1, wd, 3);
             named_bar_sync(1, 128);
             if (*abort_flag) break;
-            uint8_t *dV = sKV + sv * C::SLOT;
-            if (!cached) {
-                if (t == 0) {
-                    const CUtensorMap *m = kind == kKindCur ? &tm_vc : &tm_vt;
-                    mbar_arrive_expect_tx(&kv_full[sv], C::SLOT);
-#pragma unroll
-                    for (int hh = 0; hh < C::HALVES; ++hh)
-                        tma_load_3d(dV + hh * (kTile * 128), m, &kv_full[sv], hh * 64, h, (int)start);
-                    tma_pending |= 1u << sv;
-                    tma_par = (tma_par & ~(1u << sv)) | ((uint32_t)(((2 * j + 1) / C::NS) & 1) << sv);
-                }
-            } else {
+            uint8_t *dV = sKV + sv * C::SLOT;   // V is staged as fp16 (the PV product runs in fp16)
+            if (cached) {
 #pragma unroll
                 for (int i = 0; i < NR; ++i) {
                     const int r = my_row0 + i * RSTEP;
                     uint8_t *base = dV + hh_mine * (kTile * 128);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = cvt8(rv[i].x, rv[i].y, svv[i], true);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = cvt8(rv[i].z, rv[i].w, svv[i], true);
+                    const uint4 &v = raw[NR + i];
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = cvt_i8x8_f16(v.x, v.y, svv[i]);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = cvt_i8x8_f16(v.z, v.w, svv[i]);
                 }
-                fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                tma_pending &= ~(1u << sv);
-                if (t == 0) mbar_arrive(&kv_full[sv]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < NRB; ++i) {
+                    const int r = my_row0b + i * RSTEPB;
+                    uint8_t *base = dV + (my_chunkb / 8) * (kTile * 128);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, my_chunkb % 8)) = cvt_bf16x8_f16(raw[i]);
+                }
             }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            tma_pending &= ~(1u << sv);
+            if (t == 0) mbar_arrive(&kv_full[sv]);
         }
         // on abort, let this CTA's bulk copies land before the shared memory is released
         if (*abort_flag && t == 0) {
@@ -317,12 +380,13 @@ __global__ void __maxnreg__(152)
             for (int i = 0; i < C::NS; ++i)
                 if ((tma_pending >> i) & 1u) mbar_drain(&kv_full[i], (tma_par >> i) & 1u, 100000000ull);
         }
-    } else if (warp == 12) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp >= 12) {
+        // ------------------------------------------------------------------ MMA issuer (warp 12)
+        setmaxnreg_dec<kRegMma>();
         wd.where = 4;
-        if (lane == 0) {
+        if (warp == 12 && lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+            constexpr uint32_t idesc_pv = idesc_f16_f32(128, D, false, true);   // P and V both fp16
             const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
             const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
             const uint32_t q_addr = smem_u32(sQ);
@@ -340,6 +404,10 @@ __global__ void __maxnreg__(152)
             };
             next_s[0] = advance(0, 0);
             next_s[1] = advance(0, 1);
+            // released[s]: how many uses of K/V slot s this thread has released.  A slot is tested
+            // for use u only when uses 0..u-1 are released, so its full barrier can only be at phase
+            // u or u+1 and the parity test cannot mistake an older completion for use u.
+            uint32_t *released = misc + 8;
             uint64_t t0 = globaltimer_ns();
             uint32_t spins = 0;
             while (ok && (next_s[0] < n_tiles || next_s[1] < n_tiles || pend[0] >= 0 || pend[1] >= 0)) {
@@ -349,8 +417,9 @@ __global__ void __maxnreg__(152)
                     if (pend[q] >= 0) {
                         const int j = pend[q];
                         const int sv = (2 * j + 1) % C::NS;
-                        if (mbar_test(&p_full[q], pcount[q] & 1) &&
-                            mbar_test(&kv_full[sv], ((2 * j + 1) / C::NS) & 1)) {
+                        const uint32_t use_v = (uint32_t)((2 * j + 1) / C::NS);
+                        if (released[sv] == use_v && mbar_test(&p_full[q], pcount[q] & 1) &&
+                            mbar_test(&kv_full[sv], use_v & 1)) {
                             tc_fence_after();
                             const uint32_t vb = kv_addr + sv * C::SLOT;
 #pragma unroll
@@ -362,7 +431,10 @@ __global__ void __maxnreg__(152)
                             pcount[q]++;
                             last_pv[q] = j;
                             const int o = 1 - q;
-                            if (!uses(j, o) || last_pv[o] >= j) umma_commit(&kv_empty[sv]);
+                            if (!uses(j, o) || last_pv[o] >= j) {
+                                umma_commit(&kv_empty[sv]);
+                                released[sv] = use_v + 1;
+                            }
                             pend[q] = -1;
                             progress = true;
                         }
@@ -370,7 +442,8 @@ __global__ void __maxnreg__(152)
                     if (pend[q] < 0 && next_s[q] < n_tiles) {
                         const int j = next_s[q];
                         const int sk = (2 * j) % C::NS;
-                        if (mbar_test(&kv_full[sk], ((2 * j) / C::NS) & 1)) {
+                        const uint32_t use_k = (uint32_t)((2 * j) / C::NS);
+                        if (released[sk] == use_k && mbar_test(&kv_full[sk], use_k & 1)) {
                             tc_fence_after();
                             const uint32_t kb = kv_addr + sk * C::SLOT;
                             const uint32_t qb = q_addr + q * C::QB;
@@ -383,7 +456,10 @@ __global__ void __maxnreg__(152)
                             umma_commit(&s_full[q]);
                             last_s[q] = j;
                             const int o = 1 - q;
-                            if (!uses(j, o) || last_s[o] >= j) umma_commit(&kv_empty[sk]);
+                            if (!uses(j, o) || last_s[o] >= j) {
+                                umma_commit(&kv_empty[sk]);
+                                released[sk] = use_k + 1;
+                            }
                             pend[q] = j;
                             next_s[q] = advance(j + 1, q);
                             progress = true;
@@ -412,6 +488,7 @@ __global__ void __maxnreg__(152)
     } else {
         // ------------------------------------------------------------------ softmax warpgroups
         // Waits are made warp-uniform (__all_sync) because tcgen05.ld/st are warp-collective.
+        setmaxnreg_inc<kRegSoftmax>();
         const int q = warp >> 2;
         wd.where = 1 + q;
         const int r = (warp & 3) * 32 + lane;
@@ -472,7 +549,7 @@ __global__ void __maxnreg__(152)
                     const float a = ex2(s[half * 64 + c] - off);
                     const float b = ex2(s[half * 64 + c + 1] - off);
                     sum += a + b;
-                    __nv_bfloat162 pr = __floats2bfloat162_rn(a, b);
+                    __half2 pr = __floats2half2_rn(a, b);
                     pk[c / 2] = *reinterpret_cast<uint32_t *>(&pr);
                 }
                 tmem_st32(tS + half * 32, pk);
@@ -543,10 +620,11 @@ static EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = nullptr;
     if (!fn) {
         void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult qr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
-            qr == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+        cudaDriverEntryPointQueryResult qr = cudaDriverEntryPointSymbolNotFound;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr);
+        if (e == cudaSuccess && qr == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(ptr);
+        else cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", e != cudaSuccess ? (int)e : (int)qr,
+                       e != cudaSuccess ? cudaGetErrorString(e) : "symbol query failed");
     }
     return fn;
 }
@@ -560,9 +638,18 @@ static bool make_map(CUtensorMap *m, const void *base, int64_t n_tok, int H, int
     cuuint64_t strides[2] = {(cuuint64_t)head_stride * 2, (cuuint64_t)tok_stride * 2};
     cuuint32_t box[3] = {64, 1, (cuuint32_t)kTile};
     cuuint32_t es[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char msg[160];
+        std::snprintf(msg, sizeof(msg), "dims %llu x %llu x %llu, strides %llu %llu", (unsigned long long)dims[0],
+                      (unsigned long long)dims[1], (unsigned long long)dims[2], (unsigned long long)strides[0],
+                      (unsigned long long)strides[1]);
+        cuda_fail("cuTensorMapEncodeTiled", (int)r, msg);
+        return false;
+    }
+    return true;
 }
 
 static uint64_t g_timeout_ns = 2000000000ull;   // 2 s per wait
@@ -571,13 +658,13 @@ template <int D>
 static int launch_attn(const AttnParams &p, dim3 grid, const CUtensorMap *maps, cudaStream_t st) {
     static bool attr_set = false;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 AttnCfg<D>::SMEM) != cudaSuccess)
-            return NOMAS_ECUDA;
+        const cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   AttnCfg<D>::SMEM);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(attn smem)", (int)e, cudaGetErrorString(e));
         attr_set = true;
     }
     attn_fwd_kernel<D><<<grid, kAttnThreads, AttnCfg<D>::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
-    return cudaGetLastError() == cudaSuccess ? NOMAS_OK : NOMAS_ECUDA;
+    return check_launch("attn_fwd_kernel launch");
 }
 
 }  // namespace nomas
@@ -624,6 +711,10 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     p.ring_tokens = hv.ring_tokens;
     p.first_tok = hv.first_tok;
     p.head_rows = d.head_store_tokens;
+    p.vcur = static_cast<const __nv_bfloat16 *>(vcur);
+    p.vtxt = static_cast<const __nv_bfloat16 *>(lay.text_tokens > 0 ? vtxt : vcur);
+    p.tok_stride = tok_stride;
+    p.head_stride = head_stride;
     const uint8_t *mb = static_cast<const uint8_t *>(mask_buf);
     p.mask = mb;
     p.lists = reinterpret_cast<const int4 *>(mb + lay.off_list);

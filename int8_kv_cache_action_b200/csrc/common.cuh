@@ -236,6 +236,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B (both operands fp16).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4) | (0u << 7) | (0u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 // Byte offset of the 16-byte chunk `chunk` (0..7) of row `row` inside a 128B-swizzled tile
 // whose rows are 128 bytes (8 rows = one 1024-byte swizzle atom).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {

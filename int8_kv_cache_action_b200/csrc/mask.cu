@@ -349,5 +349,5 @@ extern "C" int nomas_mask_build(const nomas_kv_cache *c, const nomas_segment_tex
         select_kernel<<<p.H * p.n_qb, 256, p.n_cand * sizeof(float), st>>>(p);
         lists_sparse_kernel<<<p.H * ((p.n_qb + 1) / 2), 128, 2 * ((p.n_cand + 31) / 32) * sizeof(uint32_t), st>>>(p);
     }
-    return cudaGetLastError() == cudaSuccess ? NOMAS_OK : NOMAS_ECUDA;
+    return check_launch("mask_build kernels launch");
 }

@@ -1,4 +1,6 @@
 // libnomas host entry points: cache handle, buffer sizes, state, status, mask-buffer layout.
+#include <cmath>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <new>
@@ -9,10 +11,23 @@ namespace nomas {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+static thread_local char g_last_error[256] = "";
+
+int cuda_fail(const char *what, int code, const char *detail) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s failed (%d): %s", what, code, detail ? detail : "");
+    return NOMAS_ECUDA;
+}
+
+int check_launch(const char *what) {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? NOMAS_OK : cuda_fail(what, (int)e, cudaGetErrorString(e));
+}
+
 int bind_device(const nomas_kv_cache *c) {
     int cur = -1;
     if (cudaGetDevice(&cur) == cudaSuccess && cur == c->device) return NOMAS_OK;
-    return cudaSetDevice(c->device) == cudaSuccess ? NOMAS_OK : NOMAS_ECUDA;
+    const cudaError_t e = cudaSetDevice(c->device);
+    return e == cudaSuccess ? NOMAS_OK : cuda_fail("cudaSetDevice", (int)e, cudaGetErrorString(e));
 }
 
 static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -184,6 +199,8 @@ extern "C" int nomas_device_status(const nomas_kv_cache *c, nomas_stream stream)
     }
     return NOMAS_OK;
 }
+
+extern "C" const char *nomas_last_error(void) { return g_last_error; }
 
 extern "C" const char *nomas_status_string(int s) {
     switch (s) {

@@ -64,6 +64,10 @@ int compute_mask_layout(const nomas_kv_cache *c, const nomas_segment_text *seg, 
 
 bool aligned16(const void *p);
 
+// Record a failing CUDA runtime / driver call for nomas_last_error and return NOMAS_ECUDA.
+int cuda_fail(const char *what, int code, const char *detail);
+int check_launch(const char *what);
+
 // Make the cache's device current for this thread (the library links its own CUDA runtime).
 int bind_device(const nomas_kv_cache *c);
 

@@ -78,12 +78,13 @@ def test_strided_head_major_input_and_dequant():
     from int8_kv_cache_action_b200.runtime import KVCache
     gc = KVCache.for_config(cfg)
     for seg, kv in zip(cfg.prior, inp.prior):
-        # [H, S, D] storage viewed as [S, H, D]: token stride D, head stride S*D
-        k = kv.k.transpose(0, 1).contiguous().cuda().transpose(0, 1)
-        v = kv.v.transpose(0, 1).contiguous().cuda().transpose(0, 1)
-        hk = kv.head_k.transpose(0, 1).contiguous().cuda().transpose(0, 1)
-        hv = kv.head_v.transpose(0, 1).contiguous().cuda().transpose(0, 1)
-        gc.append(k, v, seg.n_frames, hk, hv)
+        # [H, S, D] storage viewed as [S, H, D]: token stride D, head stride S*D (one stride pair for all)
+        n, hl = kv.k.shape[0], kv.head_k.shape[0]
+        bufs = torch.zeros(4, cfg.heads, n, cfg.head_dim, dtype=torch.bfloat16)
+        bufs[0], bufs[1] = kv.k.transpose(0, 1), kv.v.transpose(0, 1)
+        bufs[2, :, :hl], bufs[3, :, :hl] = kv.head_k.transpose(0, 1), kv.head_v.transpose(0, 1)
+        g = bufs.cuda().transpose(1, 2)                                   # [4, S, H, D] views
+        gc.append(g[0], g[1], seg.n_frames, g[2][:hl], g[3][:hl])
     oc = oracle_cache(cfg, inp)
     _compare_cache(gc, oc)
     kd, vd = gc.dequant()

@@ -190,6 +190,29 @@ int nomas_mask_build(const nomas_kv_cache *cache, const nomas_segment_text *seg,
                      const void *q, const void *kcur, int64_t tok_stride, int64_t head_stride, void *mask_buf,
                      nomas_stream stream);
 
+/* Allocation-free variant of nomas_mask_build (the pages have no counterpart: this is an interface
+ * convenience of this library).  Some callers cannot allocate device memory on the path that builds
+ * the mask: a host framework that owns the whole device pool and hands plugins no allocator, or a
+ * latency-critical serving loop in which a cudaMalloc could synchronise the device.  In sparse mode
+ * nomas_mask_build keeps the pooled per-block query and key means (scratch) inside the caller's
+ * mask buffer; this variant keeps them in a file-scope device array of NOMAS_STATIC_POOL_FLOATS
+ * floats (8 MiB) that every GPU which loads the library holds until the process exits.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *   Arguments, mask buffer layout and results: as nomas_mask_build (dense mode forwards to it
+ *   unchanged, it needs no scratch).  The qmean / kmean regions of mask_buf are left untouched.
+ *   Limit: heads * (n_qblocks + n_cand) * head_dim <= NOMAS_STATIC_POOL_FLOATS, else
+ *   NOMAS_ECAPACITY before anything is enqueued (1280x704 shape with an 18-frame history:
+ *   1.10 M floats; 480x832: 0.22 M).
+ *   The first call on a device looks up the array's device address (once per device, with that
+ *   device current); make that first call before any stream capture.
+ *   All calls on a device share the one array and it keeps the last call's contents; every element
+ *   a call reads it has written first, so nothing needs clearing.  Calls that overlap on the GPU
+ *   (different streams, no ordering between them) race on the array. */
+#define NOMAS_STATIC_POOL_FLOATS ((size_t)2 << 20)
+int nomas_mask_build_static(const nomas_kv_cache *cache, const nomas_segment_text *seg, int mode,
+                            float keep_frac, const void *q, const void *kcur, int64_t tok_stride,
+                            int64_t head_stride, void *mask_buf, nomas_stream stream);
+
 /* Masked (or block-sparse) attention of the current segment's video queries
  * over the retained INT8 history, earlier description heads (INT8), the current
  * segment's video (bf16) and its text (bf16), with the visibility of

@@ -21,11 +21,12 @@ NOMAS_BUF_K8, NOMAS_BUF_V8, NOMAS_BUF_KS, NOMAS_BUF_VS, NOMAS_BUF_HK8, NOMAS_BUF
     NOMAS_BUF_HVS, NOMAS_BUF_ERR, NOMAS_NBUF = range(10)
 NOMAS_MODE_DENSE, NOMAS_MODE_SPARSE = 0, 1
 NOMAS_MAX_TAILS = 64
+NOMAS_STATIC_POOL_FLOATS = 2 << 20
 
 EXPORTED = ["nomas_kv_cache_bytes", "nomas_kv_cache_init", "nomas_kv_cache_destroy", "nomas_kv_cache_state",
             "nomas_kv_append", "nomas_mask_layout_query", "nomas_mask_bytes", "nomas_mask_build",
             "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string",
-            "nomas_last_error"]
+            "nomas_last_error", "nomas_mask_build_static"]
 
 
 class nomas_cache_dims(ctypes.Structure):
@@ -72,6 +73,8 @@ _sigs = {
     "nomas_mask_bytes": (_sz, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32]),
     "nomas_mask_build": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32, _p, _p,
                                         _i64, _i64, _p, _p]),
+    "nomas_mask_build_static": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32, _p,
+                                               _p, _i64, _i64, _p, _p]),
     "nomas_attn_fwd": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32, _p, _p, _p,
                                       _p, _p, _p, _i64, _i64, _f32, _p, _p, _p]),
     "nomas_kv_dequant": (ctypes.c_int, [_p, _p, _p, _p]),
@@ -159,6 +162,11 @@ def nomas_mask_bytes(handle, seg, mode, keep_frac=0.25):
 def nomas_mask_build(handle, seg, mode, keep_frac, q, kcur, tok_stride, head_stride, mask_buf, stream=0):
     return lib.nomas_mask_build(handle, ctypes.byref(seg), mode, keep_frac, q or None, kcur or None, tok_stride,
                                 head_stride, mask_buf, stream or None)
+
+
+def nomas_mask_build_static(handle, seg, mode, keep_frac, q, kcur, tok_stride, head_stride, mask_buf, stream=0):
+    return lib.nomas_mask_build_static(handle, ctypes.byref(seg), mode, keep_frac, q or None, kcur or None,
+                                       tok_stride, head_stride, mask_buf, stream or None)
 
 
 def nomas_attn_fwd(handle, seg, mode, keep_frac, mask_buf, q, kcur, vcur, ktxt, vtxt, tok_stride, head_stride,

@@ -351,3 +351,170 @@ extern "C" int nomas_mask_build(const nomas_kv_cache *c, const nomas_segment_tex
     }
     return check_launch("mask_build kernels launch");
 }
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free variant of the sparse selection: the pooled query / key means live in a
+// file-scope device array instead of the caller's mask buffer.
+// ------------------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace nomas {
+
+constexpr size_t kStaticPoolFloats = NOMAS_STATIC_POOL_FLOATS;   // 8 MiB of fp32 pooled means per device
+static __device__ __align__(256) float g_pool_scratch[kStaticPoolFloats];
+
+__global__ void qmean_to_kernel(MaskParams p, float *qmean) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t n = (int64_t)p.H * p.n_qb * p.D;
+    if (idx >= n) return;
+    const int c = (int)(idx % p.D);
+    const int64_t hb = idx / p.D;
+    const int b = (int)(hb % p.n_qb);
+    const int h = (int)(hb / p.n_qb);
+    const int64_t r0 = (int64_t)b * kTile;
+    const int nv = (int)((r0 + kTile < p.Nq) ? kTile : p.Nq - r0);
+    float acc = 0.0f;
+    for (int i = 0; i < nv; ++i)
+        acc = __fadd_rn(acc, bf16_at(p.q, (r0 + i) * p.tok_stride + (int64_t)h * p.head_stride + c));
+    qmean[idx] = __fdiv_rn(acc, (float)nv);
+}
+
+__global__ void kmean_to_kernel(MaskParams p, float *kmean) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t n = (int64_t)p.H * p.n_cand * p.D;
+    if (idx >= n) return;
+    const int c = (int)(idx % p.D);
+    const int64_t hc = idx / p.D;
+    const int cand = (int)(hc % p.n_cand);
+    const int h = (int)(hc / p.n_cand);
+    float acc = 0.0f;
+    int nv;
+    if (cand < p.n_hist_tiles) {
+        const int64_t a0 = (int64_t)cand * kTile;
+        nv = (int)((a0 + kTile < p.Lh) ? kTile : p.Lh - a0);
+        for (int i = 0; i < nv; ++i) {
+            const int64_t phys = (p.first_tok + a0 + i) % p.ring_tokens;
+            const int64_t r = (int64_t)h * p.ring_tokens + phys;
+            acc = __fadd_rn(acc, __fmul_rn((float)p.k8[r * p.D + c], p.ks[r]));
+        }
+    } else {
+        const int64_t a0 = (int64_t)(cand - p.n_hist_tiles) * kTile;
+        nv = (int)((a0 + kTile < p.Nq) ? kTile : p.Nq - a0);
+        for (int i = 0; i < nv; ++i)
+            acc = __fadd_rn(acc, bf16_at(p.kcur, (a0 + i) * p.tok_stride + (int64_t)h * p.head_stride + c));
+    }
+    kmean[idx] = __fdiv_rn(acc, (float)nv);
+}
+
+__global__ void score_from_kernel(MaskParams p, const float *qmean_all, const float *kmean_all) {
+    extern __shared__ float qm_s[];
+    const int hb = blockIdx.x;
+    const int h = hb / p.n_qb;
+    const float *qm = qmean_all + (int64_t)hb * p.D;
+    for (int c = threadIdx.x; c < p.D; c += blockDim.x) qm_s[c] = qm[c];
+    __syncthreads();
+    const float *km = kmean_all + (int64_t)h * p.n_cand * p.D;
+    float *sc = reinterpret_cast<float *>(p.buf + p.lay.off_score) + (int64_t)hb * p.n_cand;
+    for (int cand = threadIdx.x; cand < p.n_cand; cand += blockDim.x) {
+        const float *k = km + (int64_t)cand * p.D;
+        float acc = 0.0f;
+        for (int c = 0; c < p.D; ++c) acc = __fmaf_rn(qm_s[c], k[c], acc);
+        sc[cand] = acc;
+    }
+}
+
+// Device address of this file's scratch array on the current device, looked up once per device.
+static int static_pool_ptr(int device, float **out) {
+    static std::mutex mu;
+    static float *ptrs[256] = {};
+    if (device < 0 || device >= 256) return NOMAS_EINVAL;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[device]) {
+        void *ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_pool_scratch);
+        if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(g_pool_scratch)", (int)e, cudaGetErrorString(e));
+        ptrs[device] = static_cast<float *>(ptr);
+    }
+    *out = ptrs[device];
+    return NOMAS_OK;
+}
+
+}  // namespace nomas
+
+extern "C" int nomas_mask_build_static(const nomas_kv_cache *c, const nomas_segment_text *seg, int mode,
+                                       float keep_frac, const void *q, const void *kcur, int64_t tok_stride,
+                                       int64_t head_stride, void *mask_buf, nomas_stream stream) {
+    if (mode == NOMAS_MODE_DENSE)   // the dense build uses no scratch memory
+        return nomas_mask_build(c, seg, mode, keep_frac, q, kcur, tok_stride, head_stride, mask_buf, stream);
+    nomas_mask_layout lay;
+    int rc = compute_mask_layout(c, seg, mode, keep_frac, &lay);
+    if (rc) return rc;
+    if (!mask_buf || !aligned16(mask_buf)) return NOMAS_EINVAL;
+    if (!q || !kcur || !aligned16(q) || !aligned16(kcur)) return NOMAS_EINVAL;
+    if (tok_stride <= 0 || head_stride <= 0 || tok_stride % 8 || head_stride % 8) return NOMAS_EINVAL;
+    if (lay.n_cand < 1) return NOMAS_EINVAL;
+    const size_t nq_floats = (size_t)c->d.heads * lay.n_qblocks * c->d.head_dim;
+    const size_t nk_floats = (size_t)c->d.heads * lay.n_cand * c->d.head_dim;
+    if (nq_floats + nk_floats > kStaticPoolFloats) return NOMAS_ECAPACITY;
+    if (bind_device(c)) return NOMAS_ECUDA;
+    float *pool = nullptr;
+    rc = static_pool_ptr(c->device, &pool);
+    if (rc) return rc;
+    float *qmean = pool;
+    float *kmean = pool + nq_floats;
+
+    MaskParams p{};
+    const HistView hv = hist_view(c);
+    p.hdr.magic = kMaskMagic;
+    p.hdr.mode = mode;
+    p.hdr.n_qblocks = lay.n_qblocks;
+    p.hdr.n_lists = lay.n_lists;
+    p.hdr.history_tokens = lay.history_tokens;
+    p.hdr.head_tokens = lay.head_tokens;
+    p.hdr.frames_appended = c->frames_appended;
+    p.hdr.n_query = lay.n_query;
+    p.hdr.text_tokens = lay.text_tokens;
+    p.hdr.list_cap = lay.list_cap;
+    p.hdr.keep = lay.keep;
+    p.n_tails = seg->n_tails;
+    p.head_len = seg->head_len;
+    for (int i = 0; i < seg->n_tails; ++i) p.tails[i] = seg->tails[i];
+    p.T = c->d.tokens_per_frame;
+    p.H = c->d.heads;
+    p.D = c->d.head_dim;
+    p.Lh = lay.history_tokens;
+    p.Lp = lay.head_tokens;
+    p.Nq = lay.n_query;
+    p.Lt = lay.text_tokens;
+    p.n_qb = lay.n_qblocks;
+    p.n_tiles = lay.n_tiles;
+    p.n_hist_tiles = lay.n_hist_tiles;
+    p.n_head_tiles = lay.n_head_tiles;
+    p.n_cur_tiles = lay.n_cur_tiles;
+    p.n_text_tiles = lay.n_text_tiles;
+    p.n_cand = lay.n_cand;
+    p.keep = lay.keep;
+    p.n_lists = lay.n_lists;
+    p.list_cap = lay.list_cap;
+    p.buf = static_cast<uint8_t *>(mask_buf);
+    p.lay = lay;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.kcur = static_cast<const __nv_bfloat16 *>(kcur);
+    p.tok_stride = tok_stride;
+    p.head_stride = head_stride;
+    p.k8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_K8]);
+    p.ks = static_cast<const float *>(c->buf[NOMAS_BUF_KS]);
+    p.ring_tokens = hv.ring_tokens;
+    p.first_tok = hv.first_tok;
+
+    // every pooled mean is written before it is read, so the shared array needs no clearing
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    mask_prep_kernel<<<nblk(lay.text_tokens > 0 ? lay.text_tokens : 1, 256), 256, 0, st>>>(p);
+    class_map_kernel<<<nblk((int64_t)lay.n_qblocks * lay.n_tiles, 256), 256, 0, st>>>(p);
+    qmean_to_kernel<<<nblk((int64_t)nq_floats, 256), 256, 0, st>>>(p, qmean);
+    kmean_to_kernel<<<nblk((int64_t)nk_floats, 256), 256, 0, st>>>(p, kmean);
+    score_from_kernel<<<p.H * p.n_qb, 256, p.D * sizeof(float), st>>>(p, qmean, kmean);
+    select_kernel<<<p.H * p.n_qb, 256, p.n_cand * sizeof(float), st>>>(p);
+    lists_sparse_kernel<<<p.H * ((p.n_qb + 1) / 2), 128, 2 * ((p.n_cand + 31) / 32) * sizeof(uint32_t), st>>>(p);
+    return check_launch("mask_build_static kernels launch");
+}

@@ -213,23 +213,29 @@ int nomas_mask_build_static(const nomas_kv_cache *cache, const nomas_segment_tex
                             float keep_frac, const void *q, const void *kcur, int64_t tok_stride,
                             int64_t head_stride, void *mask_buf, nomas_stream stream);
 
-/* Masked (or block-sparse) attention of the current segment's video queries
- * over the retained INT8 history, earlier description heads (INT8), the current
- * segment's video (bf16) and its text (bf16), with the visibility of
- * nomas_mask_build.  Per head h and query row i:
+/* Bytes of the workspace nomas_attn_fwd needs for this cache state and segment text: fp16 copies
+ * [H][n][D] of the current segment's K and V and of the text's K and V (0 on invalid arguments). */
+size_t nomas_attn_workspace_bytes(const nomas_kv_cache *cache, const nomas_segment_text *seg);
+
+/* Masked (or block-sparse) attention of the current segment's video queries over the retained INT8
+ * history, earlier description heads (INT8), the current segment's video and its text, with the
+ * visibility of nomas_mask_build (fluxbbs.com 架构; sparse mode: same page, 单卡 4090 怎么做到的).
+ * Per head h and query row i:
  *     O[i,h] = sum_j softmax_j(softmax_scale * q_i . k^_j) v^_j   over visible j
- * with k^ = code * scale for cached keys (exactly: bf16 codes in the QK^T product,
- * the key scale applied to the fp32 score) and v^ = fp16(code * scale) for cached
- * values; the P V product runs in fp16 with fp32 accumulation.
+ * with k^ = code * scale for cached keys (the key scale is applied to the fp32 score, the codes
+ * enter the tensor core exactly) and v^ = fp16(code * scale) for cached values.  The QK^T and PV
+ * products run on the tensor cores with fp16 operands and fp32 accumulation; bf16 inputs convert
+ * to fp16 exactly for magnitudes in [2^-14, 65504] (the supported input range).
  *   q, kcur, vcur  bf16 [n_frames*T][H][D];  ktxt, vtxt bf16 [text_tokens][H][D]
- *                  (NULL allowed when the segment has no text)
+ *                  (NULL allowed when the segment has no text); all share tok_stride / head_stride
  *   out            fp32 [n_frames*T][H][D], contiguous
- *   lse            fp32 [H][n_frames*T] natural-log sum of exp of the scaled
- *                  scores, nullable */
+ *   lse            fp32 [H][n_frames*T] natural-log sum of exp of the scaled scores, nullable
+ *   workspace      device buffer of nomas_attn_workspace_bytes bytes, 16-byte aligned, caller-owned;
+ *                  overwritten by the call (calls that share it must not overlap on the GPU) */
 int nomas_attn_fwd(const nomas_kv_cache *cache, const nomas_segment_text *seg, int mode, float keep_frac,
                    const void *mask_buf, const void *q, const void *kcur, const void *vcur, const void *ktxt,
                    const void *vtxt, int64_t tok_stride, int64_t head_stride, float softmax_scale, float *out,
-                   float *lse, nomas_stream stream);
+                   float *lse, void *workspace, nomas_stream stream);
 
 /* Diagnostic: retained history in age order, dequantised as fp32 code * scale.
  *   k_out, v_out  fp32 [history_tokens][H][D] */

@@ -26,7 +26,7 @@ NOMAS_STATIC_POOL_FLOATS = 2 << 20
 EXPORTED = ["nomas_kv_cache_bytes", "nomas_kv_cache_init", "nomas_kv_cache_destroy", "nomas_kv_cache_state",
             "nomas_kv_append", "nomas_mask_layout_query", "nomas_mask_bytes", "nomas_mask_build",
             "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string",
-            "nomas_last_error", "nomas_mask_build_static"]
+            "nomas_last_error", "nomas_mask_build_static", "nomas_attn_workspace_bytes"]
 
 
 class nomas_cache_dims(ctypes.Structure):
@@ -75,8 +75,9 @@ _sigs = {
                                         _i64, _i64, _p, _p]),
     "nomas_mask_build_static": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32, _p,
                                                _p, _i64, _i64, _p, _p]),
+    "nomas_attn_workspace_bytes": (_sz, [_p, ctypes.POINTER(nomas_segment_text)]),
     "nomas_attn_fwd": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32, _p, _p, _p,
-                                      _p, _p, _p, _i64, _i64, _f32, _p, _p, _p]),
+                                      _p, _p, _p, _i64, _i64, _f32, _p, _p, _p, _p]),
     "nomas_kv_dequant": (ctypes.c_int, [_p, _p, _p, _p]),
     "nomas_device_status": (ctypes.c_int, [_p, _p]),
     "nomas_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -169,10 +170,15 @@ def nomas_mask_build_static(handle, seg, mode, keep_frac, q, kcur, tok_stride, h
                                        tok_stride, head_stride, mask_buf, stream or None)
 
 
+def nomas_attn_workspace_bytes(handle, seg):
+    return lib.nomas_attn_workspace_bytes(handle, ctypes.byref(seg))
+
+
 def nomas_attn_fwd(handle, seg, mode, keep_frac, mask_buf, q, kcur, vcur, ktxt, vtxt, tok_stride, head_stride,
-                   softmax_scale, out, lse=0, stream=0):
+                   softmax_scale, out, lse=0, workspace=0, stream=0):
     return lib.nomas_attn_fwd(handle, ctypes.byref(seg), mode, keep_frac, mask_buf, q, kcur, vcur, ktxt or None,
-                              vtxt or None, tok_stride, head_stride, softmax_scale, out, lse or None, stream or None)
+                              vtxt or None, tok_stride, head_stride, softmax_scale, out, lse or None,
+                              workspace or None, stream or None)
 
 
 def nomas_kv_dequant(handle, k_out, v_out, stream=0):

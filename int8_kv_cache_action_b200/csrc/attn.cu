@@ -1,31 +1,34 @@
 // nomas_attn_fwd: action-aware segment-causal attention over an INT8 history (fluxbbs.com "架构" for
-// the visibility; "单卡 4090 怎么做到的" for INT8 storage / BF16 compute and the sparse mode).
+// the visibility; "单卡 4090 怎么做到的" for INT8 storage and the sparse mode).
 //
 // One CTA = one head x two 128-row query tiles (Q0, Q1) that share every K/V tile of their list.
 //   warps 0-3   softmax for Q0   (TMEM lanes 0-127 of S0 / O0; one thread per query row)
 //   warps 4-7   softmax for Q1
-//   warps 8-11  loader: TMA for bf16 key tiles; INT8 keys -> bf16 codes and INT8 values x scale ->
-//               fp16, bf16 values -> fp16, all written in the 128B-swizzled UMMA layout;
-//               per-column key scale and visibility window for the softmax
+//   warps 8-11  loader: converts Q in place once; TMA for current-segment and text K/V tiles (fp16,
+//               prepared by values_f16_kernel); INT8 keys -> fp16 codes and INT8 values x scale ->
+//               fp16 written in the 128B-swizzled UMMA layout; per-column key scale and visibility
+//               window for the softmax
 //   warp 12     tcgen05.mma issuer (one thread) and TMEM owner; warps 13-15 idle
 // The register file is split per SM sub-partition (one warp of each warpgroup on each), so the
 // kernel launches at 128 registers per thread and moves them with setmaxnreg: softmax 168 each,
 // loader 112, MMA warpgroup 64 -- 2*168 + 112 + 64 = 512 = 4 x 128, the launch's own total.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D); P_q (fp16) overwrites
 // the first 64 columns of S_q and feeds the PV MMA as its A operand.
-// Precision: Q K^T runs in bf16 with the INT8 key codes exact and the key scale applied to the fp32
-// score; P V runs in fp16 (P <= 2^8 and the values fit its range), which keeps 3 more significand
-// bits than bf16 for the weights and the dequantised values (fp32 accumulation in both).
-// Per KV tile j the MMA thread issues S_q = Q_q K_j^T when K_j has landed and PV_q(j-1) has been
-// issued, and O_q += P_q V_j when softmax q has published P_q; both query tiles are interleaved so
-// that the tensor core works on one tile while the other tile's softmax runs.
-// Softmax uses a lazy rescale: the running offset moves only when the row maximum grows by more than
-// 8 (log2 units), and then O_q is rescaled in TMEM by the owning thread.  The completion of
-// S_q(j) implies completion of every earlier MMA of this thread (tcgen05.commit tracks all prior
-// operations), so O_q is idle whenever softmax q holds a fresh S_q.
+//
+// Precision: every MMA operand is fp16 with fp32 accumulation.  bf16 inputs convert to fp16
+// exactly for magnitudes in [2^-14, 65504] (the supported input range; smaller values keep 2^-24
+// absolute resolution), INT8 key codes are exact and the key scale is applied to the fp32 score,
+// cached values are fp16(code * scale), and P <= 2^8 keeps 11 significant bits.
+//
+// Scheduling: per KV tile j the MMA thread issues S_q = Q_q K_j^T when K_j has landed and PV_q of
+// the previous tile has been issued, and O_q += P_q V_j when softmax q has published P_q, so the
+// tensor core works on one query tile while the other tile's softmax runs.  Softmax uses a lazy
+// rescale: the running offset moves only when the row maximum grows by more than 8 (log2 units),
+// and then O_q is rescaled in TMEM by its owning thread; completion of S_q(j) implies completion of
+// every earlier MMA of this thread (tcgen05.commit tracks all prior operations), so O_q is idle
+// whenever softmax q holds a fresh S_q.
 #include <cmath>
 #include <cstdio>
-
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -41,7 +44,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 template <int D>
 struct AttnCfg {
     static constexpr int NS = (D == 128) ? 4 : 8;          // K/V tile slots (K_j, V_j alternate)
-    static constexpr int SLOT = kTile * D * 2;             // bytes of one bf16 tile
+    static constexpr int SLOT = kTile * D * 2;             // bytes of one 16-bit tile
     static constexpr int QB = kTile * D * 2;
     static constexpr int HALVES = D / 64;                  // 64-column (128-byte) swizzle panels
     static constexpr int KSTEPS = D / 16;
@@ -50,7 +53,7 @@ struct AttnCfg {
     static constexpr int OFF_CS = OFF_KV + NS * SLOT;      // float [kNCI][128]
     static constexpr int OFF_CW = OFF_CS + kNCI * 512;     // int2  [kNCI][128]
     static constexpr int OFF_BAR = OFF_CW + kNCI * 1024;
-    static constexpr int NBAR = 1 + 2 * NS + 2 * kNCI + 6;
+    static constexpr int NBAR = 2 + 2 * NS + 2 * kNCI + 6;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int SMEM = BYTES + 1024;              // slack for 1024-byte alignment
@@ -63,9 +66,6 @@ struct AttnParams {
     const int8_t *hk8, *hv8;
     const float *hks, *hvs;
     int64_t ring_tokens, first_tok, head_rows;
-    // current-segment and text values (bf16), staged to fp16 by the loader
-    const __nv_bfloat16 *vcur, *vtxt;
-    int64_t tok_stride, head_stride;
     // mask buffer
     const uint8_t *mask;
     const int4 *lists;
@@ -90,6 +90,23 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t f16x2_of(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
 template <int N>
 __device__ __forceinline__ void setmaxnreg_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
@@ -111,45 +128,51 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// 8 int8 codes -> 8 bf16 (exact: |code| <= 127), packed in 16 bytes.
-__device__ __forceinline__ uint4 cvt_i8x8_bf16(uint32_t lo, uint32_t hi) {
-    const uint32_t w[2] = {lo, hi};
-    uint32_t o[4];
+// 16 int8 codes -> 16 exact fp16 values (two 16-byte chunks).  Each biased byte u = b + 128 becomes
+// the low byte of the fp16 pattern 0x64uu = 1024 + u; one packed add of -1152 leaves b exactly.
+__device__ __forceinline__ void i8x16_to_f16(const uint4 &w, uint4 &lo, uint4 &hi) {
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t src = w[i >> 1];
-        const int sh = (i & 1) * 16;
-        __nv_bfloat162 pr = __floats2bfloat162_rn((float)(int8_t)((src >> sh) & 0xFF),
-                                                  (float)(int8_t)((src >> (sh + 8)) & 0xFF));
-        o[i] = *reinterpret_cast<uint32_t *>(&pr);
+        const uint32_t x = in[i] ^ 0x80808080u;
+        o[2 * i] = hadd2_u32(__byte_perm(x, 0x64646464u, 0x4140), 0xE480E480u);
+        o[2 * i + 1] = hadd2_u32(__byte_perm(x, 0x64646464u, 0x4342), 0xE480E480u);
     }
-    return make_uint4(o[0], o[1], o[2], o[3]);
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// 8 int8 codes times their row scale -> 8 fp16 (round to nearest), packed in 16 bytes.
-__device__ __forceinline__ uint4 cvt_i8x8_f16(uint32_t lo, uint32_t hi, float s) {
-    const uint32_t w[2] = {lo, hi};
-    uint32_t o[4];
+// 16 int8 codes times a row scale -> 16 fp16 values.  Each biased byte u becomes the float
+// 2^23 + u (pattern 0x4B0000uu); subtracting 2^23 + 128 leaves the code exactly in fp32, which is
+// multiplied by the scale and rounded once to fp16.
+__device__ __forceinline__ void i8x16_scaled_to_f16(const uint4 &w, float s, uint4 &lo, uint4 &hi) {
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    const float2 bias = make_float2(-8388736.0f, -8388736.0f);
+    const float2 sc = make_float2(s, s);
+    uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t src = w[i >> 1];
-        const int sh = (i & 1) * 16;
-        __half2 pr = __floats2half2_rn((float)(int8_t)((src >> sh) & 0xFF) * s,
-                                       (float)(int8_t)((src >> (sh + 8)) & 0xFF) * s);
-        o[i] = *reinterpret_cast<uint32_t *>(&pr);
+        const uint32_t x = in[i] ^ 0x80808080u;
+        float2 a = make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440)),
+                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441)));
+        float2 b = make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7442)),
+                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7443)));
+        a = __fmul2_rn(__fadd2_rn(a, bias), sc);
+        b = __fmul2_rn(__fadd2_rn(b, bias), sc);
+        o[2 * i] = f16x2_of(a.x, a.y);
+        o[2 * i + 1] = f16x2_of(b.x, b.y);
     }
-    return make_uint4(o[0], o[1], o[2], o[3]);
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// 8 bf16 -> 8 fp16 (exact for |x| >= 2^-14; below that fp16 keeps 2^-24 absolute resolution).
-__device__ __forceinline__ uint4 cvt_bf16x8_f16(const uint4 &v) {
+// 8 bf16 -> 8 fp16 (16 bytes in, 16 bytes out).
+__device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 &v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __half2 pr = __floats2half2_rn(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-        o[i] = *reinterpret_cast<uint32_t *>(&pr);
-    }
+    for (int i = 0; i < 4; ++i) o[i] = f16x2_of(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
@@ -167,8 +190,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float *sCS = reinterpret_cast<float *>(sm + C::OFF_CS);
     int2 *sCW = reinterpret_cast<int2 *>(sm + C::OFF_CW);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
-    uint64_t *bar_q = bars;
-    uint64_t *kv_full = bars + 1;
+    uint64_t *bar_q = bars;          // Q tiles landed (TMA, bf16)
+    uint64_t *q_ready = bars + 1;    // Q converted to fp16 in place
+    uint64_t *kv_full = bars + 2;
     uint64_t *kv_empty = kv_full + C::NS;
     uint64_t *ci_full = kv_empty + C::NS;
     uint64_t *ci_empty = ci_full + kNCI;
@@ -200,6 +224,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
+        mbar_init(q_ready, 1);
         for (int i = 0; i < C::NS; ++i) {
             mbar_init(&kv_full[i], 1);
             mbar_init(&kv_empty[i], 1);
@@ -235,11 +260,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // Every wait is followed by a named barrier over the 128 loader threads and a read of the
         // shared abort flag, so all loader threads leave the loop together.
         wd.where = 3;
-        const int t = threadIdx.x - 256;  // 0..127
+        const int t = threadIdx.x - 256;   // 0..127
         uint32_t tma_pending = 0, tma_par = 0;   // per slot: a TMA was issued / its phase parity
         if (t == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_kc);
+            prefetch_tmap(&tm_vc);
             mbar_arrive_expect_tx(bar_q, 2 * C::QB);
 #pragma unroll
             for (int q = 0; q < 2; ++q)
@@ -248,20 +274,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     tma_load_3d(sQ + q * C::QB + hh * (kTile * 128), &tm_q, bar_q, hh * 64, h,
                                 (int)(qrow0 + q * kTile));
         }
+        // Q: bf16 -> fp16 in place (the conversion keeps every element's byte position)
+        mbar_wait(bar_q, 0, wd, 4);
+        named_bar_sync(1, 128);
+        if (!*abort_flag) {
+#pragma unroll 4
+            for (int i = t; i < 2 * C::QB / 16; i += 128) {
+                uint4 *ptr = reinterpret_cast<uint4 *>(sQ) + i;
+                *ptr = bf16x8_to_f16(*ptr);
+            }
+            fence_proxy_async_smem();
+        }
+        named_bar_sync(1, 128);
+        if (t == 0 && !*abort_flag) mbar_arrive(q_ready);
+
         constexpr int CPR = D / 16;          // 16-byte int8 chunks per row
-        constexpr int RSTEP = 128 / CPR;     // int8 rows covered by the 128 threads in one pass
-        constexpr int NR = 128 / RSTEP;      // int8 rows per thread
-        constexpr int CPRB = D / 8;          // 16-byte bf16 chunks per row
-        constexpr int RSTEPB = 128 / CPRB;
-        constexpr int NRB = 128 / RSTEPB;    // bf16 rows per thread
-        constexpr int NRAW = (2 * NR > NRB) ? 2 * NR : NRB;
+        constexpr int RSTEP = 128 / CPR;     // rows covered by the 128 threads in one pass
+        constexpr int NR = 128 / RSTEP;      // rows per thread
         const int my_chunk = t % CPR;
         const int my_row0 = t / CPR;
         const int hh_mine = my_chunk / 4;
         const int c0_mine = (my_chunk % 4) * 2;
-        const int my_chunkb = t % CPRB;
-        const int my_row0b = t / CPRB;
-        for (int j = 0; j < n_tiles; ++j) {
+        for (int j = 0; j < n_tiles && !*abort_flag; ++j) {
             const int4 e = list[j];
             const int kind = e.x & 3;
             const int64_t start = e.y;
@@ -277,32 +311,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int64_t a = start + r;
                 return head_base + (hist ? (p.first_tok + a) % p.ring_tokens : a);
             };
-            // raw loads issued first so their latency overlaps the slot waits:
-            //   cached tile: raw[0, NR) = K codes, raw[NR, 2 NR) = V codes (16 int8 per chunk)
-            //   bf16 tile:   raw[0, NRB) = V values (8 bf16 per chunk); K arrives by TMA
-            uint4 raw[NRAW];
+            // raw INT8 loads issued first so that their latency overlaps the slot waits
+            uint4 rk[NR], rv[NR];
             float svv[NR];
-#pragma unroll
-            for (int i = 0; i < NRAW; ++i) raw[i] = make_uint4(0, 0, 0, 0);
             if (cached) {
 #pragma unroll
                 for (int i = 0; i < NR; ++i) {
                     const int r = my_row0 + i * RSTEP;
+                    rk[i] = rv[i] = make_uint4(0, 0, 0, 0);
                     svv[i] = 0.0f;
                     if (r < count) {
                         const int64_t gr = cache_row(r);
-                        raw[i] = __ldg(reinterpret_cast<const uint4 *>(src_k + gr * D) + my_chunk);
-                        raw[NR + i] = __ldg(reinterpret_cast<const uint4 *>(src_v + gr * D) + my_chunk);
+                        rk[i] = __ldg(reinterpret_cast<const uint4 *>(src_k + gr * D) + my_chunk);
+                        rv[i] = __ldg(reinterpret_cast<const uint4 *>(src_v + gr * D) + my_chunk);
                         svv[i] = __ldg(src_vs + gr);
                     }
-                }
-            } else {
-                const __nv_bfloat16 *vb = (kind == kKindCur ? p.vcur : p.vtxt) + (int64_t)h * p.head_stride;
-#pragma unroll
-                for (int i = 0; i < NRB; ++i) {
-                    const int r = my_row0b + i * RSTEPB;
-                    if (r < count)
-                        raw[i] = __ldg(reinterpret_cast<const uint4 *>(vb + (start + r) * p.tok_stride) + my_chunkb);
                 }
             }
             float cs = 0.0f;
@@ -327,7 +350,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     mbar_arrive_expect_tx(&kv_full[sk], C::SLOT);
 #pragma unroll
                     for (int hh = 0; hh < C::HALVES; ++hh)
-                        tma_load_3d(dK + hh * (kTile * 128), m, &kv_full[sk], hh * 64, h, (int)start);
+                        tma_load_3d(dK + hh * (kTile * 128), m, &kv_full[sk], hh * 64, (int)start, h);
                     tma_pending |= 1u << sk;
                     tma_par = (tma_par & ~(1u << sk)) | ((uint32_t)(((2 * j) / C::NS) & 1) << sk);
                 }
@@ -335,9 +358,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
                 for (int i = 0; i < NR; ++i) {
                     const int r = my_row0 + i * RSTEP;
+                    uint4 lo, hi;
+                    i8x16_to_f16(rk[i], lo, hi);
                     uint8_t *base = dK + hh_mine * (kTile * 128);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = cvt_i8x8_bf16(raw[i].x, raw[i].y);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = cvt_i8x8_bf16(raw[i].z, raw[i].w);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = lo;
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = hi;
                 }
                 fence_proxy_async_smem();
                 tma_pending &= ~(1u << sk);
@@ -350,28 +375,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_wait(&kv_empty[sv], (((2 * j + 1) / C::NS) & 1) ^ 1, wd, 3);
             named_bar_sync(1, 128);
             if (*abort_flag) break;
-            uint8_t *dV = sKV + sv * C::SLOT;   // V is staged as fp16 (the PV product runs in fp16)
-            if (cached) {
+            uint8_t *dV = sKV + sv * C::SLOT;
+            if (!cached) {
+                if (t == 0) {
+                    const CUtensorMap *m = kind == kKindCur ? &tm_vc : &tm_vt;
+                    mbar_arrive_expect_tx(&kv_full[sv], C::SLOT);
 #pragma unroll
-                for (int i = 0; i < NR; ++i) {
-                    const int r = my_row0 + i * RSTEP;
-                    uint8_t *base = dV + hh_mine * (kTile * 128);
-                    const uint4 &v = raw[NR + i];
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = cvt_i8x8_f16(v.x, v.y, svv[i]);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = cvt_i8x8_f16(v.z, v.w, svv[i]);
+                    for (int hh = 0; hh < C::HALVES; ++hh)
+                        tma_load_3d(dV + hh * (kTile * 128), m, &kv_full[sv], hh * 64, (int)start, h);
+                    tma_pending |= 1u << sv;
+                    tma_par = (tma_par & ~(1u << sv)) | ((uint32_t)(((2 * j + 1) / C::NS) & 1) << sv);
                 }
             } else {
 #pragma unroll
-                for (int i = 0; i < NRB; ++i) {
-                    const int r = my_row0b + i * RSTEPB;
-                    uint8_t *base = dV + (my_chunkb / 8) * (kTile * 128);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, my_chunkb % 8)) = cvt_bf16x8_f16(raw[i]);
+                for (int i = 0; i < NR; ++i) {
+                    const int r = my_row0 + i * RSTEP;
+                    uint4 lo, hi;
+                    i8x16_scaled_to_f16(rv[i], svv[i], lo, hi);
+                    uint8_t *base = dV + hh_mine * (kTile * 128);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = lo;
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = hi;
                 }
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                tma_pending &= ~(1u << sv);
+                if (t == 0) mbar_arrive(&kv_full[sv]);
             }
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            tma_pending &= ~(1u << sv);
-            if (t == 0) mbar_arrive(&kv_full[sv]);
         }
         // on abort, let this CTA's bulk copies land before the shared memory is released
         if (*abort_flag && t == 0) {
@@ -385,13 +414,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         setmaxnreg_dec<kRegMma>();
         wd.where = 4;
         if (warp == 12 && lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_pv = idesc_f16_f32(128, D, false, true);   // P and V both fp16
+            constexpr uint32_t idesc_qk = idesc_f16_f32(128, 128, false, false);
+            constexpr uint32_t idesc_pv = idesc_f16_f32(128, D, false, true);
             const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
             const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
             const uint32_t q_addr = smem_u32(sQ);
             const uint32_t kv_addr = smem_u32(sKV);
-            bool ok = mbar_wait(bar_q, 0, wd, 1);
+            bool ok = mbar_wait(q_ready, 0, wd, 1);
             int next_s[2];              // next list index whose S_q is to be issued
             int pend[2] = {-1, -1};     // list index whose PV_q waits for P_q
             int last_s[2] = {-1, -1}, last_pv[2] = {-1, -1};
@@ -513,48 +542,70 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 continue;
             }
             const bool masked = (e.x & (q ? kMask1 : kMask0)) != 0;
+            const bool cached = (e.x & 3) == kKindHist || (e.x & 3) == kKindPriorHead;
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[q], k & 1, wd, 2));
             if (!ok) break;
             tc_fence_after();
             float s[128];
 #pragma unroll
             for (int c4 = 0; c4 < 4; ++c4) tmem_ld32f_sync(tS + c4 * 32, &s[c4 * 32]);
-            const float *cs = sCS + ci * 128;
-            const int2 *cw = sCW + ci * 128;
-            float mt = -INFINITY;
+            // cached keys: apply the per-key scale (which carries softmax scale * log2 e) to the score
+            if (cached) {
+                const float4 *cs4 = reinterpret_cast<const float4 *>(sCS + ci * 128);
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                float v = s[c] * cs[c];
-                if (masked) {
-                    const int2 w = cw[c];
-                    v = (w.x <= frame && frame < w.y) ? v : -INFINITY;
+                for (int i = 0; i < 32; ++i) {
+                    if ((i & 7) == 0) asm volatile("" ::: "memory");   // bound how far loads are hoisted
+                    const float4 v = cs4[i];
+                    const float2 a = __fmul2_rn(make_float2(s[4 * i], s[4 * i + 1]), make_float2(v.x, v.y));
+                    const float2 b = __fmul2_rn(make_float2(s[4 * i + 2], s[4 * i + 3]), make_float2(v.z, v.w));
+                    s[4 * i] = a.x;
+                    s[4 * i + 1] = a.y;
+                    s[4 * i + 2] = b.x;
+                    s[4 * i + 3] = b.y;
                 }
-                s[c] = v;
-                mt = fmaxf(mt, v);
+            }
+            if (masked) {
+                const int4 *cw = reinterpret_cast<const int4 *>(sCW + ci * 128);
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    if ((i & 7) == 0) asm volatile("" ::: "memory");
+                    const int4 w = cw[i];   // windows of columns 2i and 2i+1
+                    s[2 * i] = (w.x <= frame && frame < w.y) ? s[2 * i] : -INFINITY;
+                    s[2 * i + 1] = (w.z <= frame && frame < w.w) ? s[2 * i + 1] : -INFINITY;
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_empty[ci]);
+            float mt = max3(s[0], s[1], s[2]);
+#pragma unroll
+            for (int c = 3; c < 127; c += 2) mt = max3(mt, s[c], s[c + 1]);
+            mt = fmaxf(mt, s[127]);
+            // log2 domain: cached scores are already scaled, bf16-source scores get the uniform scale
+            const float cmul = cached ? 1.0f : p.scale_log2;
+            mt *= cmul;
             const float m_new = fmaxf(m_used, mt);
             const bool grow = m_new > m_used + kRescaleThreshold;   // false while both are -inf
             const bool need_o = grow && m_used != -INFINITY;
             const float f = need_o ? ex2(m_used - m_new) : 1.0f;
             if (grow) m_used = m_new;
             const float off = (m_used == -INFINITY) ? 0.0f : m_used;
-            float sum = 0.0f;
+            const float2 cm2 = make_float2(cmul, cmul);
+            const float2 no2 = make_float2(-off, -off);
+            float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t pk[32];
+            for (int qt = 0; qt < 4; ++qt) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const float a = ex2(s[half * 64 + c] - off);
-                    const float b = ex2(s[half * 64 + c + 1] - off);
-                    sum += a + b;
-                    __half2 pr = __floats2half2_rn(a, b);
-                    pk[c / 2] = *reinterpret_cast<uint32_t *>(&pr);
+                for (int c = 0; c < 32; c += 2) {
+                    const float2 a = __ffma2_rn(make_float2(s[qt * 32 + c], s[qt * 32 + c + 1]), cm2, no2);
+                    const float p0 = ex2(a.x);
+                    const float p1 = ex2(a.y);
+                    acc = __fadd2_rn(acc, make_float2(p0, p1));
+                    pk[c / 2] = f16x2_of(p0, p1);
                 }
-                tmem_st32(tS + half * 32, pk);
+                tmem_st16(tS + qt * 16, pk);
             }
-            l = l * f + sum;
+            l = l * f + (acc.x + acc.y);
             // rescale O_q in TMEM (rare: only when some row's maximum grew past the threshold);
             // done after P so that the scores are no longer live
             if (__any_sync(0xffffffffu, need_o)) {
@@ -605,6 +656,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 }
 
+// bf16 [n][H][D] (token / head strides in elements) -> fp16 [H][n][D], for up to four tensors.
+struct F16Job {
+    const __nv_bfloat16 *src;
+    __half *dst;
+    int64_t n;
+};
+struct F16Jobs {
+    F16Job job[4];
+    int32_t n_jobs;
+    int32_t H, D;
+    int64_t tok_stride, head_stride;
+};
+
+__global__ void __launch_bounds__(256) values_f16_kernel(F16Jobs jobs) {
+    const int cpr = jobs.D / 8;   // 16-byte chunks per row
+    for (int jb = 0; jb < jobs.n_jobs; ++jb) {
+        const F16Job J = jobs.job[jb];
+        const int64_t total = J.n * jobs.H * cpr;
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+             i += (int64_t)gridDim.x * blockDim.x) {
+            const int c = (int)(i % cpr);
+            const int64_t rowi = i / cpr;              // = h * n + t  (destination order)
+            const int64_t t = rowi % J.n;
+            const int h = (int)(rowi / J.n);
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(J.src + t * jobs.tok_stride +
+                                                                  (int64_t)h * jobs.head_stride) + c);
+            reinterpret_cast<uint4 *>(J.dst + rowi * jobs.D)[c] = bf16x8_to_f16(v);
+        }
+    }
+}
+
 }  // namespace nomas
 
 // ------------------------------------------------------------------------------------------------
@@ -629,18 +711,16 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// [n_tok][H][D] bf16 with element strides; box = 128 tokens x one head x 64 channels, 128B swizzle.
-static bool make_map(CUtensorMap *m, const void *base, int64_t n_tok, int H, int D, int64_t tok_stride,
-                     int64_t head_stride) {
+// 3-D tiled map with 128B swizzle.  dims / strides are innermost first (strides in bytes for
+// dims 1 and 2); the box's inner extent is 64 elements (128 bytes).
+static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, const cuuint64_t dims[3],
+                     const cuuint64_t strides[2], const cuuint32_t box[3]) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(n_tok > 0 ? n_tok : 1)};
-    cuuint64_t strides[2] = {(cuuint64_t)head_stride * 2, (cuuint64_t)tok_stride * 2};
-    cuuint32_t box[3] = {64, 1, (cuuint32_t)kTile};
     cuuint32_t es[3] = {1, 1, 1};
-    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         char msg[160];
         std::snprintf(msg, sizeof(msg), "dims %llu x %llu x %llu, strides %llu %llu", (unsigned long long)dims[0],
@@ -650,6 +730,24 @@ static bool make_map(CUtensorMap *m, const void *base, int64_t n_tok, int H, int
         return false;
     }
     return true;
+}
+
+// Workspace: fp16 [H][n][D] copies of the current segment's K, V and the text's K, V.
+struct WsLayout {
+    size_t off[4];
+    size_t total;
+};
+static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
+    WsLayout w;
+    const size_t row = (size_t)c->d.heads * c->d.head_dim * 2;
+    size_t off = 0;
+    const int64_t n[4] = {nq, nq, lt, lt};
+    for (int i = 0; i < 4; ++i) {
+        w.off[i] = off;
+        off += ((size_t)n[i] * row + 255) / 256 * 256;
+    }
+    w.total = off;
+    return w;
 }
 
 static uint64_t g_timeout_ns = 2000000000ull;   // 2 s per wait
@@ -671,33 +769,74 @@ static int launch_attn(const AttnParams &p, dim3 grid, const CUtensorMap *maps, 
 
 using namespace nomas;
 
+extern "C" size_t nomas_attn_workspace_bytes(const nomas_kv_cache *c, const nomas_segment_text *seg) {
+    nomas_mask_layout lay;
+    if (compute_mask_layout(c, seg, NOMAS_MODE_DENSE, 0.25f, &lay) != NOMAS_OK) return 0;
+    return ws_layout(c, lay.n_query, lay.text_tokens).total;
+}
+
 extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text *seg, int mode, float keep_frac,
                               const void *mask_buf, const void *q, const void *kcur, const void *vcur,
                               const void *ktxt, const void *vtxt, int64_t tok_stride, int64_t head_stride,
-                              float softmax_scale, float *out, float *lse, nomas_stream stream) {
+                              float softmax_scale, float *out, float *lse, void *workspace, nomas_stream stream) {
     nomas_mask_layout lay;
     int rc = compute_mask_layout(c, seg, mode, keep_frac, &lay);
     if (rc) return rc;
     if (!mask_buf || !aligned16(mask_buf)) return NOMAS_EINVAL;
-    if (!q || !kcur || !vcur || !out) return NOMAS_EINVAL;
-    if (!aligned16(q) || !aligned16(kcur) || !aligned16(vcur) || !aligned16(out)) return NOMAS_EINVAL;
+    if (!q || !kcur || !vcur || !out || !workspace) return NOMAS_EINVAL;
+    if (!aligned16(q) || !aligned16(kcur) || !aligned16(vcur) || !aligned16(out) || !aligned16(workspace))
+        return NOMAS_EINVAL;
     if (lay.text_tokens > 0 && (!ktxt || !vtxt || !aligned16(ktxt) || !aligned16(vtxt))) return NOMAS_EINVAL;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return NOMAS_EINVAL;
     if (tok_stride <= 0 || head_stride <= 0 || tok_stride % 8 || head_stride % 8) return NOMAS_EINVAL;
     if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale)) return NOMAS_EINVAL;
     const auto &d = c->d;
     const int D = d.head_dim;
+    const int H = d.heads;
     if (bind_device(c)) return NOMAS_ECUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+    // fp16 copies of the current segment's and the text's K / V (HBM-bound pre-pass)
+    const WsLayout ws = ws_layout(c, lay.n_query, lay.text_tokens);
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    F16Jobs jobs{};
+    jobs.H = H;
+    jobs.D = D;
+    jobs.tok_stride = tok_stride;
+    jobs.head_stride = head_stride;
+    const void *srcs[4] = {kcur, vcur, ktxt, vtxt};
+    const int64_t ns[4] = {lay.n_query, lay.n_query, lay.text_tokens, lay.text_tokens};
+    for (int i = 0; i < 4; ++i) {
+        if (ns[i] == 0) continue;
+        F16Job &J = jobs.job[jobs.n_jobs++];
+        J.src = static_cast<const __nv_bfloat16 *>(srcs[i]);
+        J.dst = reinterpret_cast<__half *>(wsb + ws.off[i]);
+        J.n = ns[i];
+    }
+    {
+        const int64_t chunks = (2 * lay.n_query + 2 * lay.text_tokens) * H * (D / 8);
+        int64_t blocks = (chunks + 255) / 256;
+        if (blocks > 148 * 16) blocks = 148 * 16;
+        values_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(jobs);
+        rc = check_launch("values_f16_kernel launch");
+        if (rc) return rc;
+    }
+
     CUtensorMap maps[5];
-    const void *kt = lay.text_tokens > 0 ? ktxt : q;
-    const void *vt = lay.text_tokens > 0 ? vtxt : q;
-    const int64_t nt = lay.text_tokens > 0 ? lay.text_tokens : lay.n_query;
-    if (!make_map(&maps[0], q, lay.n_query, d.heads, D, tok_stride, head_stride) ||
-        !make_map(&maps[1], kcur, lay.n_query, d.heads, D, tok_stride, head_stride) ||
-        !make_map(&maps[2], vcur, lay.n_query, d.heads, D, tok_stride, head_stride) ||
-        !make_map(&maps[3], kt, nt, d.heads, D, tok_stride, head_stride) ||
-        !make_map(&maps[4], vt, nt, d.heads, D, tok_stride, head_stride))
-        return NOMAS_ECUDA;
+    {
+        const cuuint64_t dq[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)lay.n_query};
+        const cuuint64_t sq[2] = {(cuuint64_t)head_stride * 2, (cuuint64_t)tok_stride * 2};
+        const cuuint32_t bq[3] = {64, 1, (cuuint32_t)kTile};
+        if (!make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, dq, sq, bq)) return NOMAS_ECUDA;
+        const cuuint32_t bk[3] = {64, (cuuint32_t)kTile, 1};
+        for (int i = 0; i < 4; ++i) {
+            const int64_t n = ns[i] > 0 ? ns[i] : 1;
+            const size_t off = ns[i] > 0 ? ws.off[i] : ws.off[0];
+            const cuuint64_t dk[3] = {(cuuint64_t)D, (cuuint64_t)n, (cuuint64_t)H};
+            const cuuint64_t sk[2] = {(cuuint64_t)D * 2, (cuuint64_t)n * D * 2};
+            if (!make_map(&maps[1 + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wsb + off, dk, sk, bk)) return NOMAS_ECUDA;
+        }
+    }
     const HistView hv = hist_view(c);
     AttnParams p{};
     p.k8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_K8]);
@@ -711,10 +850,6 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     p.ring_tokens = hv.ring_tokens;
     p.first_tok = hv.first_tok;
     p.head_rows = d.head_store_tokens;
-    p.vcur = static_cast<const __nv_bfloat16 *>(vcur);
-    p.vtxt = static_cast<const __nv_bfloat16 *>(lay.text_tokens > 0 ? vtxt : vcur);
-    p.tok_stride = tok_stride;
-    p.head_stride = head_stride;
     const uint8_t *mb = static_cast<const uint8_t *>(mask_buf);
     p.mask = mb;
     p.lists = reinterpret_cast<const int4 *>(mb + lay.off_list);
@@ -733,7 +868,7 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     p.expect.keep = lay.keep;
     p.sparse = mode == NOMAS_MODE_SPARSE;
     p.n_pairs = (lay.n_qblocks + 1) / 2;
-    p.H = d.heads;
+    p.H = H;
     p.T = d.tokens_per_frame;
     p.Nq = lay.n_query;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
@@ -741,7 +876,6 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     p.lse = lse;
     p.err = static_cast<int *>(c->buf[NOMAS_BUF_ERR]);
     p.timeout_ns = g_timeout_ns;
-    dim3 grid((unsigned)p.n_pairs, (unsigned)d.heads);
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    dim3 grid((unsigned)p.n_pairs, (unsigned)H);
     return D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
 }

@@ -127,8 +127,15 @@ class KVCache:
         N._check(rc, "nomas_mask_build")
         return mask_buf, lay
 
+    def workspace(self, seg):
+        """A device buffer of the size nomas_attn_fwd needs for this segment (torch-allocated)."""
+        n = N.nomas_attn_workspace_bytes(self.handle, seg)
+        if n == 0:
+            raise ValueError("invalid segment text")
+        return torch.empty(n, dtype=torch.uint8, device=self.device)
+
     def attention(self, seg, mask_buf, q, kcur, vcur, ktxt, vtxt, softmax_scale=None, mode=N.NOMAS_MODE_DENSE,
-                  keep_frac=0.25, out=None, lse=None, want_lse=False, stream=None):
+                  keep_frac=0.25, out=None, lse=None, want_lse=False, workspace=None, stream=None):
         ts, hs = _bf16_strides(q)
         for t in (kcur, vcur) + ((ktxt, vtxt) if ktxt is not None and ktxt.shape[0] else ()):
             if _bf16_strides(t) != (ts, hs):
@@ -140,10 +147,13 @@ class KVCache:
             lse = torch.empty((H, nq), dtype=torch.float32, device=self.device)
         scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(D)
         has_txt = ktxt is not None and ktxt.shape[0] > 0
+        if workspace is None:
+            workspace = self.workspace(seg)
         rc = N.nomas_attn_fwd(self.handle, seg, mode, keep_frac, mask_buf.data_ptr(), q.data_ptr(),
                               kcur.data_ptr(), vcur.data_ptr(), ktxt.data_ptr() if has_txt else 0,
                               vtxt.data_ptr() if has_txt else 0, ts, hs, scale, out.data_ptr(),
-                              lse.data_ptr() if lse is not None else 0, _stream_handle(stream))
+                              lse.data_ptr() if lse is not None else 0, workspace.data_ptr(),
+                              _stream_handle(stream))
         N._check(rc, "nomas_attn_fwd")
         return out, lse
 

@@ -4,7 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 
-#include "../../include/nomas.h"
+#include "nomas.h"
 
 struct nomas_kv_cache {
     nomas_cache_dims d;

@@ -213,8 +213,11 @@ int nomas_mask_build_static(const nomas_kv_cache *cache, const nomas_segment_tex
                             float keep_frac, const void *q, const void *kcur, int64_t tok_stride,
                             int64_t head_stride, void *mask_buf, nomas_stream stream);
 
-/* Bytes of the workspace nomas_attn_fwd needs for this cache state and segment text: fp16 copies
- * [H][n][D] of the current segment's K and V and of the text's K and V (0 on invalid arguments). */
+/* Bytes of the workspace nomas_attn_fwd needs for this cache and segment text (0 on invalid
+ * arguments).  The size depends only on the cache dimensions and the segment text, not on how much
+ * history is retained.  nomas_attn_fwd fills it with its operand copies: fp16 keys [H][n][D] and
+ * transposed fp16 values [H][D][n] of the current segment and the text, and the retained INT8
+ * history in age order (keys [H][tokens][D], transposed values [H][D][tokens], scales). */
 size_t nomas_attn_workspace_bytes(const nomas_kv_cache *cache, const nomas_segment_text *seg);
 
 /* Masked (or block-sparse) attention of the current segment's video queries over the retained INT8

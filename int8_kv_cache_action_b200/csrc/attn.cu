@@ -1,32 +1,38 @@
 // nomas_attn_fwd: action-aware segment-causal attention over an INT8 history (fluxbbs.com "架构" for
 // the visibility; "单卡 4090 怎么做到的" for INT8 storage and the sparse mode).
 //
-// One CTA = one head x two 128-row query tiles (Q0, Q1) that share every K/V tile of their list.
-//   warps 0-3   softmax for Q0   (TMEM lanes 0-127 of S0 / O0; one thread per query row)
-//   warps 4-7   softmax for Q1
-//   warps 8-11  loader: converts Q in place once; TMA for current-segment and text K/V tiles (fp16,
-//               prepared by values_f16_kernel); INT8 keys -> fp16 codes and INT8 values x scale ->
-//               fp16 written in the 128B-swizzled UMMA layout; per-column key scale and visibility
-//               window for the softmax
-//   warp 12     tcgen05.mma issuer (one thread) and TMEM owner; warps 13-15 idle
+// One CTA = one head x one 128-row query block.  Roles (16 warps, one CTA per SM):
+//   warps 0-3   softmax over key columns 0-63 of every S tile (TMEM lanes 0-127, one thread per row)
+//   warps 4-7   softmax over key columns 64-127; the two halves of a row swap their maxima through
+//               shared memory, so both apply the same offset
+//   warps 8-11  converter: per-column key scale and visibility window; an INT8 tile, which TMA lands
+//               in the upper half of its slot, becomes fp16 in place (key codes exactly, values as
+//               fp16(code * scale) with one scale per key)
+//   warp 12     tcgen05.mma issuer (one thread) and TMEM owner
+//   warp 13     TMA producer (one thread); warps 14-15 idle
 // The register file is split per SM sub-partition (one warp of each warpgroup on each), so the
 // kernel launches at 128 registers per thread and moves them with setmaxnreg: softmax 168 each,
-// loader 112, MMA warpgroup 64 -- 2*168 + 112 + 64 = 512 = 4 x 128, the launch's own total.
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [384,384+D); P_q (fp16) overwrites
-// the first 64 columns of S_q and feeds the PV MMA as its A operand.
+// converter 112, MMA / producer warpgroup 64 -- 2*168 + 112 + 64 = 512 = 4 x 128.
+//
+// TMEM (512 columns): Q (fp16 pairs) at [0, D/2), S double buffer at [128, 256) and [256, 384),
+// O at [384, 384 + D).  P (fp16) overwrites the first 32 columns of each 64-column half of its S
+// buffer, so each softmax half writes only columns it has already read.
+//
+// Both products are TS MMAs (A from TMEM) with a K-major B in 128-byte-swizzled shared memory:
+//   S_b  = Q K_j^T     B = K_j    [128 keys][D]
+//   O   += P_j V_j     B = V_j^T  [D][128 keys]   (values are stored transposed by the pre-pass)
+// For D = 128 the two share one instruction descriptor: a change of MMA shape between consecutive
+// tcgen05.mma batches stalls the tensor pipe, and the pipe only reaches full rate with more than
+// two batches in flight, which the S -> softmax -> PV dependency does not allow.  The issue order
+// S_0, S_1, PV_0, S_2, PV_1, ... computes S_{j+1} while the softmax works on S_j; S_{j+2} reuses
+// the buffer of S_j after PV_j, which tcgen05's in-order execution makes safe.
 //
 // Precision: every MMA operand is fp16 with fp32 accumulation.  bf16 inputs convert to fp16
 // exactly for magnitudes in [2^-14, 65504] (the supported input range; smaller values keep 2^-24
 // absolute resolution), INT8 key codes are exact and the key scale is applied to the fp32 score,
-// cached values are fp16(code * scale), and P <= 2^8 keeps 11 significant bits.
-//
-// Scheduling: per KV tile j the MMA thread issues S_q = Q_q K_j^T when K_j has landed and PV_q of
-// the previous tile has been issued, and O_q += P_q V_j when softmax q has published P_q, so the
-// tensor core works on one query tile while the other tile's softmax runs.  Softmax uses a lazy
-// rescale: the running offset moves only when the row maximum grows by more than 8 (log2 units),
-// and then O_q is rescaled in TMEM by its owning thread; completion of S_q(j) implies completion of
-// every earlier MMA of this thread (tcgen05.commit tracks all prior operations), so O_q is idle
-// whenever softmax q holds a fresh S_q.
+// cached values are fp16(code * scale), and P <= 2^8 keeps 11 significant bits.  Softmax uses a
+// lazy rescale: the running offset moves only when the row maximum grows by more than 8 (log2
+// units); O is then rescaled in TMEM once the previous PV has completed.
 #include <cmath>
 #include <cstdio>
 #include <cuda_fp16.h>
@@ -40,32 +46,39 @@ constexpr int kRegSoftmax = 168, kRegLoader = 112, kRegMma = 64;
 static_assert(2 * kRegSoftmax + kRegLoader + kRegMma == 4 * 128, "register split must equal the launch total");
 constexpr int kNCI = 4;                     // column-info ring depth
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr uint32_t kTmQ = 0, kTmS = 128, kTmO = 384;
 
 template <int D>
 struct AttnCfg {
-    static constexpr int NS = (D == 128) ? 4 : 8;          // K/V tile slots (K_j, V_j alternate)
-    static constexpr int SLOT = kTile * D * 2;             // bytes of one 16-bit tile
-    static constexpr int QB = kTile * D * 2;
-    static constexpr int HALVES = D / 64;                  // 64-column (128-byte) swizzle panels
+    static constexpr int NK = (D == 128) ? 3 : 6;          // K tile slots
+    static constexpr int NV = NK;                          // V^T tile slots
+    static constexpr int SLOT = kTile * D * 2;             // one fp16 tile
+    static constexpr int HALF = SLOT / 2;                  // an INT8 tile lands in the upper half
+    static constexpr int KPANEL = kTile * 128;             // K: 64 columns (128 B) of 128 rows
+    static constexpr int VPANEL = D * 128;                 // V^T: 64 keys (128 B) of D rows
     static constexpr int KSTEPS = D / 16;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_KV = OFF_Q + 2 * QB;
-    static constexpr int OFF_CS = OFF_KV + NS * SLOT;      // float [kNCI][128]
-    static constexpr int OFF_CW = OFF_CS + kNCI * 512;     // int2  [kNCI][128]
-    static constexpr int OFF_BAR = OFF_CW + kNCI * 1024;
-    static constexpr int NBAR = 2 + 2 * NS + 2 * kNCI + 6;
+    static constexpr int CHUNKS = kTile * D / 16 / 128;    // 16-byte INT8 chunks per converter thread
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + NK * SLOT;
+    static constexpr int OFF_CS = OFF_V + NV * SLOT;       // float [kNCI][128] key scale x log2 e
+    static constexpr int OFF_CW = OFF_CS + kNCI * 512;     // int2  [kNCI][128] key frame windows
+    static constexpr int OFF_VS = OFF_CW + kNCI * 1024;    // float [128] value scales of one tile
+    static constexpr int OFF_XM = OFF_VS + 512;            // float [2 buffers][2 halves][128] maxima
+    static constexpr int OFF_XL = OFF_XM + 2048;           // float [2 halves][128] row sums
+    static constexpr int OFF_BAR = OFF_XL + 1024;
+    // q_ready; k_full, k_empty, k_tma [NK]; v_full, v_empty, v_tma [NV]; ci_full, ci_empty [kNCI];
+    // s_full, p_full, xm_bar [2]; pv_done; o_final; xl_bar
+    static constexpr int NBAR = 1 + 3 * NK + 3 * NV + 2 * kNCI + 6 + 3;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int SMEM = BYTES + 1024;              // slack for 1024-byte alignment
+    static_assert(CHUNKS * 128 * 16 == kTile * D, "converter chunk split");
 };
 
 struct AttnParams {
-    // cached keys / values
-    const int8_t *k8, *v8;
-    const float *ks, *vs;
-    const int8_t *hk8, *hv8;
-    const float *hks, *hvs;
-    int64_t ring_tokens, first_tok, head_rows;
+    const float *ksl, *vsl;     // retained-history scales in age order, [H][hist_stride]
+    const float *hks, *hvs;     // description-head scales, [H][head_rows]
+    int64_t hist_stride, head_rows;
     // mask buffer
     const uint8_t *mask;
     const int4 *lists;
@@ -74,7 +87,9 @@ struct AttnParams {
     MaskHeader expect;
     int32_t sparse;
     int32_t n_pairs;
-    // shapes
+    // queries and shapes
+    const __nv_bfloat16 *q;
+    int64_t tok_stride, head_stride;
     int32_t H, T;
     int64_t Nq;
     float scale_log2;           // softmax_scale * log2(e)
@@ -116,18 +131,6 @@ __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // 16 int8 codes -> 16 exact fp16 values (two 16-byte chunks).  Each biased byte u = b + 128 becomes
 // the low byte of the fp16 pattern 0x64uu = 1024 + u; one packed add of -1152 leaves b exactly.
 __device__ __forceinline__ void i8x16_to_f16(const uint4 &w, uint4 &lo, uint4 &hi) {
@@ -143,13 +146,13 @@ __device__ __forceinline__ void i8x16_to_f16(const uint4 &w, uint4 &lo, uint4 &h
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// 16 int8 codes times a row scale -> 16 fp16 values.  Each biased byte u becomes the float
-// 2^23 + u (pattern 0x4B0000uu); subtracting 2^23 + 128 leaves the code exactly in fp32, which is
-// multiplied by the scale and rounded once to fp16.
-__device__ __forceinline__ void i8x16_scaled_to_f16(const uint4 &w, float s, uint4 &lo, uint4 &hi) {
+// 16 int8 codes, each times its own scale -> 16 fp16 values (a V^T row chunk: one scale per key).
+// Each biased byte u becomes the float 2^23 + u (pattern 0x4B0000uu); subtracting 2^23 + 128 leaves
+// the code exactly in fp32, which is multiplied by its scale and rounded once to fp16.
+__device__ __forceinline__ void i8x16_keyscaled_to_f16(const uint4 &w, const float4 (&s)[4], uint4 &lo,
+                                                       uint4 &hi) {
     const uint32_t in[4] = {w.x, w.y, w.z, w.w};
     const float2 bias = make_float2(-8388736.0f, -8388736.0f);
-    const float2 sc = make_float2(s, s);
     uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -158,8 +161,8 @@ __device__ __forceinline__ void i8x16_scaled_to_f16(const uint4 &w, float s, uin
                                __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441)));
         float2 b = make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7442)),
                                __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7443)));
-        a = __fmul2_rn(__fadd2_rn(a, bias), sc);
-        b = __fmul2_rn(__fadd2_rn(b, bias), sc);
+        a = __fmul2_rn(__fadd2_rn(a, bias), make_float2(s[i].x, s[i].y));
+        b = __fmul2_rn(__fadd2_rn(b, bias), make_float2(s[i].z, s[i].w));
         o[2 * i] = f16x2_of(a.x, a.y);
         o[2 * i + 1] = f16x2_of(b.x, b.y);
     }
@@ -176,37 +179,43 @@ __device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 &v) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+__device__ __forceinline__ bool is_cached(int kind) { return kind == kKindHist || kind == kKindPriorHead; }
+
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kc,
-                    const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_kt,
-                    const __grid_constant__ CUtensorMap tm_vt, const AttnParams p) {
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_kc, const __grid_constant__ CUtensorMap tm_kt,
+                    const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_vt,
+                    const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_kp,
+                    const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_vp,
+                    const AttnParams p) {
     using C = AttnCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-    uint8_t *sQ = sm + C::OFF_Q;
-    uint8_t *sKV = sm + C::OFF_KV;
+    uint8_t *sK = sm + C::OFF_K;
+    uint8_t *sV = sm + C::OFF_V;
     float *sCS = reinterpret_cast<float *>(sm + C::OFF_CS);
     int2 *sCW = reinterpret_cast<int2 *>(sm + C::OFF_CW);
+    float *sVS = reinterpret_cast<float *>(sm + C::OFF_VS);
+    float *sXM = reinterpret_cast<float *>(sm + C::OFF_XM);
+    float *sXL = reinterpret_cast<float *>(sm + C::OFF_XL);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
-    uint64_t *bar_q = bars;          // Q tiles landed (TMA, bf16)
-    uint64_t *q_ready = bars + 1;    // Q converted to fp16 in place
-    uint64_t *kv_full = bars + 2;
-    uint64_t *kv_empty = kv_full + C::NS;
-    uint64_t *ci_full = kv_empty + C::NS;
-    uint64_t *ci_empty = ci_full + kNCI;
-    uint64_t *s_full = ci_empty + kNCI;
-    uint64_t *p_full = s_full + 2;
-    uint64_t *o_final = p_full + 2;
+    uint64_t *q_ready = bars;
+    uint64_t *k_full = bars + 1, *k_empty = k_full + C::NK, *k_tma = k_empty + C::NK;
+    uint64_t *v_full = k_tma + C::NK, *v_empty = v_full + C::NV, *v_tma = v_empty + C::NV;
+    uint64_t *ci_full = v_tma + C::NV, *ci_empty = ci_full + kNCI;
+    uint64_t *s_full = ci_empty + kNCI, *p_full = s_full + 2, *xm_bar = p_full + 2;
+    uint64_t *pv_done = xm_bar + 2, *o_final = pv_done + 1, *xl_bar = o_final + 1;
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int pair = blockIdx.x;
+    const int qb = blockIdx.x;   // 128-row query block
     const int h = blockIdx.y;
-    const int list_id = p.sparse ? h * p.n_pairs + pair : pair;
+    const int use_bit = (qb & 1) ? kUse1 : kUse0;
+    const int mask_bit = (qb & 1) ? kMask1 : kMask0;
+    const int list_id = p.sparse ? h * p.n_pairs + (qb >> 1) : (qb >> 1);
     const int4 *list = p.lists + (int64_t)list_id * p.expect.list_cap;
 
     // header check (every thread reads the same words; all take the same branch)
@@ -223,23 +232,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int n_tiles = p.counts[list_id];
 
     if (threadIdx.x == 0) {
-        mbar_init(bar_q, 1);
-        mbar_init(q_ready, 1);
-        for (int i = 0; i < C::NS; ++i) {
-            mbar_init(&kv_full[i], 1);
-            mbar_init(&kv_empty[i], 1);
+        mbar_init(q_ready, 8);
+        for (int i = 0; i < C::NK; ++i) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&k_tma[i], 1);
+        }
+        for (int i = 0; i < C::NV; ++i) {
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+            mbar_init(&v_tma[i], 1);
         }
         for (int i = 0; i < kNCI; ++i) {
             mbar_init(&ci_full[i], 1);
             mbar_init(&ci_empty[i], 8);
         }
-        for (int q = 0; q < 2; ++q) {
-            mbar_init(&s_full[q], 1);
-            mbar_init(&p_full[q], 4);
-            mbar_init(&o_final[q], 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&p_full[b], 8);
+            mbar_init(&xm_bar[b], 8);
         }
+        mbar_init(pv_done, 1);
+        mbar_init(o_final, 1);
+        mbar_init(xl_bar, 8);
         misc[1] = 0;
-        for (int i = 0; i < C::NS; ++i) misc[8 + i] = 0;
         fence_mbar_init();
     }
     if (warp == 12) {
@@ -252,322 +268,289 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t tmem = misc[0];
 
     Watchdog wd{p.err, abort_flag, p.timeout_ns, 0};
-    const int64_t qrow0 = (int64_t)pair * 2 * kTile;
+    const int64_t qrow0 = (int64_t)qb * kTile;
 
     if (warp >= 8 && warp < 12) {
-        // ------------------------------------------------------------------ loader warpgroup
+        // ------------------------------------------------------------------ converter warpgroup
+        // Every wait is followed by a named barrier over the 128 converter threads and a read of the
+        // shared abort flag, so all converter threads leave the loop together.
         setmaxnreg_dec<kRegLoader>();
-        // Every wait is followed by a named barrier over the 128 loader threads and a read of the
-        // shared abort flag, so all loader threads leave the loop together.
         wd.where = 3;
         const int t = threadIdx.x - 256;   // 0..127
-        uint32_t tma_pending = 0, tma_par = 0;   // per slot: a TMA was issued / its phase parity
-        if (t == 0) {
-            prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_kc);
-            prefetch_tmap(&tm_vc);
-            mbar_arrive_expect_tx(bar_q, 2 * C::QB);
-#pragma unroll
-            for (int q = 0; q < 2; ++q)
-#pragma unroll
-                for (int hh = 0; hh < C::HALVES; ++hh)
-                    tma_load_3d(sQ + q * C::QB + hh * (kTile * 128), &tm_q, bar_q, hh * 64, h,
-                                (int)(qrow0 + q * kTile));
-        }
-        // Q: bf16 -> fp16 in place (the conversion keeps every element's byte position)
-        mbar_wait(bar_q, 0, wd, 4);
-        named_bar_sync(1, 128);
-        if (!*abort_flag) {
-#pragma unroll 4
-            for (int i = t; i < 2 * C::QB / 16; i += 128) {
-                uint4 *ptr = reinterpret_cast<uint4 *>(sQ) + i;
-                *ptr = bf16x8_to_f16(*ptr);
-            }
-            fence_proxy_async_smem();
-        }
-        named_bar_sync(1, 128);
-        if (t == 0 && !*abort_flag) mbar_arrive(q_ready);
-
-        constexpr int CPR = D / 16;          // 16-byte int8 chunks per row
-        constexpr int RSTEP = 128 / CPR;     // rows covered by the 128 threads in one pass
-        constexpr int NR = 128 / RSTEP;      // rows per thread
-        const int my_chunk = t % CPR;
-        const int my_row0 = t / CPR;
-        const int hh_mine = my_chunk / 4;
-        const int c0_mine = (my_chunk % 4) * 2;
+        uint32_t kpar = 0, vpar = 0;        // per slot: parity of the next INT8 landing
+        int u = 0;                          // index among this block's tiles
         for (int j = 0; j < n_tiles && !*abort_flag; ++j) {
             const int4 e = list[j];
+            if (!(e.x & use_bit)) continue;
             const int kind = e.x & 3;
             const int64_t start = e.y;
             const int count = e.z;
-            const bool cached = kind == kKindHist || kind == kKindPriorHead;
+            const bool cached = is_cached(kind);
             const bool hist = kind == kKindHist;
-            const int8_t *src_k = hist ? p.k8 : p.hk8;
-            const int8_t *src_v = hist ? p.v8 : p.hv8;
-            const float *src_ks = hist ? p.ks : p.hks;
-            const float *src_vs = hist ? p.vs : p.hvs;
-            const int64_t head_base = (int64_t)h * (hist ? p.ring_tokens : p.head_rows);
-            auto cache_row = [&](int r) -> int64_t {  // head-major row index of tile row r
-                const int64_t a = start + r;
-                return head_base + (hist ? (p.first_tok + a) % p.ring_tokens : a);
-            };
-            // raw INT8 loads issued first so that their latency overlaps the slot waits
-            uint4 rk[NR], rv[NR];
-            float svv[NR];
-            if (cached) {
-#pragma unroll
-                for (int i = 0; i < NR; ++i) {
-                    const int r = my_row0 + i * RSTEP;
-                    rk[i] = rv[i] = make_uint4(0, 0, 0, 0);
-                    svv[i] = 0.0f;
-                    if (r < count) {
-                        const int64_t gr = cache_row(r);
-                        rk[i] = __ldg(reinterpret_cast<const uint4 *>(src_k + gr * D) + my_chunk);
-                        rv[i] = __ldg(reinterpret_cast<const uint4 *>(src_v + gr * D) + my_chunk);
-                        svv[i] = __ldg(src_vs + gr);
-                    }
-                }
-            }
-            float cs = 0.0f;
+            float cs = 0.0f, vsc = 0.0f;
             int2 w = make_int2(kAlwaysHi, 0);
             if (t < count) {
                 w = kind == kKindText ? p.txtwin[start + t] : make_int2(0, kAlwaysHi);
-                cs = cached ? __ldg(src_ks + cache_row(t)) * p.scale_log2 : p.scale_log2;
+                cs = p.scale_log2;
+                if (cached) {
+                    const int64_t i = hist ? (int64_t)h * p.hist_stride + start + t : (int64_t)h * p.head_rows + start + t;
+                    cs *= __ldg((hist ? p.ksl : p.hks) + i);
+                    vsc = __ldg((hist ? p.vsl : p.hvs) + i);
+                }
             }
-            const int ci = j % kNCI;
-            const int sk = (2 * j) % C::NS;
-            const int sv = (2 * j + 1) % C::NS;
-            if (mbar_wait(&ci_empty[ci], ((j / kNCI) & 1) ^ 1, wd, 1))
-                mbar_wait(&kv_empty[sk], (((2 * j) / C::NS) & 1) ^ 1, wd, 2);
+            const int ci = u % kNCI;
+            mbar_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, wd, 1);
             named_bar_sync(1, 128);
             if (*abort_flag) break;
             sCS[ci * 128 + t] = cs;
             sCW[ci * 128 + t] = w;
-            uint8_t *dK = sKV + sk * C::SLOT;
-            if (!cached) {
-                if (t == 0) {
-                    const CUtensorMap *m = kind == kKindCur ? &tm_kc : &tm_kt;
-                    mbar_arrive_expect_tx(&kv_full[sk], C::SLOT);
-#pragma unroll
-                    for (int hh = 0; hh < C::HALVES; ++hh)
-                        tma_load_3d(dK + hh * (kTile * 128), m, &kv_full[sk], hh * 64, (int)start, h);
-                    tma_pending |= 1u << sk;
-                    tma_par = (tma_par & ~(1u << sk)) | ((uint32_t)(((2 * j) / C::NS) & 1) << sk);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < NR; ++i) {
-                    const int r = my_row0 + i * RSTEP;
-                    uint4 lo, hi;
-                    i8x16_to_f16(rk[i], lo, hi);
-                    uint8_t *base = dK + hh_mine * (kTile * 128);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = lo;
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = hi;
-                }
-                fence_proxy_async_smem();
-                tma_pending &= ~(1u << sk);
-            }
             named_bar_sync(1, 128);
-            if (t == 0) {
-                mbar_arrive(&ci_full[ci]);
-                if (cached) mbar_arrive(&kv_full[sk]);
-            }
-            mbar_wait(&kv_empty[sv], (((2 * j + 1) / C::NS) & 1) ^ 1, wd, 3);
-            named_bar_sync(1, 128);
-            if (*abort_flag) break;
-            uint8_t *dV = sKV + sv * C::SLOT;
-            if (!cached) {
-                if (t == 0) {
-                    const CUtensorMap *m = kind == kKindCur ? &tm_vc : &tm_vt;
-                    mbar_arrive_expect_tx(&kv_full[sv], C::SLOT);
+            if (t == 0) mbar_arrive(&ci_full[ci]);
+            if (cached) {
+                // keys: INT8 codes in the upper half of the slot -> exact fp16 codes over the slot
+                const int sk = u % C::NK;
+                mbar_wait(&k_tma[sk], (kpar >> sk) & 1u, wd, 2);
+                kpar ^= 1u << sk;
+                named_bar_sync(1, 128);
+                if (*abort_flag) break;
+                uint8_t *slot = sK + sk * C::SLOT;
+                uint4 raw[C::CHUNKS];
 #pragma unroll
-                    for (int hh = 0; hh < C::HALVES; ++hh)
-                        tma_load_3d(dV + hh * (kTile * 128), m, &kv_full[sv], hh * 64, (int)start, h);
-                    tma_pending |= 1u << sv;
-                    tma_par = (tma_par & ~(1u << sv)) | ((uint32_t)(((2 * j + 1) / C::NS) & 1) << sv);
-                }
-            } else {
+                for (int i = 0; i < C::CHUNKS; ++i) raw[i] = reinterpret_cast<const uint4 *>(slot + C::HALF)[t + 128 * i];
+                named_bar_sync(1, 128);   // every code is in registers before any fp16 lands on it
 #pragma unroll
-                for (int i = 0; i < NR; ++i) {
-                    const int r = my_row0 + i * RSTEP;
+                for (int i = 0; i < C::CHUNKS; ++i) {
+                    const int idx = t + 128 * i;
+                    const int row = idx / (D / 16), c = idx % (D / 16);
                     uint4 lo, hi;
-                    i8x16_scaled_to_f16(rv[i], svv[i], lo, hi);
-                    uint8_t *base = dV + hh_mine * (kTile * 128);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine)) = lo;
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, c0_mine + 1)) = hi;
+                    i8x16_to_f16(raw[i], lo, hi);
+                    uint8_t *base = slot + (c / 4) * C::KPANEL;
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(row, (c % 4) * 2)) = lo;
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(row, (c % 4) * 2 + 1)) = hi;
                 }
                 fence_proxy_async_smem();
                 named_bar_sync(1, 128);
-                tma_pending &= ~(1u << sv);
-                if (t == 0) mbar_arrive(&kv_full[sv]);
-            }
-        }
-        // on abort, let this CTA's bulk copies land before the shared memory is released
-        if (*abort_flag && t == 0) {
-            mbar_drain(bar_q, 0, 100000000ull);
+                if (t == 0) mbar_arrive(&k_full[sk]);
+                // values: V^T INT8 rows (one scale per key) -> fp16(code * scale)
+                const int sv = u % C::NV;
+                sVS[t] = vsc;   // readers of the previous tile's scales passed the barrier above
+                mbar_wait(&v_tma[sv], (vpar >> sv) & 1u, wd, 3);
+                vpar ^= 1u << sv;
+                named_bar_sync(1, 128);
+                if (*abort_flag) break;
+                slot = sV + sv * C::SLOT;
 #pragma unroll
-            for (int i = 0; i < C::NS; ++i)
-                if ((tma_pending >> i) & 1u) mbar_drain(&kv_full[i], (tma_par >> i) & 1u, 100000000ull);
+                for (int i = 0; i < C::CHUNKS; ++i) raw[i] = reinterpret_cast<const uint4 *>(slot + C::HALF)[t + 128 * i];
+                const int kc = t % 8;   // this thread's 16-key chunk of every row (idx % 8 == t % 8)
+                float4 s4[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s4[i] = reinterpret_cast<const float4 *>(sVS + kc * 16)[i];
+                named_bar_sync(1, 128);
+#pragma unroll
+                for (int i = 0; i < C::CHUNKS; ++i) {
+                    const int d = (t + 128 * i) / 8;
+                    uint4 lo, hi;
+                    i8x16_keyscaled_to_f16(raw[i], s4, lo, hi);
+                    uint8_t *base = slot + (kc / 4) * C::VPANEL;
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(d, (kc % 4) * 2)) = lo;
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(d, (kc % 4) * 2 + 1)) = hi;
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (t == 0) mbar_arrive(&v_full[sv]);
+            }
+            ++u;
         }
     } else if (warp >= 12) {
-        // ------------------------------------------------------------------ MMA issuer (warp 12)
         setmaxnreg_dec<kRegMma>();
-        wd.where = 4;
         if (warp == 12 && lane == 0) {
-            constexpr uint32_t idesc_qk = idesc_f16_f32(128, 128, false, false);
-            constexpr uint32_t idesc_pv = idesc_f16_f32(128, D, false, true);
-            const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
-            const uint32_t tO[2] = {tmem + 256u, tmem + 384u};
-            const uint32_t q_addr = smem_u32(sQ);
-            const uint32_t kv_addr = smem_u32(sKV);
+            // -------------------------------------------------------------- MMA issuer
+            wd.where = 4;
+            constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);
+            constexpr uint32_t idesc_o = idesc_f16_f32(128, D, false, false);
+            const uint32_t tQ = tmem + kTmQ, tO = tmem + kTmO;
+            const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
             bool ok = mbar_wait(q_ready, 0, wd, 1);
-            int next_s[2];              // next list index whose S_q is to be issued
-            int pend[2] = {-1, -1};     // list index whose PV_q waits for P_q
-            int last_s[2] = {-1, -1}, last_pv[2] = {-1, -1};
-            uint32_t pcount[2] = {0, 0};
-            bool first_pv[2] = {true, true};
-            auto uses = [&](int j, int q) -> bool { return (list[j].x & (q ? kUse1 : kUse0)) != 0; };
-            auto advance = [&](int j, int q) -> int {
-                while (j < n_tiles && !uses(j, q)) ++j;
-                return j;
+            auto issue_pv = [&](int v) -> bool {
+                const int sv = v % C::NV;
+                if (!mbar_wait(&p_full[v & 1], (v >> 1) & 1, wd, 3)) return false;
+                if (!mbar_wait(&v_full[sv], (v / C::NV) & 1, wd, 4)) return false;
+                tc_fence_after();
+                const uint32_t vb = v_addr + sv * C::SLOT;
+                const uint32_t tP = tmem + kTmS + (v & 1) * 128;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    umma_ts(tO, tP + (kk / 4) * 64 + (kk % 4) * 8,
+                            sdesc_sw128(vb + (kk / 4) * C::VPANEL + (kk % 4) * 32, 16, 1024), idesc_o,
+                            (v > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&v_empty[sv]);
+                umma_commit(pv_done);
+                return true;
             };
-            next_s[0] = advance(0, 0);
-            next_s[1] = advance(0, 1);
-            // released[s]: how many uses of K/V slot s this thread has released.  A slot is tested
-            // for use u only when uses 0..u-1 are released, so its full barrier can only be at phase
-            // u or u+1 and the parity test cannot mistake an older completion for use u.
-            uint32_t *released = misc + 8;
-            uint64_t t0 = globaltimer_ns();
-            uint32_t spins = 0;
-            while (ok && (next_s[0] < n_tiles || next_s[1] < n_tiles || pend[0] >= 0 || pend[1] >= 0)) {
-                bool progress = false;
+            int u = 0;
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                if (!(list[j].x & use_bit)) continue;
+                const int sk = u % C::NK;
+                ok = mbar_wait(&k_full[sk], (u / C::NK) & 1, wd, 2);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t kb = k_addr + sk * C::SLOT;
+                const uint32_t tS = tmem + kTmS + (u & 1) * 128;
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    if (pend[q] >= 0) {
-                        const int j = pend[q];
-                        const int sv = (2 * j + 1) % C::NS;
-                        const uint32_t use_v = (uint32_t)((2 * j + 1) / C::NS);
-                        if (released[sv] == use_v && mbar_test(&p_full[q], pcount[q] & 1) &&
-                            mbar_test(&kv_full[sv], use_v & 1)) {
-                            tc_fence_after();
-                            const uint32_t vb = kv_addr + sv * C::SLOT;
-#pragma unroll
-                            for (int kk = 0; kk < 8; ++kk) {
-                                const uint64_t bdesc = sdesc_sw128(vb + kk * 16 * 128, kTile * 128, 1024);
-                                umma_ts(tO[q], tS[q] + kk * 8, bdesc, idesc_pv, (kk > 0 || !first_pv[q]) ? 1u : 0u);
-                            }
-                            first_pv[q] = false;
-                            pcount[q]++;
-                            last_pv[q] = j;
-                            const int o = 1 - q;
-                            if (!uses(j, o) || last_pv[o] >= j) {
-                                umma_commit(&kv_empty[sv]);
-                                released[sv] = use_v + 1;
-                            }
-                            pend[q] = -1;
-                            progress = true;
-                        }
-                    }
-                    if (pend[q] < 0 && next_s[q] < n_tiles) {
-                        const int j = next_s[q];
-                        const int sk = (2 * j) % C::NS;
-                        const uint32_t use_k = (uint32_t)((2 * j) / C::NS);
-                        if (released[sk] == use_k && mbar_test(&kv_full[sk], use_k & 1)) {
-                            tc_fence_after();
-                            const uint32_t kb = kv_addr + sk * C::SLOT;
-                            const uint32_t qb = q_addr + q * C::QB;
-#pragma unroll
-                            for (int kk = 0; kk < C::KSTEPS; ++kk) {
-                                const uint32_t off = (kk / 4) * (kTile * 128) + (kk % 4) * 32;
-                                umma_ss(tS[q], sdesc_sw128(qb + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                                        idesc_qk, kk > 0 ? 1u : 0u);
-                            }
-                            umma_commit(&s_full[q]);
-                            last_s[q] = j;
-                            const int o = 1 - q;
-                            if (!uses(j, o) || last_s[o] >= j) {
-                                umma_commit(&kv_empty[sk]);
-                                released[sk] = use_k + 1;
-                            }
-                            pend[q] = j;
-                            next_s[q] = advance(j + 1, q);
-                            progress = true;
-                        }
-                    }
-                }
-                if (progress) {
-                    spins = 0;
-                    t0 = globaltimer_ns();
-                } else if (++spins > 64) {
-                    spins = 0;
-                    if (*abort_flag) ok = false;
-                    else if (globaltimer_ns() - t0 > p.timeout_ns) {
-                        set_device_error(p.err, NOMAS_ETIMEOUT, 405);
-                        *abort_flag = 1;
-                        ok = false;
-                    }
-                }
+                for (int kk = 0; kk < C::KSTEPS; ++kk)
+                    umma_ts(tS, tQ + kk * 8, sdesc_sw128(kb + (kk / 4) * C::KPANEL + (kk % 4) * 32, 16, 1024),
+                            idesc_s, kk > 0 ? 1u : 0u);
+                umma_commit(&s_full[u & 1]);
+                umma_commit(&k_empty[sk]);
+                if (u >= 1) ok = issue_pv(u - 1);
+                ++u;
             }
-            umma_commit(&o_final[0]);
-            umma_commit(&o_final[1]);
+            if (ok && u >= 1) ok = issue_pv(u - 1);
+            umma_commit(o_final);
             // the MMAs must be complete before the CTA releases TMEM, also on the abort path
-            if (!ok) mbar_drain(&o_final[1], 0, 100000000ull);
+            if (!ok) mbar_drain(o_final, 0, 100000000ull);
+        } else if (warp == 13 && lane == 0) {
+            // -------------------------------------------------------------- TMA producer
+            wd.where = 5;
+            prefetch_tmap(&tm_kc);
+            prefetch_tmap(&tm_vc);
+            prefetch_tmap(&tm_kh);
+            prefetch_tmap(&tm_vh);
+            uint32_t kpar = 0, vpar = 0;             // per slot: parity of the next INT8 landing
+            uint32_t kpend = 0, vpend = 0;           // per slot: a copy was issued
+            uint32_t kwait8 = 0, vwait8 = 0;         // per slot: it signals the INT8 barrier
+            uint32_t kwpar = 0, vwpar = 0;           // per slot: parity of that signal
+            int u = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int4 e = list[j];
+                if (!(e.x & use_bit)) continue;
+                const int kind = e.x & 3;
+                const int start = e.y;
+                const bool cached = is_cached(kind);
+                const bool hist = kind == kKindHist;
+                const int sk = u % C::NK;
+                if (!mbar_wait(&k_empty[sk], ((u / C::NK) & 1) ^ 1, wd, 1)) break;
+                uint8_t *dk = sK + sk * C::SLOT;
+                if (!cached) {
+                    mbar_arrive_expect_tx(&k_full[sk], C::SLOT);
+#pragma unroll
+                    for (int hh = 0; hh < D / 64; ++hh)
+                        tma_load_3d(dk + hh * C::KPANEL, kind == kKindCur ? &tm_kc : &tm_kt, &k_full[sk], hh * 64,
+                                    start, h);
+                    kwait8 &= ~(1u << sk);
+                    kwpar = (kwpar & ~(1u << sk)) | ((uint32_t)((u / C::NK) & 1) << sk);
+                } else {
+                    mbar_arrive_expect_tx(&k_tma[sk], C::HALF);
+                    tma_load_3d(dk + C::HALF, hist ? &tm_kh : &tm_kp, &k_tma[sk], 0, start, h);
+                    kwait8 |= 1u << sk;
+                    kwpar = (kwpar & ~(1u << sk)) | (((kpar >> sk) & 1u) << sk);
+                    kpar ^= 1u << sk;
+                }
+                kpend |= 1u << sk;
+                const int sv = u % C::NV;
+                if (!mbar_wait(&v_empty[sv], ((u / C::NV) & 1) ^ 1, wd, 2)) break;
+                uint8_t *dv = sV + sv * C::SLOT;
+                if (!cached) {
+                    mbar_arrive_expect_tx(&v_full[sv], C::SLOT);
+#pragma unroll
+                    for (int pp = 0; pp < 2; ++pp)
+                        tma_load_3d(dv + pp * C::VPANEL, kind == kKindCur ? &tm_vc : &tm_vt, &v_full[sv],
+                                    start + 64 * pp, 0, h);
+                    vwait8 &= ~(1u << sv);
+                    vwpar = (vwpar & ~(1u << sv)) | ((uint32_t)((u / C::NV) & 1) << sv);
+                } else {
+                    mbar_arrive_expect_tx(&v_tma[sv], C::HALF);
+                    tma_load_3d(dv + C::HALF, hist ? &tm_vh : &tm_vp, &v_tma[sv], start, 0, h);
+                    vwait8 |= 1u << sv;
+                    vwpar = (vwpar & ~(1u << sv)) | (((vpar >> sv) & 1u) << sv);
+                    vpar ^= 1u << sv;
+                }
+                vpend |= 1u << sv;
+                ++u;
+            }
+            // the bulk copies must land before the CTA's shared memory is released (a no-op unless
+            // this CTA is aborting)
+            for (int i = 0; i < C::NK; ++i)
+                if ((kpend >> i) & 1u) mbar_drain(((kwait8 >> i) & 1u) ? &k_tma[i] : &k_full[i], (kwpar >> i) & 1u, 100000000ull);
+            for (int i = 0; i < C::NV; ++i)
+                if ((vpend >> i) & 1u) mbar_drain(((vwait8 >> i) & 1u) ? &v_tma[i] : &v_full[i], (vwpar >> i) & 1u, 100000000ull);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ softmax warpgroups
         // Waits are made warp-uniform (__all_sync) because tcgen05.ld/st are warp-collective.
         setmaxnreg_inc<kRegSoftmax>();
-        const int q = warp >> 2;
-        wd.where = 1 + q;
-        const int r = (warp & 3) * 32 + lane;
-        const int64_t row = qrow0 + q * kTile + r;
-        const int frame = (int)((row < p.Nq ? row : 0) / p.T);
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_base + (uint32_t)(q * 128);
-        const uint32_t tO = tmem + lane_base + 256u + (uint32_t)(q * 128);
+        const int half = warp >> 2;         // key columns [64 * half, 64 * half + 64) of each tile
+        const int g = warp & 3;             // TMEM lane group
+        wd.where = 1 + half;
+        const int r = g * 32 + lane;
+        const int64_t row = qrow0 + r;
+        const bool row_ok = row < p.Nq;
+        const int frame = (int)((row_ok ? row : 0) / p.T);
+        const uint32_t lane_base = (uint32_t)(g * 32) << 16;
+        constexpr int DH = D / 2;           // head-dim elements of Q and O handled by this half
+        // Q row r, elements [half * DH, half * DH + DH) -> fp16 pairs in TMEM
+        {
+            uint32_t qp[DH / 2];
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.q + (row_ok ? row : 0) * p.tok_stride +
+                                                               (int64_t)h * p.head_stride + half * DH);
+#pragma unroll
+            for (int i = 0; i < DH / 8; ++i) {
+                const uint4 v = row_ok ? bf16x8_to_f16(__ldg(src + i)) : make_uint4(0, 0, 0, 0);
+                qp[4 * i] = v.x;
+                qp[4 * i + 1] = v.y;
+                qp[4 * i + 2] = v.z;
+                qp[4 * i + 3] = v.w;
+            }
+            const uint32_t tq = tmem + lane_base + kTmQ + (uint32_t)(half * DH / 2);
+            if constexpr (DH / 2 == 32) {
+                tmem_st32(tq, qp);
+            } else {
+                tmem_st16(tq, qp);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(q_ready);
+        }
         float m_used = -INFINITY;
         float l = 0.0f;
-        uint32_t k = 0;
+        int u = 0;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             const int4 e = list[j];
-            const int ci = j % kNCI;
-            ok = __all_sync(0xffffffffu, mbar_wait(&ci_full[ci], (j / kNCI) & 1, wd, 1));
+            if (!(e.x & use_bit)) continue;
+            const int ci = u % kNCI;
+            const int b = u & 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&ci_full[ci], (u / kNCI) & 1, wd, 1));
             if (!ok) break;
-            const bool used = (e.x & (q ? kUse1 : kUse0)) != 0;
-            if (!used) {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ci_empty[ci]);
-                continue;
-            }
-            const bool masked = (e.x & (q ? kMask1 : kMask0)) != 0;
-            const bool cached = (e.x & 3) == kKindHist || (e.x & 3) == kKindPriorHead;
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[q], k & 1, wd, 2));
+            const bool masked = (e.x & mask_bit) != 0;
+            const bool cached = is_cached(e.x & 3);
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (u >> 1) & 1, wd, 2));
             if (!ok) break;
             tc_fence_after();
-            float s[128];
-#pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) tmem_ld32f_sync(tS + c4 * 32, &s[c4 * 32]);
+            const uint32_t tS = tmem + lane_base + kTmS + (uint32_t)(b * 128 + half * 64);
+            float s[64];
+            tmem_ld64f_sync(tS, s);
             // cached keys: apply the per-key scale (which carries softmax scale * log2 e) to the score
             if (cached) {
-                const float4 *cs4 = reinterpret_cast<const float4 *>(sCS + ci * 128);
+                const float4 *cs4 = reinterpret_cast<const float4 *>(sCS + ci * 128 + half * 64);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     if ((i & 7) == 0) asm volatile("" ::: "memory");   // bound how far loads are hoisted
                     const float4 v = cs4[i];
                     const float2 a = __fmul2_rn(make_float2(s[4 * i], s[4 * i + 1]), make_float2(v.x, v.y));
-                    const float2 b = __fmul2_rn(make_float2(s[4 * i + 2], s[4 * i + 3]), make_float2(v.z, v.w));
+                    const float2 c = __fmul2_rn(make_float2(s[4 * i + 2], s[4 * i + 3]), make_float2(v.z, v.w));
                     s[4 * i] = a.x;
                     s[4 * i + 1] = a.y;
-                    s[4 * i + 2] = b.x;
-                    s[4 * i + 3] = b.y;
+                    s[4 * i + 2] = c.x;
+                    s[4 * i + 3] = c.y;
                 }
             }
             if (masked) {
-                const int4 *cw = reinterpret_cast<const int4 *>(sCW + ci * 128);
+                const int4 *cw = reinterpret_cast<const int4 *>(sCW + ci * 128 + half * 64);
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
+                for (int i = 0; i < 32; ++i) {
                     if ((i & 7) == 0) asm volatile("" ::: "memory");
                     const int4 w = cw[i];   // windows of columns 2i and 2i+1
                     s[2 * i] = (w.x <= frame && frame < w.y) ? s[2 * i] : -INFINITY;
@@ -576,13 +559,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_empty[ci]);
-            float mt = max3(s[0], s[1], s[2]);
+            // row maximum over this half (two independent max3 chains), then swapped with the other half
+            float m0 = max3(s[0], s[1], s[2]), m1 = max3(s[32], s[33], s[34]);
 #pragma unroll
-            for (int c = 3; c < 127; c += 2) mt = max3(mt, s[c], s[c + 1]);
-            mt = fmaxf(mt, s[127]);
-            // log2 domain: cached scores are already scaled, bf16-source scores get the uniform scale
+            for (int c = 3; c < 31; c += 2) {
+                m0 = max3(m0, s[c], s[c + 1]);
+                m1 = max3(m1, s[32 + c], s[33 + c]);
+            }
+            const float pm = fmaxf(fmaxf(m0, s[31]), fmaxf(m1, s[63]));
+            sXM[(b * 2 + half) * 128 + r] = pm;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&xm_bar[b]);
+            ok = __all_sync(0xffffffffu, mbar_wait(&xm_bar[b], (u >> 1) & 1, wd, 3));
+            if (!ok) break;
+            const float po = sXM[(b * 2 + (half ^ 1)) * 128 + r];
+            // log2 domain: cached scores are already scaled, bf16-source scores take the uniform scale
+            // (a positive factor commutes with the maximum exactly); both halves compute the same values
             const float cmul = cached ? 1.0f : p.scale_log2;
-            mt *= cmul;
+            const float mt = fmaxf(pm, po) * cmul;
             const float m_new = fmaxf(m_used, mt);
             const bool grow = m_new > m_used + kRescaleThreshold;   // false while both are -inf
             const bool need_o = grow && m_used != -INFINITY;
@@ -591,26 +585,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float off = (m_used == -INFINITY) ? 0.0f : m_used;
             const float2 cm2 = make_float2(cmul, cmul);
             const float2 no2 = make_float2(-off, -off);
-            float2 acc = make_float2(0.0f, 0.0f);
+            float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
-            for (int qt = 0; qt < 4; ++qt) {
+            for (int qt = 0; qt < 2; ++qt) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const float2 a = __ffma2_rn(make_float2(s[qt * 32 + c], s[qt * 32 + c + 1]), cm2, no2);
                     const float p0 = ex2(a.x);
                     const float p1 = ex2(a.y);
-                    acc = __fadd2_rn(acc, make_float2(p0, p1));
+                    acc[(c >> 1) & 1] = __fadd2_rn(acc[(c >> 1) & 1], make_float2(p0, p1));
                     pk[c / 2] = f16x2_of(p0, p1);
                 }
                 tmem_st16(tS + qt * 16, pk);
             }
-            l = l * f + (acc.x + acc.y);
-            // rescale O_q in TMEM (rare: only when some row's maximum grew past the threshold);
-            // done after P so that the scores are no longer live
+            l = l * f + ((acc[0].x + acc[1].x) + (acc[0].y + acc[1].y));
+            // rescale this half of O (rare: only when some row's maximum grew past the threshold) once
+            // PV of the previous tile is complete; S_u's completion already implies PV_{u-2}'s
             if (__any_sync(0xffffffffu, need_o)) {
+                ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (u - 1) & 1, wd, 4));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(half * DH);
 #pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                for (int c0 = 0; c0 < DH; c0 += 32) {
                     uint32_t rr[32];
                     tmem_ld32_sync(tO + c0, rr);
 #pragma unroll
@@ -621,30 +619,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[q]);
-            ++k;
+            if (lane == 0) mbar_arrive(&p_full[b]);
+            ++u;
         }
-        // epilogue: O / l
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_final[q], 0, wd, 3));
+        // epilogue: the two halves' row sums, then O / l over this half's columns
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_final, 0, wd, 5));
+        if (ok) {
+            sXL[half * 128 + r] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xl_bar);
+            ok = __all_sync(0xffffffffu, mbar_wait(xl_bar, 0, wd, 6));
+        }
         if (ok) {
             tc_fence_after();
-            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            float *dst = p.out + (row * p.H + h) * (int64_t)D;
+            const float lt = l + sXL[(half ^ 1) * 128 + r];
+            const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
+            float *dst = p.out + (row * p.H + h) * (int64_t)D + half * DH;
+            const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(half * DH);
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 0; c0 < DH; c0 += 32) {
                 uint32_t rr[32];
                 tmem_ld32_sync(tO + c0, rr);
-                if (row < p.Nq) {
+                if (row_ok) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 4) {
-                        const float4 v = make_float4(__uint_as_float(rr[i]) * inv, __uint_as_float(rr[i + 1]) * inv,
-                                                     __uint_as_float(rr[i + 2]) * inv, __uint_as_float(rr[i + 3]) * inv);
+                        float4 v = make_float4(__uint_as_float(rr[i]) * inv, __uint_as_float(rr[i + 1]) * inv,
+                                               __uint_as_float(rr[i + 2]) * inv, __uint_as_float(rr[i + 3]) * inv);
+                        if (lt == 0.0f) v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);   // no visible key at all
                         *reinterpret_cast<float4 *>(dst + c0 + i) = v;
                     }
                 }
             }
-            if (p.lse && row < p.Nq)
-                p.lse[(int64_t)h * p.Nq + row] = (m_used + log2f(l)) * 0.69314718055994530942f;
+            if (p.lse && row_ok && half == 0)
+                p.lse[(int64_t)h * p.Nq + row] = (m_used + log2f(lt)) * 0.69314718055994530942f;
         }
     }
 
@@ -656,20 +663,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 }
 
-// bf16 [n][H][D] (token / head strides in elements) -> fp16 [H][n][D], for up to four tensors.
+// ---------------------------------------------------------------------------------------------
+// Pre-pass (HBM-bound): operand copies in the layouts the attention kernel's TMA boxes read.
+// ---------------------------------------------------------------------------------------------
+
+// bf16 [n][H][D] (token / head strides in elements) -> fp16 [H][n][D], for up to two tensors.
 struct F16Job {
     const __nv_bfloat16 *src;
     __half *dst;
     int64_t n;
 };
 struct F16Jobs {
-    F16Job job[4];
+    F16Job job[2];
     int32_t n_jobs;
     int32_t H, D;
     int64_t tok_stride, head_stride;
 };
 
-__global__ void __launch_bounds__(256) values_f16_kernel(F16Jobs jobs) {
+__global__ void __launch_bounds__(256) keys_f16_kernel(F16Jobs jobs) {
     const int cpr = jobs.D / 8;   // 16-byte chunks per row
     for (int jb = 0; jb < jobs.n_jobs; ++jb) {
         const F16Job J = jobs.job[jb];
@@ -684,6 +695,118 @@ __global__ void __launch_bounds__(256) values_f16_kernel(F16Jobs jobs) {
                                                                   (int64_t)h * jobs.head_stride) + c);
             reinterpret_cast<uint4 *>(J.dst + rowi * jobs.D)[c] = bf16x8_to_f16(v);
         }
+    }
+}
+
+// bf16 [n][H][D] -> fp16 V^T [H][D][np] (np = n rounded up to 8; the padding is zero), for up to
+// two tensors.  One block transposes 64 tokens x D of one head through shared memory.
+struct VtJob {
+    const __nv_bfloat16 *src;
+    __half *dst;
+    int64_t n, np;
+};
+struct VtJobs {
+    VtJob job[2];
+    int32_t H, D;
+    int64_t tok_stride, head_stride;
+};
+
+__global__ void __launch_bounds__(256) values_t16_kernel(VtJobs jobs) {
+    __shared__ __align__(16) __half tile[64][128 + 8];
+    const VtJob J = jobs.job[blockIdx.z];
+    const int h = blockIdx.y;
+    const int64_t t0 = (int64_t)blockIdx.x * 64;
+    if (t0 >= J.np) return;
+    const int D = jobs.D;
+    const int cpr = D / 8;
+    for (int i = threadIdx.x; i < 64 * cpr; i += blockDim.x) {
+        const int r = i / cpr, c = i % cpr;
+        const int64_t t = t0 + r;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (t < J.n)
+            v = bf16x8_to_f16(__ldg(reinterpret_cast<const uint4 *>(J.src + t * jobs.tok_stride +
+                                                                    (int64_t)h * jobs.head_stride) + c));
+        *reinterpret_cast<uint4 *>(&tile[r][c * 8]) = v;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < D * 8; i += blockDim.x) {
+        const int d = i / 8, c = i % 8;   // row d, tokens [t0 + 8c, t0 + 8c + 8)
+        const int64_t t = t0 + c * 8;
+        if (t >= J.np) continue;
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const __half a = tile[c * 8 + 2 * k][d], b = tile[c * 8 + 2 * k + 1][d];
+            w[k] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+        }
+        *reinterpret_cast<uint4 *>(J.dst + ((int64_t)h * D + d) * J.np + t) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// INT8 history in age order for the attention kernel's TMA boxes:
+//   z = 0: ring rows of the retained history -> K8 rows [H][Lh][D], V^T [H][D][lhp] (lhp = Lh rounded
+//          up to 16, zero padding), key / value scales [H][lhp];
+//   z = 1: description-head store rows [0, Lp) -> V^T [H][D][lpp] (keys and scales are read in place).
+struct HistPrep {
+    const int8_t *k8, *v8, *hv8;
+    const float *ks, *vs;
+    int8_t *k8l, *v8t, *hv8t;
+    float *ksl, *vsl;
+    int64_t ring_tokens, first_tok, Lh, lhp, Lp, lpp, head_rows;
+    int32_t H, D;
+};
+
+__global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
+    __shared__ __align__(16) int8_t tile[64][128 + 16];
+    const bool heads = blockIdx.z == 1;
+    const int h = blockIdx.y;
+    const int64_t n = heads ? P.Lp : P.Lh, np = heads ? P.lpp : P.lhp;
+    const int64_t t0 = (int64_t)blockIdx.x * 64;
+    if (t0 >= np) return;
+    const int D = P.D;
+    const int cpr = D / 16;
+    auto src_row = [&](int64_t a) -> int64_t {
+        return heads ? (int64_t)h * P.head_rows + a : (int64_t)h * P.ring_tokens + (P.first_tok + a) % P.ring_tokens;
+    };
+    for (int i = threadIdx.x; i < 64 * cpr; i += blockDim.x) {
+        const int r = i / cpr, c = i % cpr;
+        const int64_t a = t0 + r;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (a < n) {
+            const int64_t sr = src_row(a);
+            v = __ldg(reinterpret_cast<const uint4 *>((heads ? P.hv8 : P.v8) + sr * D) + c);
+            if (!heads)
+                reinterpret_cast<uint4 *>(P.k8l + ((int64_t)h * P.Lh + a) * D)[c] =
+                    __ldg(reinterpret_cast<const uint4 *>(P.k8 + sr * D) + c);
+        }
+        *reinterpret_cast<uint4 *>(&tile[r][c * 16]) = v;
+    }
+    if (!heads && threadIdx.x < 64) {
+        const int64_t a = t0 + threadIdx.x;
+        if (a < np) {
+            float ks = 0.0f, vs = 0.0f;
+            if (a < n) {
+                const int64_t sr = src_row(a);
+                ks = __ldg(P.ks + sr);
+                vs = __ldg(P.vs + sr);
+            }
+            P.ksl[(int64_t)h * P.lhp + a] = ks;
+            P.vsl[(int64_t)h * P.lhp + a] = vs;
+        }
+    }
+    __syncthreads();
+    int8_t *dst = heads ? P.hv8t : P.v8t;
+    for (int i = threadIdx.x; i < D * 4; i += blockDim.x) {
+        const int d = i / 4, c = i % 4;   // row d, tokens [t0 + 16c, t0 + 16c + 16)
+        const int64_t t = t0 + c * 16;
+        if (t >= np) continue;
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            w[k] = (uint32_t)(uint8_t)tile[c * 16 + 4 * k][d] | ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 1][d] << 8) |
+                   ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 2][d] << 16) |
+                   ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 3][d] << 24);
+        *reinterpret_cast<uint4 *>(dst + ((int64_t)h * D + d) * np + t) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -711,16 +834,14 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D tiled map with 128B swizzle.  dims / strides are innermost first (strides in bytes for
-// dims 1 and 2); the box's inner extent is 64 elements (128 bytes).
+// 3-D tiled map.  dims / strides are innermost first (strides in bytes for dims 1 and 2).
 static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, const cuuint64_t dims[3],
-                     const cuuint64_t strides[2], const cuuint32_t box[3]) {
+                     const cuuint64_t strides[2], const cuuint32_t box[3], CUtensorMapSwizzle swz) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint32_t es[3] = {1, 1, 1};
     const CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                           swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         char msg[160];
         std::snprintf(msg, sizeof(msg), "dims %llu x %llu x %llu, strides %llu %llu", (unsigned long long)dims[0],
@@ -732,20 +853,41 @@ static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, c
     return true;
 }
 
-// Workspace: fp16 [H][n][D] copies of the current segment's K, V and the text's K, V.
+static int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+// Workspace regions (256-byte aligned), sized for the largest history the cache can retain so that
+// the size does not depend on the cache state:
+//   kc, kt   fp16 [H][n][D]       current-segment / text keys
+//   vc, vt   fp16 [H][D][np8]     current-segment / text values, transposed
+//   k8l      int8 [H][Lh][D]      retained-history keys in age order
+//   v8t      int8 [H][D][lhp]     retained-history values, transposed
+//   ksl, vsl fp32 [H][lhp]        their scales
+//   hv8t     int8 [H][D][lpp]     description-head values, transposed
 struct WsLayout {
-    size_t off[4];
-    size_t total;
+    size_t kc, kt, vc, vt, k8l, v8t, ksl, vsl, hv8t, total;
 };
 static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
+    const auto &d = c->d;
+    const int64_t H = d.heads, D = d.head_dim;
+    const int64_t frames = d.window_frames > 0 && d.window_frames < d.capacity_frames ? d.window_frames : d.capacity_frames;
+    const int64_t lh = frames * d.tokens_per_frame, lhp = round_up(lh, 16);
+    const int64_t lpp = round_up(d.head_store_tokens, 16);
     WsLayout w;
-    const size_t row = (size_t)c->d.heads * c->d.head_dim * 2;
     size_t off = 0;
-    const int64_t n[4] = {nq, nq, lt, lt};
-    for (int i = 0; i < 4; ++i) {
-        w.off[i] = off;
-        off += ((size_t)n[i] * row + 255) / 256 * 256;
-    }
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += (bytes + 255) / 256 * 256;
+        return o;
+    };
+    w.kc = take((size_t)H * nq * D * 2);
+    w.kt = take((size_t)H * lt * D * 2);
+    w.vc = take((size_t)H * D * round_up(nq, 8) * 2);
+    w.vt = take((size_t)H * D * round_up(lt, 8) * 2);
+    w.k8l = take((size_t)H * lh * D);
+    w.v8t = take((size_t)H * D * lhp);
+    w.ksl = take((size_t)H * lhp * 4);
+    w.vsl = take((size_t)H * lhp * 4);
+    w.hv8t = take((size_t)H * D * lpp);
     w.total = off;
     return w;
 }
@@ -761,7 +903,8 @@ static int launch_attn(const AttnParams &p, dim3 grid, const CUtensorMap *maps, 
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(attn smem)", (int)e, cudaGetErrorString(e));
         attr_set = true;
     }
-    attn_fwd_kernel<D><<<grid, kAttnThreads, AttnCfg<D>::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);
+    attn_fwd_kernel<D><<<grid, kAttnThreads, AttnCfg<D>::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                                      maps[5], maps[6], maps[7], p);
     return check_launch("attn_fwd_kernel launch");
 }
 
@@ -795,60 +938,111 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     const int H = d.heads;
     if (bind_device(c)) return NOMAS_ECUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t Nq = lay.n_query, Lt = lay.text_tokens, Lh = lay.history_tokens, Lp = lay.head_tokens;
+    const int64_t nqp = round_up(Nq, 8), ltp = round_up(Lt, 8), lhp = round_up(Lh, 16), lpp = round_up(Lp, 16);
 
-    // fp16 copies of the current segment's and the text's K / V (HBM-bound pre-pass)
-    const WsLayout ws = ws_layout(c, lay.n_query, lay.text_tokens);
+    // ---- pre-pass: fp16 keys, transposed fp16 values, INT8 history in age order
+    const WsLayout ws = ws_layout(c, Nq, Lt);
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
-    F16Jobs jobs{};
-    jobs.H = H;
-    jobs.D = D;
-    jobs.tok_stride = tok_stride;
-    jobs.head_stride = head_stride;
-    const void *srcs[4] = {kcur, vcur, ktxt, vtxt};
-    const int64_t ns[4] = {lay.n_query, lay.n_query, lay.text_tokens, lay.text_tokens};
-    for (int i = 0; i < 4; ++i) {
-        if (ns[i] == 0) continue;
-        F16Job &J = jobs.job[jobs.n_jobs++];
-        J.src = static_cast<const __nv_bfloat16 *>(srcs[i]);
-        J.dst = reinterpret_cast<__half *>(wsb + ws.off[i]);
-        J.n = ns[i];
-    }
     {
-        const int64_t chunks = (2 * lay.n_query + 2 * lay.text_tokens) * H * (D / 8);
-        int64_t blocks = (chunks + 255) / 256;
+        F16Jobs jobs{};
+        jobs.H = H;
+        jobs.D = D;
+        jobs.tok_stride = tok_stride;
+        jobs.head_stride = head_stride;
+        jobs.job[jobs.n_jobs++] = F16Job{static_cast<const __nv_bfloat16 *>(kcur), reinterpret_cast<__half *>(wsb + ws.kc), Nq};
+        if (Lt > 0)
+            jobs.job[jobs.n_jobs++] =
+                F16Job{static_cast<const __nv_bfloat16 *>(ktxt), reinterpret_cast<__half *>(wsb + ws.kt), Lt};
+        int64_t blocks = ((Nq + Lt) * H * (D / 8) + 255) / 256;
         if (blocks > 148 * 16) blocks = 148 * 16;
-        values_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(jobs);
-        rc = check_launch("values_f16_kernel launch");
-        if (rc) return rc;
-    }
+        keys_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(jobs);
+        if ((rc = check_launch("keys_f16_kernel launch"))) return rc;
 
-    CUtensorMap maps[5];
-    {
-        const cuuint64_t dq[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)lay.n_query};
-        const cuuint64_t sq[2] = {(cuuint64_t)head_stride * 2, (cuuint64_t)tok_stride * 2};
-        const cuuint32_t bq[3] = {64, 1, (cuuint32_t)kTile};
-        if (!make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, dq, sq, bq)) return NOMAS_ECUDA;
-        const cuuint32_t bk[3] = {64, (cuuint32_t)kTile, 1};
-        for (int i = 0; i < 4; ++i) {
-            const int64_t n = ns[i] > 0 ? ns[i] : 1;
-            const size_t off = ns[i] > 0 ? ws.off[i] : ws.off[0];
-            const cuuint64_t dk[3] = {(cuuint64_t)D, (cuuint64_t)n, (cuuint64_t)H};
-            const cuuint64_t sk[2] = {(cuuint64_t)D * 2, (cuuint64_t)n * D * 2};
-            if (!make_map(&maps[1 + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, wsb + off, dk, sk, bk)) return NOMAS_ECUDA;
-        }
+        VtJobs vj{};
+        vj.H = H;
+        vj.D = D;
+        vj.tok_stride = tok_stride;
+        vj.head_stride = head_stride;
+        vj.job[0] = VtJob{static_cast<const __nv_bfloat16 *>(vcur), reinterpret_cast<__half *>(wsb + ws.vc), Nq, nqp};
+        vj.job[1] = VtJob{static_cast<const __nv_bfloat16 *>(Lt > 0 ? vtxt : vcur), reinterpret_cast<__half *>(wsb + ws.vt),
+                          Lt, ltp};
+        const dim3 vgrid((unsigned)((nqp > ltp ? nqp : ltp) + 63) / 64, (unsigned)H, Lt > 0 ? 2u : 1u);
+        values_t16_kernel<<<vgrid, 256, 0, st>>>(vj);
+        if ((rc = check_launch("values_t16_kernel launch"))) return rc;
     }
     const HistView hv = hist_view(c);
+    if (Lh > 0 || Lp > 0) {
+        HistPrep hp{};
+        hp.k8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_K8]);
+        hp.v8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_V8]);
+        hp.hv8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_HV8]);
+        hp.ks = static_cast<const float *>(c->buf[NOMAS_BUF_KS]);
+        hp.vs = static_cast<const float *>(c->buf[NOMAS_BUF_VS]);
+        hp.k8l = reinterpret_cast<int8_t *>(wsb + ws.k8l);
+        hp.v8t = reinterpret_cast<int8_t *>(wsb + ws.v8t);
+        hp.hv8t = reinterpret_cast<int8_t *>(wsb + ws.hv8t);
+        hp.ksl = reinterpret_cast<float *>(wsb + ws.ksl);
+        hp.vsl = reinterpret_cast<float *>(wsb + ws.vsl);
+        hp.ring_tokens = hv.ring_tokens;
+        hp.first_tok = hv.first_tok;
+        hp.Lh = Lh;
+        hp.lhp = lhp;
+        hp.Lp = Lp;
+        hp.lpp = lpp;
+        hp.head_rows = d.head_store_tokens;
+        hp.H = H;
+        hp.D = D;
+        const int64_t nmax = lhp > lpp ? lhp : lpp;
+        const dim3 hgrid((unsigned)((nmax + 63) / 64), (unsigned)H, 2u);
+        hist_prep_kernel<<<hgrid, 256, 0, st>>>(hp);
+        if ((rc = check_launch("hist_prep_kernel launch"))) return rc;
+    }
+
+    // ---- tensor maps (an extent of zero gets a one-row map that no tile reads)
+    CUtensorMap maps[8];
+    {
+        const CUtensorMapDataType F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16, U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+        const cuuint32_t bk[3] = {64, (cuuint32_t)kTile, 1};        // K: 64 columns x 128 keys
+        const cuuint32_t bv[3] = {64, (cuuint32_t)D, 1};            // V^T: 64 keys x D rows
+        const cuuint32_t bk8[3] = {(cuuint32_t)D, (cuuint32_t)kTile, 1};
+        const cuuint32_t bv8[3] = {(cuuint32_t)kTile, (cuuint32_t)D, 1};
+        auto kmap16 = [&](CUtensorMap *m, size_t off, int64_t n) {
+            const int64_t nn = n > 0 ? n : 1;
+            const cuuint64_t dm[3] = {(cuuint64_t)D, (cuuint64_t)nn, (cuuint64_t)H};
+            const cuuint64_t sd[2] = {(cuuint64_t)D * 2, (cuuint64_t)nn * D * 2};
+            return make_map(m, F16, wsb + off, dm, sd, bk, CU_TENSOR_MAP_SWIZZLE_128B);
+        };
+        auto vmap16 = [&](CUtensorMap *m, size_t off, int64_t n, int64_t np) {
+            const int64_t nn = n > 0 ? n : 1, pp = np > 0 ? np : 8;
+            const cuuint64_t dm[3] = {(cuuint64_t)nn, (cuuint64_t)D, (cuuint64_t)H};
+            const cuuint64_t sd[2] = {(cuuint64_t)pp * 2, (cuuint64_t)D * pp * 2};
+            return make_map(m, F16, wsb + off, dm, sd, bv, CU_TENSOR_MAP_SWIZZLE_128B);
+        };
+        auto kmap8 = [&](CUtensorMap *m, const void *base, int64_t n, int64_t head_stride_rows) {
+            const int64_t nn = n > 0 ? n : 1;
+            const cuuint64_t dm[3] = {(cuuint64_t)D, (cuuint64_t)nn, (cuuint64_t)H};
+            const cuuint64_t sd[2] = {(cuuint64_t)D, (cuuint64_t)(head_stride_rows > 0 ? head_stride_rows : 1) * D};
+            return make_map(m, U8, base, dm, sd, bk8, CU_TENSOR_MAP_SWIZZLE_NONE);
+        };
+        auto vmap8 = [&](CUtensorMap *m, size_t off, int64_t n, int64_t np) {
+            const int64_t nn = n > 0 ? n : 1, pp = np > 0 ? np : 16;
+            const cuuint64_t dm[3] = {(cuuint64_t)nn, (cuuint64_t)D, (cuuint64_t)H};
+            const cuuint64_t sd[2] = {(cuuint64_t)pp, (cuuint64_t)D * pp};
+            return make_map(m, U8, wsb + off, dm, sd, bv8, CU_TENSOR_MAP_SWIZZLE_NONE);
+        };
+        if (!kmap16(&maps[0], ws.kc, Nq) || !kmap16(&maps[1], ws.kt, Lt) || !vmap16(&maps[2], ws.vc, Nq, nqp) ||
+            !vmap16(&maps[3], ws.vt, Lt, ltp) || !kmap8(&maps[4], wsb + ws.k8l, Lh, Lh) ||
+            !kmap8(&maps[5], c->buf[NOMAS_BUF_HK8], Lp, d.head_store_tokens) || !vmap8(&maps[6], ws.v8t, Lh, lhp) ||
+            !vmap8(&maps[7], ws.hv8t, Lp, lpp))
+            return NOMAS_ECUDA;
+    }
     AttnParams p{};
-    p.k8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_K8]);
-    p.v8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_V8]);
-    p.ks = static_cast<const float *>(c->buf[NOMAS_BUF_KS]);
-    p.vs = static_cast<const float *>(c->buf[NOMAS_BUF_VS]);
-    p.hk8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_HK8]);
-    p.hv8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_HV8]);
+    p.ksl = reinterpret_cast<const float *>(wsb + ws.ksl);
+    p.vsl = reinterpret_cast<const float *>(wsb + ws.vsl);
     p.hks = static_cast<const float *>(c->buf[NOMAS_BUF_HKS]);
     p.hvs = static_cast<const float *>(c->buf[NOMAS_BUF_HVS]);
-    p.ring_tokens = hv.ring_tokens;
-    p.first_tok = hv.first_tok;
+    p.hist_stride = lhp;
     p.head_rows = d.head_store_tokens;
     const uint8_t *mb = static_cast<const uint8_t *>(mask_buf);
     p.mask = mb;
@@ -868,14 +1062,17 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     p.expect.keep = lay.keep;
     p.sparse = mode == NOMAS_MODE_SPARSE;
     p.n_pairs = (lay.n_qblocks + 1) / 2;
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.tok_stride = tok_stride;
+    p.head_stride = head_stride;
     p.H = H;
     p.T = d.tokens_per_frame;
-    p.Nq = lay.n_query;
+    p.Nq = Nq;
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.out = out;
     p.lse = lse;
     p.err = static_cast<int *>(c->buf[NOMAS_BUF_ERR]);
     p.timeout_ns = g_timeout_ns;
-    dim3 grid((unsigned)p.n_pairs, (unsigned)H);
+    dim3 grid((unsigned)lay.n_qblocks, (unsigned)H);
     return D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
 }

@@ -194,6 +194,19 @@ __device__ __forceinline__ void tmem_ld32f_sync(uint32_t taddr, float *r) {
         : "r"(taddr)
         : "memory");
 }
+// 64 consecutive TMEM columns of this thread's lane in one load, then one wait.
+__device__ __forceinline__ void tmem_ld64f_sync(uint32_t taddr, float *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : NOMAS_F8(0), NOMAS_F8(8), NOMAS_F8(16), NOMAS_F8(24), NOMAS_F8(32), NOMAS_F8(40), NOMAS_F8(48), NOMAS_F8(56)
+        : "r"(taddr)
+        : "memory");
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "

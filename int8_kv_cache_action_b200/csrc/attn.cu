@@ -5,9 +5,9 @@
 //   warps 0-3   softmax over key columns 0-63 of every S tile (TMEM lanes 0-127, one thread per row)
 //   warps 4-7   softmax over key columns 64-127; the two halves of a row swap their maxima through
 //               shared memory, so both apply the same offset
-//   warps 8-11  converter: per-column key scale and visibility window; an INT8 tile, which TMA lands
-//               in the upper half of its slot, becomes fp16 in place (key codes exactly, values as
-//               fp16(code * scale) with one scale per key)
+//   warps 8-11  converter: per-column key scale, value scale and visibility window; an INT8 tile,
+//               which TMA lands in the upper half of its slot, becomes exact fp16 codes in place;
+//               each warp converts its own rows
 //   warp 12     tcgen05.mma issuer (one thread) and TMEM owner
 //   warp 13     TMA producer (one thread); warps 14-15 idle
 // The register file is split per SM sub-partition (one warp of each warpgroup on each), so the
@@ -29,10 +29,12 @@
 //
 // Precision: every MMA operand is fp16 with fp32 accumulation.  bf16 inputs convert to fp16
 // exactly for magnitudes in [2^-14, 65504] (the supported input range; smaller values keep 2^-24
-// absolute resolution), INT8 key codes are exact and the key scale is applied to the fp32 score,
-// cached values are fp16(code * scale), and P <= 2^8 keeps 11 significant bits.  Softmax uses a
-// lazy rescale: the running offset moves only when the row maximum grows by more than 8 (log2
-// units); O is then rescaled in TMEM once the previous PV has completed.
+// absolute resolution).  INT8 codes enter the tensor core exactly: a key's scale multiplies its fp32
+// score, a value's scale multiplies the fp32 probability before P is rounded to fp16 (so P * v uses
+// the product p * scale * code, rounded once).  Softmax uses a lazy rescale: the running offset
+// moves only when the row maximum grows by more than 6 (log2 units), so p <= 64 and p * scale stays
+// inside fp16 for every input in the supported range (absmax <= 65504 gives scale <= 516); O is
+// then rescaled in TMEM once the previous PV has completed.
 #include <cmath>
 #include <cstdio>
 #include <cuda_fp16.h>
@@ -45,7 +47,7 @@ constexpr int kAttnThreads = 512;
 constexpr int kRegSoftmax = 168, kRegLoader = 112, kRegMma = 64;
 static_assert(2 * kRegSoftmax + kRegLoader + kRegMma == 4 * 128, "register split must equal the launch total");
 constexpr int kNCI = 4;                     // column-info ring depth
-constexpr float kRescaleThreshold = 8.0f;   // log2 units
+constexpr float kRescaleThreshold = 6.0f;   // log2 units: P <= 64
 constexpr uint32_t kTmQ = 0, kTmS = 128, kTmO = 384;
 
 template <int D>
@@ -61,9 +63,9 @@ struct AttnCfg {
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + NK * SLOT;
     static constexpr int OFF_CS = OFF_V + NV * SLOT;       // float [kNCI][128] key scale x log2 e
-    static constexpr int OFF_CW = OFF_CS + kNCI * 512;     // int2  [kNCI][128] key frame windows
-    static constexpr int OFF_VS = OFF_CW + kNCI * 1024;    // float [128] value scales of one tile
-    static constexpr int OFF_XM = OFF_VS + 512;            // float [2 buffers][2 halves][128] maxima
+    static constexpr int OFF_CV = OFF_CS + kNCI * 512;     // float [kNCI][128] value scale
+    static constexpr int OFF_CW = OFF_CV + kNCI * 512;     // int2  [kNCI][128] key frame windows
+    static constexpr int OFF_XM = OFF_CW + kNCI * 1024;    // float [2 buffers][2 halves][128] maxima
     static constexpr int OFF_XL = OFF_XM + 2048;           // float [2 halves][128] row sums
     static constexpr int OFF_BAR = OFF_XL + 1024;
     // q_ready; k_full, k_empty, k_tma [NK]; v_full, v_empty, v_tma [NV]; ci_full, ci_empty [kNCI];
@@ -146,30 +148,6 @@ __device__ __forceinline__ void i8x16_to_f16(const uint4 &w, uint4 &lo, uint4 &h
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// 16 int8 codes, each times its own scale -> 16 fp16 values (a V^T row chunk: one scale per key).
-// Each biased byte u becomes the float 2^23 + u (pattern 0x4B0000uu); subtracting 2^23 + 128 leaves
-// the code exactly in fp32, which is multiplied by its scale and rounded once to fp16.
-__device__ __forceinline__ void i8x16_keyscaled_to_f16(const uint4 &w, const float4 (&s)[4], uint4 &lo,
-                                                       uint4 &hi) {
-    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-    const float2 bias = make_float2(-8388736.0f, -8388736.0f);
-    uint32_t o[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t x = in[i] ^ 0x80808080u;
-        float2 a = make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440)),
-                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441)));
-        float2 b = make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7442)),
-                               __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7443)));
-        a = __fmul2_rn(__fadd2_rn(a, bias), make_float2(s[i].x, s[i].y));
-        b = __fmul2_rn(__fadd2_rn(b, bias), make_float2(s[i].z, s[i].w));
-        o[2 * i] = f16x2_of(a.x, a.y);
-        o[2 * i + 1] = f16x2_of(b.x, b.y);
-    }
-    lo = make_uint4(o[0], o[1], o[2], o[3]);
-    hi = make_uint4(o[4], o[5], o[6], o[7]);
-}
-
 // 8 bf16 -> 8 fp16 (16 bytes in, 16 bytes out).
 __device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 &v) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -180,6 +158,31 @@ __device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 &v) {
 }
 
 __device__ __forceinline__ bool is_cached(int kind) { return kind == kKindHist || kind == kKindPriorHead; }
+
+// Walks a CTA's tile list, each entry loaded two entries ahead of its use.
+struct ListCursor {
+    const int4 *list;
+    int n, j;
+    int4 a, b;
+    __device__ __forceinline__ ListCursor(const int4 *l, int n_) : list(l), n(n_), j(0) {
+        a = n > 0 ? list[0] : make_int4(0, 0, 0, 0);
+        b = n > 1 ? list[1] : make_int4(0, 0, 0, 0);
+    }
+    // the next entry carrying `bit`; false at the end of the list
+    __device__ __forceinline__ bool next(int bit, int4 &e) {
+        while (j < n) {
+            const int4 c = a;
+            a = b;
+            b = (j + 2 < n) ? list[j + 2] : make_int4(0, 0, 0, 0);
+            ++j;
+            if (c.x & bit) {
+                e = c;
+                return true;
+            }
+        }
+        return false;
+    }
+};
 
 template <int D>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -195,8 +198,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t *sK = sm + C::OFF_K;
     uint8_t *sV = sm + C::OFF_V;
     float *sCS = reinterpret_cast<float *>(sm + C::OFF_CS);
+    float *sCV = reinterpret_cast<float *>(sm + C::OFF_CV);
     int2 *sCW = reinterpret_cast<int2 *>(sm + C::OFF_CW);
-    float *sVS = reinterpret_cast<float *>(sm + C::OFF_VS);
     float *sXM = reinterpret_cast<float *>(sm + C::OFF_XM);
     float *sXL = reinterpret_cast<float *>(sm + C::OFF_XL);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
@@ -234,17 +237,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(q_ready, 8);
         for (int i = 0; i < C::NK; ++i) {
-            mbar_init(&k_full[i], 1);
+            mbar_init(&k_full[i], 4);
             mbar_init(&k_empty[i], 1);
             mbar_init(&k_tma[i], 1);
         }
         for (int i = 0; i < C::NV; ++i) {
-            mbar_init(&v_full[i], 1);
+            mbar_init(&v_full[i], 4);
             mbar_init(&v_empty[i], 1);
             mbar_init(&v_tma[i], 1);
         }
         for (int i = 0; i < kNCI; ++i) {
-            mbar_init(&ci_full[i], 1);
+            mbar_init(&ci_full[i], 4);
             mbar_init(&ci_empty[i], 8);
         }
         for (int b = 0; b < 2; ++b) {
@@ -272,52 +275,86 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
     if (warp >= 8 && warp < 12) {
         // ------------------------------------------------------------------ converter warpgroup
-        // Every wait is followed by a named barrier over the 128 converter threads and a read of the
-        // shared abort flag, so all converter threads leave the loop together.
+        // Each warp works on its own rows and signals the barriers itself (full barriers count four
+        // converter warps; the producer adds three arrivals when TMA alone fills a slot).  An INT8
+        // row and the second fp16 panel of the same row occupy the same 128 bytes of the slot, and
+        // the first panel lies below the INT8 half, so for D = 128 (and for V^T at any D) the eight
+        // lanes that share a row only need __syncwarp between reading it and writing over it.  Keys
+        // at D = 64 overlap across warps and take a named barrier, followed by a read of the shared
+        // abort decision so that all converter warps leave together.
         setmaxnreg_dec<kRegLoader>();
         wd.where = 3;
         const int t = threadIdx.x - 256;   // 0..127
-        uint32_t kpar = 0, vpar = 0;        // per slot: parity of the next INT8 landing
-        int u = 0;                          // index among this block's tiles
-        for (int j = 0; j < n_tiles && !*abort_flag; ++j) {
-            const int4 e = list[j];
-            if (!(e.x & use_bit)) continue;
+        const int kc = t % 8;               // V^T: this thread's 16-key chunk in every row it converts
+        struct ColInfo {
+            float cs, vs;
+            int2 w;
+        };
+        // Column info of a tile (key scale x log2 e, value scale, frame window), loaded one tile
+        // ahead of its use.
+        auto col_info = [&](const int4 &e) -> ColInfo {
+            ColInfo ci{0.0f, 0.0f, make_int2(kAlwaysHi, 0)};
             const int kind = e.x & 3;
             const int64_t start = e.y;
-            const int count = e.z;
-            const bool cached = is_cached(kind);
-            const bool hist = kind == kKindHist;
-            float cs = 0.0f, vsc = 0.0f;
-            int2 w = make_int2(kAlwaysHi, 0);
-            if (t < count) {
-                w = kind == kKindText ? p.txtwin[start + t] : make_int2(0, kAlwaysHi);
-                cs = p.scale_log2;
-                if (cached) {
-                    const int64_t i = hist ? (int64_t)h * p.hist_stride + start + t : (int64_t)h * p.head_rows + start + t;
-                    cs *= __ldg((hist ? p.ksl : p.hks) + i);
-                    vsc = __ldg((hist ? p.vsl : p.hvs) + i);
+            if (t < e.z) {
+                ci.w = kind == kKindText ? p.txtwin[start + t] : make_int2(0, kAlwaysHi);
+                ci.cs = p.scale_log2;
+                if (is_cached(kind)) {
+                    const bool hist = kind == kKindHist;
+                    const int64_t i = (int64_t)h * (hist ? p.hist_stride : p.head_rows) + start + t;
+                    ci.cs *= __ldg((hist ? p.ksl : p.hks) + i);
+                    ci.vs = __ldg((hist ? p.vsl : p.hvs) + i);
                 }
             }
+            return ci;
+        };
+        // Waits are warp-wide for D = 128; at D = 64 the key conversion needs all four warps, so there
+        // every wait ends in a named barrier whose OR-reduced abort flag all four warps agree on.
+        auto conv_wait = [&](uint64_t *bar, uint32_t par, int site) -> bool {
+            if constexpr (D == 64) {
+                mbar_wait(bar, par, wd, site);
+                return !named_bar_or(1, 128, *abort_flag != 0);
+            } else {
+                return __all_sync(0xffffffffu, mbar_wait(bar, par, wd, site));
+            }
+        };
+        ListCursor cursor(list, n_tiles);
+        uint32_t kpar = 0, vpar = 0;        // per slot: parity of the next INT8 landing
+        int u = 0;                          // index among this block's tiles
+        int4 en;
+        bool have = cursor.next(use_bit, en);
+        ColInfo nxt;
+        if (have) nxt = col_info(en);
+        bool ok = true;
+        while (have) {
+            const int4 e = en;
+            const bool cached = is_cached(e.x & 3);
+            const ColInfo cur = nxt;
+            have = cursor.next(use_bit, en);
+            if (have) nxt = col_info(en);
             const int ci = u % kNCI;
-            mbar_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, wd, 1);
-            named_bar_sync(1, 128);
-            if (*abort_flag) break;
-            sCS[ci * 128 + t] = cs;
-            sCW[ci * 128 + t] = w;
-            named_bar_sync(1, 128);
-            if (t == 0) mbar_arrive(&ci_full[ci]);
+            ok = conv_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, 1);
+            if (!ok) break;
+            sCS[ci * 128 + t] = cur.cs;
+            sCV[ci * 128 + t] = cur.vs;
+            sCW[ci * 128 + t] = cur.w;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ci_full[ci]);
             if (cached) {
                 // keys: INT8 codes in the upper half of the slot -> exact fp16 codes over the slot
                 const int sk = u % C::NK;
-                mbar_wait(&k_tma[sk], (kpar >> sk) & 1u, wd, 2);
-                kpar ^= 1u << sk;
-                named_bar_sync(1, 128);
-                if (*abort_flag) break;
                 uint8_t *slot = sK + sk * C::SLOT;
                 uint4 raw[C::CHUNKS];
+                ok = conv_wait(&k_tma[sk], (kpar >> sk) & 1u, 2);
+                if (!ok) break;
+                kpar ^= 1u << sk;
 #pragma unroll
                 for (int i = 0; i < C::CHUNKS; ++i) raw[i] = reinterpret_cast<const uint4 *>(slot + C::HALF)[t + 128 * i];
-                named_bar_sync(1, 128);   // every code is in registers before any fp16 lands on it
+                if constexpr (D == 64) {
+                    named_bar_sync(1, 128);   // every code is in registers before any fp16 lands on it
+                } else {
+                    __syncwarp();             // the row's eight chunks are read before its panel 1 is written
+                }
 #pragma unroll
                 for (int i = 0; i < C::CHUNKS; ++i) {
                     const int idx = t + 128 * i;
@@ -328,36 +365,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     *reinterpret_cast<uint4 *>(base + sw128_offset(row, (c % 4) * 2)) = lo;
                     *reinterpret_cast<uint4 *>(base + sw128_offset(row, (c % 4) * 2 + 1)) = hi;
                 }
-                fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (t == 0) mbar_arrive(&k_full[sk]);
-                // values: V^T INT8 rows (one scale per key) -> fp16(code * scale)
+                // values: V^T INT8 rows -> exact fp16 codes (the softmax multiplies P by the value scale)
                 const int sv = u % C::NV;
-                sVS[t] = vsc;   // readers of the previous tile's scales passed the barrier above
-                mbar_wait(&v_tma[sv], (vpar >> sv) & 1u, wd, 3);
+                ok = conv_wait(&v_tma[sv], (vpar >> sv) & 1u, 3);
+                if (!ok) break;
                 vpar ^= 1u << sv;
-                named_bar_sync(1, 128);
-                if (*abort_flag) break;
                 slot = sV + sv * C::SLOT;
 #pragma unroll
                 for (int i = 0; i < C::CHUNKS; ++i) raw[i] = reinterpret_cast<const uint4 *>(slot + C::HALF)[t + 128 * i];
-                const int kc = t % 8;   // this thread's 16-key chunk of every row (idx % 8 == t % 8)
-                float4 s4[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) s4[i] = reinterpret_cast<const float4 *>(sVS + kc * 16)[i];
-                named_bar_sync(1, 128);
+                __syncwarp();
 #pragma unroll
                 for (int i = 0; i < C::CHUNKS; ++i) {
                     const int d = (t + 128 * i) / 8;
                     uint4 lo, hi;
-                    i8x16_keyscaled_to_f16(raw[i], s4, lo, hi);
+                    i8x16_to_f16(raw[i], lo, hi);
                     uint8_t *base = slot + (kc / 4) * C::VPANEL;
                     *reinterpret_cast<uint4 *>(base + sw128_offset(d, (kc % 4) * 2)) = lo;
                     *reinterpret_cast<uint4 *>(base + sw128_offset(d, (kc % 4) * 2 + 1)) = hi;
                 }
-                fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (t == 0) mbar_arrive(&v_full[sv]);
+                fence_proxy_async_smem();   // one fence publishes both tiles to the tensor core
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&k_full[sk]);
+                    mbar_arrive(&v_full[sv]);
+                }
             }
             ++u;
         }
@@ -388,8 +419,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 return true;
             };
             int u = 0;
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                if (!(list[j].x & use_bit)) continue;
+            ListCursor cursor(list, n_tiles);
+            int4 e;
+            while (ok && cursor.next(use_bit, e)) {
                 const int sk = u % C::NK;
                 ok = mbar_wait(&k_full[sk], (u / C::NK) & 1, wd, 2);
                 if (!ok) break;
@@ -421,9 +453,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t kwait8 = 0, vwait8 = 0;         // per slot: it signals the INT8 barrier
             uint32_t kwpar = 0, vwpar = 0;           // per slot: parity of that signal
             int u = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int4 e = list[j];
-                if (!(e.x & use_bit)) continue;
+            ListCursor cursor(list, n_tiles);
+            int4 e;
+            while (cursor.next(use_bit, e)) {
                 const int kind = e.x & 3;
                 const int start = e.y;
                 const bool cached = is_cached(kind);
@@ -433,6 +465,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 uint8_t *dk = sK + sk * C::SLOT;
                 if (!cached) {
                     mbar_arrive_expect_tx(&k_full[sk], C::SLOT);
+                    mbar_arrive_cnt(&k_full[sk], 3);   // stands in for the converter warps
 #pragma unroll
                     for (int hh = 0; hh < D / 64; ++hh)
                         tma_load_3d(dk + hh * C::KPANEL, kind == kKindCur ? &tm_kc : &tm_kt, &k_full[sk], hh * 64,
@@ -452,6 +485,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 uint8_t *dv = sV + sv * C::SLOT;
                 if (!cached) {
                     mbar_arrive_expect_tx(&v_full[sv], C::SLOT);
+                    mbar_arrive_cnt(&v_full[sv], 3);
 #pragma unroll
                     for (int pp = 0; pp < 2; ++pp)
                         tma_load_3d(dv + pp * C::VPANEL, kind == kKindCur ? &tm_vc : &tm_vt, &v_full[sv],
@@ -517,9 +551,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         float l = 0.0f;
         int u = 0;
         bool ok = true;
-        for (int j = 0; j < n_tiles; ++j) {
-            const int4 e = list[j];
-            if (!(e.x & use_bit)) continue;
+        ListCursor cursor(list, n_tiles);
+        int4 e;
+        while (cursor.next(use_bit, e)) {
             const int ci = u % kNCI;
             const int b = u & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(&ci_full[ci], (u / kNCI) & 1, wd, 1));
@@ -557,8 +591,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     s[2 * i + 1] = (w.z <= frame && frame < w.w) ? s[2 * i + 1] : -INFINITY;
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ci_empty[ci]);
             // row maximum over this half (two independent max3 chains), then swapped with the other half
             float m0 = max3(s[0], s[1], s[2]), m1 = max3(s[32], s[33], s[34]);
 #pragma unroll
@@ -586,19 +618,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float2 cm2 = make_float2(cmul, cmul);
             const float2 no2 = make_float2(-off, -off);
             float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+            const float2 *cv2 = reinterpret_cast<const float2 *>(sCV + ci * 128 + half * 64);
 #pragma unroll
             for (int qt = 0; qt < 2; ++qt) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const float2 a = __ffma2_rn(make_float2(s[qt * 32 + c], s[qt * 32 + c + 1]), cm2, no2);
-                    const float p0 = ex2(a.x);
-                    const float p1 = ex2(a.y);
-                    acc[(c >> 1) & 1] = __fadd2_rn(acc[(c >> 1) & 1], make_float2(p0, p1));
-                    pk[c / 2] = f16x2_of(p0, p1);
+                    float2 pe = make_float2(ex2(a.x), ex2(a.y));
+                    acc[(c >> 1) & 1] = __fadd2_rn(acc[(c >> 1) & 1], pe);
+                    // cached values enter the tensor core as exact codes: P carries their scale
+                    if (cached) pe = __fmul2_rn(pe, cv2[(qt * 32 + c) / 2]);
+                    pk[c / 2] = f16x2_of(pe.x, pe.y);
                 }
                 tmem_st16(tS + qt * 16, pk);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ci_empty[ci]);   // column info no longer needed
             l = l * f + ((acc[0].x + acc[1].x) + (acc[0].y + acc[1].y));
             // rescale this half of O (rare: only when some row's maximum grew past the threshold) once
             // PV of the previous tile is complete; S_u's completion already implies PV_{u-2}'s

@@ -1,0 +1,66 @@
+"""Host side of the multi-GPU bench path on CPU: two gloo ranks with different step times; the job
+time is the slowest rank's and the throughput counts the work of both ranks (weak scaling)."""
+import multiprocessing as mp
+import os
+import socket
+
+import pytest
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+
+    def reduce_max(x):
+        t = torch.tensor([x], dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    local_ms = 10.0 + 5.0 * rank          # rank 1 is slower
+    ms, value = bench.aggregate_ranks(local_ms, 1e12, world, reduce_max)
+    q.put((rank, ms, value))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_max_over_ranks_and_whole_job_work(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    slowest = 10.0 + 5.0 * (world - 1)
+    for _, ms, value in res:
+        assert ms == slowest
+        assert value == pytest.approx(world * 1e12 / (slowest * 1e-3))
+
+
+def test_single_rank_is_local_time():
+    import bench
+    ms, value = bench.aggregate_ranks(4.0, 2e12, 1, reduce_max=lambda x: 1e9)
+    assert ms == 4.0 and value == pytest.approx(2e12 / 4e-3)
+
+
+def test_traffic_is_dropped_when_the_kernel_changed(tmp_path):
+    import json
+    import bench
+    f = tmp_path / "t.json"
+    f.write_text(json.dumps({"attn_source_sha256_16": bench.source_digest(), "bytes_per_launch": 123}))
+    assert bench.measured_traffic(str(f)) == 123
+    f.write_text(json.dumps({"attn_source_sha256_16": "0" * 16, "bytes_per_launch": 123}))
+    assert bench.measured_traffic(str(f)) is None

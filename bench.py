@@ -198,37 +198,32 @@ def run_ours(args, rank, world, local_rank):
         if rc != 0:
             raise N.NomasError(rc, what)
 
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-
-    def step(record=None):
-        if record is not None:
+    def step(ev=None):
+        if ev is not None:
             ev[0].record(st)
         check(N.nomas_kv_append(cache.handle, pk.data_ptr(), pv.data_ptr(), pk.stride(0), pk.stride(1),
                                 n_frames_prev, 0, 0, 0, s), "append")
-        if record is not None:
+        if ev is not None:
             ev[1].record(st)
         check(N.nomas_mask_build(cache.handle, seg, 0, 0.25, 0, 0, ts, hs, mbuf_d.data_ptr(), s), "mask dense")
-        if record is not None:
+        if ev is not None:
             ev[2].record(st)
         check(N.nomas_attn_fwd(cache.handle, seg, 0, 0.25, mbuf_d.data_ptr(), q.data_ptr(), kc.data_ptr(),
                                vc.data_ptr(), kt.data_ptr(), vt.data_ptr(), ts, hs, scale, out_d.data_ptr(), 0,
                                ws.data_ptr(), s),
               "attn dense")
-        if record is not None:
+        if ev is not None:
             ev[3].record(st)
         check(N.nomas_mask_build(cache.handle, seg, 1, 0.25, q.data_ptr(), kc.data_ptr(), ts, hs,
                                  mbuf_s.data_ptr(), s), "mask sparse")
-        if record is not None:
+        if ev is not None:
             ev[4].record(st)
         check(N.nomas_attn_fwd(cache.handle, seg, 1, 0.25, mbuf_s.data_ptr(), q.data_ptr(), kc.data_ptr(),
                                vc.data_ptr(), kt.data_ptr(), vt.data_ptr(), ts, hs, scale, out_s.data_ptr(), 0,
                                ws.data_ptr(), s),
               "attn sparse")
-        if record is not None:
+        if ev is not None:
             ev[5].record(st)
-            torch.cuda.synchronize()
-            for i in range(5):
-                record[i].append(ev[i].elapsed_time(ev[i + 1]))
 
     for _ in range(args.warmup):
         step()
@@ -263,11 +258,14 @@ def run_ours(args, rank, world, local_rank):
     ms, _ = aggregate_ranks(ms, 0.0, world, reduce_max)
     if cache.status() != 0:
         raise RuntimeError("device error in the timed region")
-    # per-phase breakdown (separate pass with events between the phases)
-    rec = [[] for _ in range(5)]
-    for _ in range(max(3, min(args.steps, 10))):
-        step(rec)
-    ph = [statistics.mean(r) for r in rec]
+    # per-phase breakdown: a separate pass of steps issued back to back with events between the
+    # phases (no host synchronisation inside the pass, so no phase includes host launch latency)
+    n_ph = max(3, min(args.steps, 10))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_ph)]
+    for k in range(n_ph):
+        step(evs[k])
+    torch.cuda.synchronize()
+    ph = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(n_ph)) for i in range(5)]
 
     # end to end: pinned host inputs -> device, the same C-ABI calls, device -> host of the outputs
     e2e = None

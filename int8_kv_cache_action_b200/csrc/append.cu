@@ -2,9 +2,9 @@
 // sliding-window ring (fluxbbs.com "单卡 4090 怎么做到的", first and second techniques: INT8
 // storage with float scales; 18 retained history latent frames) and the description-head store.
 //
-// HBM-bound: per (token, head) 2*D bf16 read, 2*D int8 + 2 fp32 written.  One group of D/8 lanes
-// handles one (token, head): each lane holds 8 channels of K and 8 of V in one 16-byte load each,
-// the absmax is reduced with xor-shuffles inside the group, and each lane stores 8 codes (8 bytes).
+// HBM-bound: per (token, head) 2*D bf16 read, 2*D int8 + 2 fp32 written.  One group of D/16 lanes
+// handles one (token, head): each lane holds 16 channels of K and 16 of V (two 16-byte loads each),
+// the absmax is reduced with xor-shuffles inside the group, and each lane stores 16 codes.
 #include "common.cuh"
 
 namespace nomas {
@@ -27,18 +27,6 @@ struct AppendArgs {
     float *vs;
 };
 
-// rint(x / s) in fp32 with IEEE division and round-half-even, clamped to [-127, 127].
-// y = x * RN(1/s) is within 2^-16 + 2^-17 of RN(x/s) for |x/s| <= 127 (two roundings of relative
-// size 2^-24 each, one more for RN(x/s) itself), so when y is farther than 2^-15 from the nearest
-// half-integer both round to the same integer; otherwise (rare) the exact quotient is computed.
-__device__ __forceinline__ float quant_code(float x, float s, float r) {
-    const float y = x * r;
-    const float fl = floorf(y);
-    const float dist = fabsf((y - fl) - 0.5f);
-    float q = (dist > 0x1p-15f) ? rintf(y) : rintf(__fdiv_rn(x, s));
-    return fminf(fmaxf(q, -127.0f), 127.0f);
-}
-
 template <int LPV>
 __device__ __forceinline__ float group_max(float a) {
 #pragma unroll
@@ -46,77 +34,130 @@ __device__ __forceinline__ float group_max(float a) {
     return a;
 }
 
-__device__ __forceinline__ void unpack8(const uint4 &w, float (&x)[8]) {
-    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+__device__ __forceinline__ void unpack16(const uint4 &w0, const uint4 &w1, float (&x)[16]) {
+    const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
         x[2 * i] = __uint_as_float(u[i] << 16);
         x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
     }
 }
 
+// Codes rint(x / s) in fp32 with IEEE division and round-half-even for the 16 channels this lane
+// holds; s = RN(absmax / 127) over the group's D channels, so |x / s| <= 127 (1 + 2^-23) and every
+// code lies in [-127, 127].
+// y = x * RN(1/s) is within 2^-16 + 2^-17 of RN(x/s) for |x/s| <= 127 (two roundings of relative
+// size 2^-24 each, one more for RN(x/s) itself), so when y is farther than 2^-15 from the nearest
+// half-integer both round to the same integer.  Otherwise (rare, and always when 1/s overflows) the
+// exact quotient decides; the warp takes that branch only when one of its lanes needs it.
+// Rounding uses t = y + 1.5 * 2^23: the fp32 add rounds y half-to-even to an integer and leaves it,
+// as a two's-complement byte, in the low byte of t's bit pattern; y - (t - 1.5 * 2^23) is exact.
 template <int LPV>
-__device__ __forceinline__ uint2 quant8(const float (&x)[8], float &s_out) {
+__device__ __forceinline__ uint4 quant16(const float (&x)[16], float &s_out) {
+    constexpr float kMagic = 12582912.0f;                 // 1.5 * 2^23
+    constexpr float kFar = 0.5f - 0x1p-15f;               // |y - rint(y)| below this: not near a tie
     float a = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(x[i]));
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
     a = group_max<LPV>(a);
     const float s = __fdiv_rn(a, 127.0f);
     s_out = s;
-    uint32_t lo = 0, hi = 0;
-    if (s > 0.0f) {
-        const float r = __frcp_rn(s);
+    const bool nz = s > 0.0f;
+    const float r = nz ? __frcp_rn(s) : 0.0f;
+    const float2 r2 = make_float2(r, r), m2 = make_float2(kMagic, kMagic), nm2 = make_float2(-kMagic, -kMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+    uint32_t tb[16];
+    bool slow = false;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t b = (uint32_t)((int)quant_code(x[i], s, r)) & 0xFFu;
-            if (i < 4) lo |= b << (8 * i);
-            else hi |= b << (8 * (i - 4));
+    for (int i = 0; i < 8; ++i) {
+        const float2 y = __fmul2_rn(make_float2(x[2 * i], x[2 * i + 1]), r2);
+        const float2 t = __fadd2_rn(y, m2);
+        const float2 q = __fadd2_rn(t, nm2);
+        const float2 d = __ffma2_rn(q, neg1, y);          // y - rint(y), exact
+        slow |= !(fabsf(d.x) < kFar) || !(fabsf(d.y) < kFar);   // NaN (1/s overflowed) counts as near
+        tb[2 * i] = __float_as_uint(t.x);
+        tb[2 * i + 1] = __float_as_uint(t.y);
+    }
+    if (__any_sync(0xffffffffu, slow && nz)) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float y = x[i] * r;
+            const float d = y - __fsub_rn(__fadd_rn(y, kMagic), kMagic);
+            if (nz && !(fabsf(d) < kFar)) tb[i] = __float_as_uint(__fadd_rn(rintf(__fdiv_rn(x[i], s)), kMagic));
         }
     }
-    return make_uint2(lo, hi);
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)   // low bytes of t[4i .. 4i+3]
+        w[i] = __byte_perm(__byte_perm(tb[4 * i], tb[4 * i + 1], 0x0040), __byte_perm(tb[4 * i + 2], tb[4 * i + 3], 0x0040),
+                           0x5410);
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
+
+// Work unit of a warp: one head of a block of kTokBlock consecutive tokens.  A group of D/16 lanes
+// quantises one (token, head) with 16 channels per lane; the warp's groups split the block's tokens
+// (IPG each), issue all their 16-byte loads before quantising, and write kTokBlock consecutive
+// destination rows and scales of that head.  Index arithmetic is one 32-bit division per unit;
+// destination rows advance incrementally across frame boundaries.
+constexpr int kTokBlock = 8;
 
 template <int D>
 __global__ void __launch_bounds__(256) quant_append_kernel(AppendArgs a) {
-    constexpr int LPV = D / 8;          // lanes per (token, head) vector
-    constexpr int GPW = 32 / LPV;       // groups per warp
+    constexpr int LPV = D / 16;             // lanes per (token, head) vector
+    constexpr int GPW = 32 / LPV;           // groups per warp
+    constexpr int IPG = kTokBlock / GPW;    // tokens per group and unit
+    static_assert(IPG >= 1 && IPG * GPW == kTokBlock, "token block split");
     const int lane = threadIdx.x & 31;
     const int sub = lane % LPV;
     const int grp = lane / LPV;
-    const int64_t n_items = a.n_tok * a.heads;
-    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t wstride = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t base = warp0 * GPW; base < n_items; base += wstride * GPW) {
-        const int64_t it = base + grp;
-        const bool ok = it < n_items;
-        const int64_t itc = ok ? it : base;
-        // item order: head-major, so consecutive groups write consecutive destination rows
-        const int h = (int)(itc / a.n_tok);
-        const int64_t t = itc - (int64_t)h * a.n_tok;
-        const int64_t src = t * a.tok_stride + (int64_t)h * a.head_stride + sub * 8;
-        const uint4 rk = __ldg(reinterpret_cast<const uint4 *>(a.k + src));
-        const uint4 rv = __ldg(reinterpret_cast<const uint4 *>(a.v + src));
-        float xk[8], xv[8];
-        unpack8(rk, xk);
-        unpack8(rv, xv);
-        float sk, sv;
-        const uint2 qk = quant8<LPV>(xk, sk);
-        const uint2 qv = quant8<LPV>(xv, sv);
-        int64_t row;
-        if (a.head_mode) {
-            row = a.dst_row0 + t;
-        } else {
-            const int64_t f = t / a.tokens_per_frame;
-            const int64_t slot = (a.first_slot + f) % a.capacity_frames;
-            row = slot * a.tokens_per_frame + (t - f * a.tokens_per_frame);
+    const int n_tok = (int)a.n_tok;
+    const int T = a.tokens_per_frame, C = a.capacity_frames;
+    const int n_units = (n_tok + kTokBlock - 1) / kTokBlock * a.heads;
+    const int warp0 = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    const int nwarps = (int)(((int64_t)gridDim.x * blockDim.x) >> 5);
+    for (int unit = warp0; unit < n_units; unit += nwarps) {
+        const int tb = unit / a.heads;
+        const int h = unit - tb * a.heads;
+        const int t0 = tb * kTokBlock + grp * IPG;
+        uint4 rk[IPG][2], rv[IPG][2];
+#pragma unroll
+        for (int i = 0; i < IPG; ++i) {
+            const int t = t0 + i < n_tok ? t0 + i : 0;   // rows past the end read token 0, dropped below
+            const int64_t src = (int64_t)t * a.tok_stride + (int64_t)h * a.head_stride + sub * 16;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                rk[i][c] = __ldg(reinterpret_cast<const uint4 *>(a.k + src) + c);
+                rv[i][c] = __ldg(reinterpret_cast<const uint4 *>(a.v + src) + c);
+            }
         }
-        const int64_t di = (int64_t)h * a.rows_per_head + row;
-        if (ok) {
-            *reinterpret_cast<uint2 *>(a.k8 + di * D + sub * 8) = qk;
-            *reinterpret_cast<uint2 *>(a.v8 + di * D + sub * 8) = qv;
-            if (sub == 0) {
-                a.ks[di] = sk;
-                a.vs[di] = sv;
+        // destination row of t0: ring slot of its frame (video) or the head store's next row
+        int r = 0, slot = 0;
+        if (!a.head_mode) {
+            const int f = t0 / T;
+            r = t0 - f * T;
+            slot = (a.first_slot + f) % C;
+        }
+#pragma unroll
+        for (int i = 0; i < IPG; ++i) {
+            float x[16];
+            float sk, sv;
+            unpack16(rk[i][0], rk[i][1], x);
+            const uint4 qk = quant16<LPV>(x, sk);
+            unpack16(rv[i][0], rv[i][1], x);
+            const uint4 qv = quant16<LPV>(x, sv);
+            const int64_t row = a.head_mode ? a.dst_row0 + t0 + i : (int64_t)slot * T + r;
+            const int64_t di = (int64_t)h * a.rows_per_head + row;
+            if (t0 + i < n_tok) {
+                *reinterpret_cast<uint4 *>(a.k8 + di * D + sub * 16) = qk;
+                *reinterpret_cast<uint4 *>(a.v8 + di * D + sub * 16) = qv;
+                if (sub == 0) {
+                    a.ks[di] = sk;
+                    a.vs[di] = sv;
+                }
+            }
+            if (++r == T) {   // next token starts the next frame
+                r = 0;
+                slot = slot + 1 == C ? 0 : slot + 1;
             }
         }
     }
@@ -157,10 +198,11 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
 
 static int launch_append(const AppendArgs &a, int D, cudaStream_t st) {
     if (a.n_tok <= 0) return NOMAS_OK;
-    const int64_t groups = a.n_tok * a.heads;
-    const int64_t threads = groups * (D / 8);
-    int64_t blocks = (threads + 255) / 256;
-    if (blocks > 148 * 32) blocks = 148 * 32;
+    if (a.n_tok >= (int64_t)1 << 30) return NOMAS_EINVAL;   // 32-bit token indices
+    const int64_t units = (a.n_tok + kTokBlock - 1) / kTokBlock * a.heads;   // one warp each
+    if (units >= (int64_t)1 << 31) return NOMAS_EINVAL;
+    int64_t blocks = (units * 32 + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
     if (D == 128) quant_append_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(a);
     else quant_append_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(a);
     return check_launch("quant_append_kernel launch");

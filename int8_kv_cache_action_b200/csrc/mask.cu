@@ -114,23 +114,33 @@ __device__ __forceinline__ int mask_flag(int8_t cls, int32_t count) { return (cl
 
 // Dense lists: one thread per pair of query blocks (one attention CTA); lists are head-independent.
 __global__ void lists_dense_kernel(MaskParams p) {
-    const int pr = blockIdx.x * blockDim.x + threadIdx.x;
-    if (pr >= p.n_lists) return;
+    // one warp per list: lanes test 32 tiles at a time, kept tiles are compacted in index order
+    const int pr = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+    const int lane = threadIdx.x & 31;
+    if (pr >= p.n_lists) return;   // warp-uniform
     const int b0 = 2 * pr, b1 = 2 * pr + 1;
     const int8_t *cls = reinterpret_cast<const int8_t *>(p.buf + p.lay.off_class);
     int4 *out = reinterpret_cast<int4 *>(p.buf + p.lay.off_list) + (int64_t)pr * p.list_cap;
     int n = 0;
-    for (int j = 0; j < p.n_tiles; ++j) {
-        const int8_t c0 = cls[(int64_t)b0 * p.n_tiles + j];
-        const int8_t c1 = b1 < p.n_qb ? cls[(int64_t)b1 * p.n_tiles + j] : 0;
-        if (c0 == 0 && c1 == 0) continue;
-        const TileInfo ti = tile_info(p, j);
-        int f = ti.kind;
-        if (c0) f |= kUse0 | (mask_flag(c0, ti.count) ? kMask0 : 0);
-        if (c1) f |= kUse1 | (mask_flag(c1, ti.count) ? kMask1 : 0);
-        out[n++] = make_int4(f, (int)ti.start, ti.count, j);
+    for (int j0 = 0; j0 < p.n_tiles; j0 += 32) {
+        const int j = j0 + lane;
+        int8_t c0 = 0, c1 = 0;
+        if (j < p.n_tiles) {
+            c0 = cls[(int64_t)b0 * p.n_tiles + j];
+            c1 = b1 < p.n_qb ? cls[(int64_t)b1 * p.n_tiles + j] : 0;
+        }
+        const bool keep = c0 != 0 || c1 != 0;
+        const uint32_t m = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+            const TileInfo ti = tile_info(p, j);
+            int f = ti.kind;
+            if (c0) f |= kUse0 | (mask_flag(c0, ti.count) ? kMask0 : 0);
+            if (c1) f |= kUse1 | (mask_flag(c1, ti.count) ? kMask1 : 0);
+            out[n + __popc(m & ((1u << lane) - 1u))] = make_int4(f, (int)ti.start, ti.count, j);
+        }
+        n += __popc(m);
     }
-    reinterpret_cast<int32_t *>(p.buf + p.lay.off_count)[pr] = n;
+    if (lane == 0) reinterpret_cast<int32_t *>(p.buf + p.lay.off_count)[pr] = n;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -183,23 +193,52 @@ __global__ void kmean_kernel(MaskParams p) {
     reinterpret_cast<float *>(p.buf + p.lay.off_kmean)[idx] = __fdiv_rn(acc, (float)nv);
 }
 
-// score[h][b][cand] = fmaf chain over channels in ascending order from +0.0f.
-__global__ void score_kernel(MaskParams p) {
-    extern __shared__ float qm_s[];
-    const int hb = blockIdx.x;  // h * n_qb + b
-    const int h = hb / p.n_qb;
-    const float *qm = reinterpret_cast<const float *>(p.buf + p.lay.off_qmean) + (int64_t)hb * p.D;
-    for (int c = threadIdx.x; c < p.D; c += blockDim.x) qm_s[c] = qm[c];
-    __syncthreads();
-    const float *km = reinterpret_cast<const float *>(p.buf + p.lay.off_kmean) + (int64_t)h * p.n_cand * p.D;
-    float *sc = reinterpret_cast<float *>(p.buf + p.lay.off_score) + (int64_t)hb * p.n_cand;
-    for (int cand = threadIdx.x; cand < p.n_cand; cand += blockDim.x) {
-        const float *k = km + (int64_t)cand * p.D;
-        float acc = 0.0f;
-        for (int c = 0; c < p.D; ++c) acc = __fmaf_rn(qm_s[c], k[c], acc);
-        sc[cand] = acc;
+// score[h][b][cand] = fmaf chain over channels in ascending order from +0.0f.  One block covers
+// kScoreQB query blocks of one head; candidate means are staged 32 at a time in shared memory (rows
+// padded by one float so the 32 lanes of a warp, one candidate each, hit distinct banks), and each
+// thread runs the chain of one (query block, candidate) pair.
+constexpr int kScoreQB = 8;
+
+__device__ __forceinline__ void score_block(const MaskParams &p, const float *qmean_all, const float *kmean_all) {
+    extern __shared__ float sh[];
+    const int D = p.D;
+    const int qb_chunks = (p.n_qb + kScoreQB - 1) / kScoreQB;
+    const int h = blockIdx.x / qb_chunks;
+    const int b0 = (blockIdx.x % qb_chunks) * kScoreQB;
+    float *qm_s = sh;                     // [kScoreQB][D]
+    float *km_s = sh + kScoreQB * D;      // [32][D + 1]
+    for (int i = threadIdx.x; i < kScoreQB * D; i += blockDim.x) {
+        const int b = b0 + i / D;
+        qm_s[i] = b < p.n_qb ? qmean_all[((int64_t)h * p.n_qb + b) * D + i % D] : 0.0f;
+    }
+    const int bl = threadIdx.x >> 5, cl = threadIdx.x & 31;
+    const int b = b0 + bl;
+    const float *km = kmean_all + (int64_t)h * p.n_cand * D;
+    float *sc = reinterpret_cast<float *>(p.buf + p.lay.off_score);
+    for (int c0 = 0; c0 < p.n_cand; c0 += 32) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < 32 * D; i += blockDim.x) {
+            const int cand = c0 + i / D;
+            km_s[(i / D) * (D + 1) + i % D] = cand < p.n_cand ? km[(int64_t)cand * D + i % D] : 0.0f;
+        }
+        __syncthreads();
+        const int cand = c0 + cl;
+        if (b < p.n_qb && cand < p.n_cand) {
+            const float *q = qm_s + bl * D, *k = km_s + cl * (D + 1);
+            float acc = 0.0f;
+            for (int c = 0; c < D; ++c) acc = __fmaf_rn(q[c], k[c], acc);
+            sc[((int64_t)h * p.n_qb + b) * p.n_cand + cand] = acc;
+        }
     }
 }
+
+__global__ void __launch_bounds__(32 * kScoreQB) score_kernel(MaskParams p) {
+    score_block(p, reinterpret_cast<const float *>(p.buf + p.lay.off_qmean),
+                reinterpret_cast<const float *>(p.buf + p.lay.off_kmean));
+}
+
+static size_t score_smem(int D) { return (size_t)(kScoreQB * D + 32 * (D + 1)) * sizeof(float); }
+static unsigned score_grid(const MaskParams &p) { return (unsigned)(p.H * ((p.n_qb + kScoreQB - 1) / kScoreQB)); }
 
 // Rank every candidate (score descending, index ascending); ranks below keep are written in order.
 __global__ void select_kernel(MaskParams p) {
@@ -341,11 +380,11 @@ extern "C" int nomas_mask_build(const nomas_kv_cache *c, const nomas_segment_tex
     mask_prep_kernel<<<nblk(lay.text_tokens > 0 ? lay.text_tokens : 1, 256), 256, 0, st>>>(p);
     class_map_kernel<<<nblk((int64_t)lay.n_qblocks * lay.n_tiles, 256), 256, 0, st>>>(p);
     if (!sp) {
-        lists_dense_kernel<<<nblk(lay.n_lists, 64), 64, 0, st>>>(p);
+        lists_dense_kernel<<<nblk((int64_t)lay.n_lists * 32, 128), 128, 0, st>>>(p);
     } else {
         qmean_kernel<<<nblk((int64_t)p.H * p.n_qb * p.D, 256), 256, 0, st>>>(p);
         kmean_kernel<<<nblk((int64_t)p.H * p.n_cand * p.D, 256), 256, 0, st>>>(p);
-        score_kernel<<<p.H * p.n_qb, 256, p.D * sizeof(float), st>>>(p);
+        score_kernel<<<score_grid(p), 32 * kScoreQB, score_smem(p.D), st>>>(p);
         select_kernel<<<p.H * p.n_qb, 256, p.n_cand * sizeof(float), st>>>(p);
         lists_sparse_kernel<<<p.H * ((p.n_qb + 1) / 2), 128, 2 * ((p.n_cand + 31) / 32) * sizeof(uint32_t), st>>>(p);
     }
@@ -406,21 +445,9 @@ __global__ void kmean_to_kernel(MaskParams p, float *kmean) {
     kmean[idx] = __fdiv_rn(acc, (float)nv);
 }
 
-__global__ void score_from_kernel(MaskParams p, const float *qmean_all, const float *kmean_all) {
-    extern __shared__ float qm_s[];
-    const int hb = blockIdx.x;
-    const int h = hb / p.n_qb;
-    const float *qm = qmean_all + (int64_t)hb * p.D;
-    for (int c = threadIdx.x; c < p.D; c += blockDim.x) qm_s[c] = qm[c];
-    __syncthreads();
-    const float *km = kmean_all + (int64_t)h * p.n_cand * p.D;
-    float *sc = reinterpret_cast<float *>(p.buf + p.lay.off_score) + (int64_t)hb * p.n_cand;
-    for (int cand = threadIdx.x; cand < p.n_cand; cand += blockDim.x) {
-        const float *k = km + (int64_t)cand * p.D;
-        float acc = 0.0f;
-        for (int c = 0; c < p.D; ++c) acc = __fmaf_rn(qm_s[c], k[c], acc);
-        sc[cand] = acc;
-    }
+__global__ void __launch_bounds__(32 * kScoreQB) score_from_kernel(MaskParams p, const float *qmean_all,
+                                                                      const float *kmean_all) {
+    score_block(p, qmean_all, kmean_all);
 }
 
 // Device address of this file's scratch array on the current device, looked up once per device.
@@ -513,7 +540,7 @@ extern "C" int nomas_mask_build_static(const nomas_kv_cache *c, const nomas_segm
     class_map_kernel<<<nblk((int64_t)lay.n_qblocks * lay.n_tiles, 256), 256, 0, st>>>(p);
     qmean_to_kernel<<<nblk((int64_t)nq_floats, 256), 256, 0, st>>>(p, qmean);
     kmean_to_kernel<<<nblk((int64_t)nk_floats, 256), 256, 0, st>>>(p, kmean);
-    score_from_kernel<<<p.H * p.n_qb, 256, p.D * sizeof(float), st>>>(p, qmean, kmean);
+    score_from_kernel<<<score_grid(p), 32 * kScoreQB, score_smem(p.D), st>>>(p, qmean, kmean);
     select_kernel<<<p.H * p.n_qb, 256, p.n_cand * sizeof(float), st>>>(p);
     lists_sparse_kernel<<<p.H * ((p.n_qb + 1) / 2), 128, 2 * ((p.n_cand + 31) / 32) * sizeof(uint32_t), st>>>(p);
     return check_launch("mask_build_static kernels launch");

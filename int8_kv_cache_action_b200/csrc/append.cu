@@ -94,31 +94,32 @@ __device__ __forceinline__ uint4 quant16(const float (&x)[16], float &s_out) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Work unit of a warp: one head of a block of kTokBlock consecutive tokens.  A group of D/16 lanes
-// quantises one (token, head) with 16 channels per lane; the warp's groups split the block's tokens
-// (IPG each), issue all their 16-byte loads before quantising, and write kTokBlock consecutive
-// destination rows and scales of that head.  Index arithmetic is one 32-bit division per unit;
-// destination rows advance incrementally across frame boundaries.
-constexpr int kTokBlock = 8;
+// Work unit of a warp: one head of a block of kTokBlock consecutive tokens, one token per group of
+// D/16 lanes (16 channels per lane).  The warp issues all its 16-byte loads before quantising and
+// writes kTokBlock consecutive destination rows and scales of that head.  Index arithmetic is one
+// 32-bit division per unit; destination rows advance incrementally across frame boundaries.  At most
+// 64 registers, so four 256-thread blocks share an SM.
+template <int D>
+constexpr int kTokBlock = 32 / (D / 16);    // one token per group of D/16 lanes
 
 template <int D>
-__global__ void __launch_bounds__(256) quant_append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(256, 4) quant_append_kernel(AppendArgs a) {
     constexpr int LPV = D / 16;             // lanes per (token, head) vector
     constexpr int GPW = 32 / LPV;           // groups per warp
-    constexpr int IPG = kTokBlock / GPW;    // tokens per group and unit
-    static_assert(IPG >= 1 && IPG * GPW == kTokBlock, "token block split");
+    constexpr int IPG = kTokBlock<D> / GPW; // tokens per group and unit
+    static_assert(IPG >= 1 && IPG * GPW == kTokBlock<D>, "token block split");
     const int lane = threadIdx.x & 31;
     const int sub = lane % LPV;
     const int grp = lane / LPV;
     const int n_tok = (int)a.n_tok;
     const int T = a.tokens_per_frame, C = a.capacity_frames;
-    const int n_units = (n_tok + kTokBlock - 1) / kTokBlock * a.heads;
+    const int n_units = (n_tok + kTokBlock<D> - 1) / kTokBlock<D> * a.heads;
     const int warp0 = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
     const int nwarps = (int)(((int64_t)gridDim.x * blockDim.x) >> 5);
     for (int unit = warp0; unit < n_units; unit += nwarps) {
         const int tb = unit / a.heads;
         const int h = unit - tb * a.heads;
-        const int t0 = tb * kTokBlock + grp * IPG;
+        const int t0 = tb * kTokBlock<D> + grp * IPG;
         uint4 rk[IPG][2], rv[IPG][2];
 #pragma unroll
         for (int i = 0; i < IPG; ++i) {
@@ -199,10 +200,11 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
 static int launch_append(const AppendArgs &a, int D, cudaStream_t st) {
     if (a.n_tok <= 0) return NOMAS_OK;
     if (a.n_tok >= (int64_t)1 << 30) return NOMAS_EINVAL;   // 32-bit token indices
-    const int64_t units = (a.n_tok + kTokBlock - 1) / kTokBlock * a.heads;   // one warp each
+    const int64_t tbk = D == 128 ? kTokBlock<128> : kTokBlock<64>;
+    const int64_t units = (a.n_tok + tbk - 1) / tbk * a.heads;   // one warp each
     if (units >= (int64_t)1 << 31) return NOMAS_EINVAL;
     int64_t blocks = (units * 32 + 255) / 256;
-    if (blocks > 148 * 16) blocks = 148 * 16;
+    if (blocks > 148 * 32) blocks = 148 * 32;
     if (D == 128) quant_append_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(a);
     else quant_append_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(a);
     return check_launch("quant_append_kernel launch");

@@ -297,6 +297,76 @@ def run_ours(args, rank, world, local_rank):
                 clocks=clk.summary(), e2e=e2e, cfg=cfg)
 
 
+def per_config(args):
+    """One JSON line per config: the attention call (its mode: dense, or sparse for C3) timed with CUDA
+    events over back-to-back calls after 3 warm-ups, and the quantise-append of one 30-frame (C0: 2)
+    segment into a fresh cache of the config's dimensions."""
+    import torch
+    from int8_kv_cache_action_b200 import _nomas as N
+    from int8_kv_cache_action_b200.runtime import KVCache, mask_views, segment_text_of
+    from int8_kv_cache_action_b200.workloads import CONFIGS, make_inputs, APPEND_BYTES_PER_TOKEN_HEAD
+    dev = torch.device("cuda", 0)
+    for name in ("C0", "C1", "C2", "C3", "C4"):
+        cfg = CONFIGS[name]
+        inp = make_inputs(cfg)
+        cache = KVCache.for_config(cfg, dev)
+        for seg, kv in zip(cfg.prior, inp.prior):
+            cache.append(kv.k.to(dev), kv.v.to(dev), seg.n_frames,
+                         None if kv.head_k is None else kv.head_k.to(dev),
+                         None if kv.head_v is None else kv.head_v.to(dev))
+        seg = segment_text_of(cfg.current)
+        q, kc, vc, kt, vt = (getattr(inp, n).to(dev) for n in ("q", "k_cur", "v_cur", "k_txt", "v_txt"))
+        buf, lay = cache.build_mask(seg, cfg.mode, cfg.keep_frac, q, kc)
+        ws = cache.workspace(seg)
+        out = torch.empty((cfg.n_query, cfg.heads, cfg.head_dim), dtype=torch.float32, device=dev)
+        st = cache.state()
+        if cfg.mode:
+            flops = 4.0 * cfg.head_dim * sparse_key_sum(mask_views(buf, lay)["sel"], cfg, st["history_tokens"],
+                                                        st["head_tokens"])
+        else:
+            flops = 4.0 * cfg.head_dim * cfg.heads * visible_key_sum(cfg, st["history_tokens"], st["head_tokens"])
+
+        def attn():
+            cache.attention(seg, buf, q, kc, vc, kt, vt, mode=cfg.mode, keep_frac=cfg.keep_frac, workspace=ws,
+                            out=out)
+
+        reps = 10 if cfg.n_query > 1000 else 50
+        for _ in range(3):
+            attn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            attn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        status = cache.status()
+        # append: the config's last prior segment (or the current segment's K/V) into a fresh cache
+        src = inp.prior[-1] if cfg.prior else None
+        k_app = (src.k if src is not None else inp.k_cur).to(dev)
+        v_app = (src.v if src is not None else inp.v_cur).to(dev)
+        nf = k_app.shape[0] // cfg.tokens_per_frame
+        kept = min(nf, cfg.window_frames) if cfg.window_frames > 0 else nf
+        fresh = [KVCache.for_config(cfg, dev) for _ in range(reps + 3)]
+        for c in fresh[:3]:
+            c.append(k_app, v_app, nf)
+        torch.cuda.synchronize()
+        e0.record()
+        for c in fresh[3:]:
+            c.append(k_app, v_app, nf)
+        e1.record()
+        torch.cuda.synchronize()
+        app_ms = e0.elapsed_time(e1) / reps
+        app_bytes = kept * cfg.tokens_per_frame * cfg.heads * APPEND_BYTES_PER_TOKEN_HEAD(cfg.head_dim)
+        print(json.dumps({"config": name, "workload": cfg.name, "mode": "sparse" if cfg.mode else "dense",
+                          "attn_ms": ms, "attn_tflops": flops / (ms * 1e-3) / 1e12, "attn_flops": flops,
+                          "append_ms": app_ms, "append_gbs": app_bytes / (app_ms * 1e-3) / 1e9,
+                          "append_kv_tokens_per_s": kept * cfg.tokens_per_frame * cfg.heads / (app_ms * 1e-3),
+                          "status": status}), flush=True)
+        del cache, fresh
+
+
 def cpu_oracle_sample(seconds_budget=15.0, rows_per_head_start=16):
     """Time the CPU oracle (as it stands) on a bounded sample of the same workload's dense attention."""
     import numpy as np
@@ -343,6 +413,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--per-config", action="store_true",
+                    help="print one line per config (attention call and append) instead of the step line")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -366,6 +438,10 @@ def main():
                                  "sample": vals[0]["sample"]},
                 "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
+        return
+
+    if args.per_config:
+        per_config(args)
         return
 
     import torch

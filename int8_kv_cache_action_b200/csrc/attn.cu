@@ -287,23 +287,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int t = threadIdx.x - 256;   // 0..127
         const int kc = t % 8;               // V^T: this thread's 16-key chunk in every row it converts
         struct ColInfo {
-            float cs, vs;
+            float ks, vs;   // raw key / value scale (cached tiles), 1 / 0 otherwise
             int2 w;
         };
-        // Column info of a tile (key scale x log2 e, value scale, frame window), loaded one tile
-        // ahead of its use.
+        // Column info of a tile (key scale, value scale, frame window), loaded one tile ahead of its
+        // use: only loads happen here, so nothing waits for them until the next tile consumes them.
         auto col_info = [&](const int4 &e) -> ColInfo {
             ColInfo ci{0.0f, 0.0f, make_int2(kAlwaysHi, 0)};
             const int kind = e.x & 3;
             const int64_t start = e.y;
             if (t < e.z) {
-                ci.w = kind == kKindText ? p.txtwin[start + t] : make_int2(0, kAlwaysHi);
-                ci.cs = p.scale_log2;
+                if (kind == kKindText) {
+                    ci.w = p.txtwin[start + t];
+                } else {
+                    ci.w = make_int2(0, kAlwaysHi);
+                }
                 if (is_cached(kind)) {
                     const bool hist = kind == kKindHist;
                     const int64_t i = (int64_t)h * (hist ? p.hist_stride : p.head_rows) + start + t;
-                    ci.cs *= __ldg((hist ? p.ksl : p.hks) + i);
+                    ci.ks = __ldg((hist ? p.ksl : p.hks) + i);
                     ci.vs = __ldg((hist ? p.vsl : p.hvs) + i);
+                } else {
+                    ci.ks = 1.0f;
                 }
             }
             return ci;
@@ -335,7 +340,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int ci = u % kNCI;
             ok = conv_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, 1);
             if (!ok) break;
-            sCS[ci * 128 + t] = cur.cs;
+            sCS[ci * 128 + t] = p.scale_log2 * cur.ks;
             sCV[ci * 128 + t] = cur.vs;
             sCW[ci * 128 + t] = cur.w;
             __syncwarp();

@@ -225,10 +225,11 @@ size_t nomas_attn_workspace_bytes(const nomas_kv_cache *cache, const nomas_segme
  * visibility of nomas_mask_build (fluxbbs.com 架构; sparse mode: same page, 单卡 4090 怎么做到的).
  * Per head h and query row i:
  *     O[i,h] = sum_j softmax_j(softmax_scale * q_i . k^_j) v^_j   over visible j
- * with k^ = code * scale for cached keys (the key scale is applied to the fp32 score, the codes
- * enter the tensor core exactly) and v^ = fp16(code * scale) for cached values.  The QK^T and PV
- * products run on the tensor cores with fp16 operands and fp32 accumulation; bf16 inputs convert
- * to fp16 exactly for magnitudes in [2^-14, 65504] (the supported input range).
+ * with k^ = code * scale and v^ = code * scale for cached keys and values.  The codes enter the
+ * tensor core exactly: the key scale multiplies the fp32 score and the value scale the fp32
+ * probability, which is then rounded once to fp16 (so each term p * v^ is fp16(p * scale) * code).
+ * The QK^T and PV products run on the tensor cores with fp16 operands and fp32 accumulation; bf16
+ * inputs convert to fp16 exactly for magnitudes in [2^-14, 65504] (the supported input range).
  *   q, kcur, vcur  bf16 [n_frames*T][H][D];  ktxt, vtxt bf16 [text_tokens][H][D]
  *                  (NULL allowed when the segment has no text); all share tok_stride / head_stride
  *   out            fp32 [n_frames*T][H][D], contiguous

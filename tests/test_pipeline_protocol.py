@@ -1,18 +1,24 @@
-"""CPU model of the attention kernel's per-CTA barrier protocol (loader, MMA issuer, two softmax
-warpgroups) run over dense and sparse tile-use patterns.  It checks that the protocol cannot deadlock
-and that every MMA reads the tile the loader last put in its slot, under random orders of
-asynchronous completion.  The model mirrors the kernel's waits one for one (slot/ring indices, use
-counts and parities); it exercises no GPU.
+"""CPU model of the attention kernel's per-CTA barrier protocol: TMA producer, four converter warps,
+the in-order tcgen05 MMA issuer and eight softmax warps (two column halves x four TMEM lane
+groups).  Random tile-kind sequences (TMA-filled fp16 tiles and INT8 tiles converted in place),
+random delays of every asynchronous completion (TMA landings, MMA completions in issue order) and
+random rescale decisions are run against invariants:
 
-Barrier semantics modelled: a phase completes when its arrival count is reached; a parity test is
-true iff the barrier's current phase parity differs from the tested parity (so a barrier that ran two
-phases ahead is indistinguishable from one that did not -- the reason the MMA issuer guards each slot
-test with its own count of released uses)."""
+- no deadlock;
+- the K / V^T slot an MMA reads holds the tile the protocol says (converted, for INT8 tiles) from
+  the MMA's issue to its completion;
+- the softmax reads S_u from its buffer and the column info of tile u, and reads its partner half's
+  maximum of tile u;
+- PV_u reads P_u complete in both halves and before S_{u+2} overwrites the buffer;
+- an O rescale runs only after PV_{u-1} has completed and before PV_u is issued;
+- the epilogue sees every PV applied.
+
+The model mirrors the kernel's waits one for one (slot and ring indices, per-slot INT8 parity bits,
+phase parities); it exercises no GPU.  Barrier semantics: a phase completes when its arrival count is
+reached; a parity test is true iff the barrier's current phase parity differs from the tested one."""
 import random
 
 import pytest
-
-USE0, USE1 = 4, 8
 
 
 class Bar:
@@ -21,7 +27,7 @@ class Bar:
 
     def arrive(self, n=1):
         self.pending -= n
-        assert self.pending >= 0
+        assert self.pending >= 0, "more arrivals than the phase expects"
         if self.pending == 0:
             self.phase += 1
             self.pending = self.count
@@ -30,131 +36,246 @@ class Bar:
         return (self.phase & 1) != parity
 
 
-def run(flags, ns=4, nci=4, seed=0, guard=True):
-    """Returns (finished, stale_reads)."""
-    n = len(flags)
-    uses = lambda j, q: bool(flags[j] & (USE1 if q else USE0))
-    kv_full = [Bar(1) for _ in range(ns)]
-    kv_empty = [Bar(1) for _ in range(ns)]
-    ci_full = [Bar(1) for _ in range(nci)]
-    ci_empty = [Bar(8) for _ in range(nci)]
-    s_full, p_full = [Bar(1), Bar(1)], [Bar(4), Bar(4)]
-    commits, slot, stale = [], [None] * ns, []
+class Violation(AssertionError):
+    pass
+
+
+def check(cond, what):
+    if not cond:
+        raise Violation(what)
+
+
+def run(kinds, nk=3, nv=3, nci=4, seed=0, rescale_p=0.2, swap_order=False, rescale_parity_shift=0,
+        producer_skips_empty_wait=False):
+    """kinds[u] is True for an INT8 (cached) tile.  Returns True when every role finished."""
+    n = len(kinds)
     rng = random.Random(seed)
+    k_full, k_empty, k_tma = [Bar(4) for _ in range(nk)], [Bar(1) for _ in range(nk)], [Bar(1) for _ in range(nk)]
+    v_full, v_empty, v_tma = [Bar(4) for _ in range(nv)], [Bar(1) for _ in range(nv)], [Bar(1) for _ in range(nv)]
+    ci_full, ci_empty = [Bar(4) for _ in range(nci)], [Bar(8) for _ in range(nci)]
+    s_full, p_full, xm_bar = [Bar(1), Bar(1)], [Bar(8), Bar(8)], [Bar(8), Bar(8)]
+    pv_done, o_final = Bar(1), Bar(1)
+    kslot, vslot = [None] * nk, [None] * nv          # (tile, state); INT8 state counts converted warps
+    sbuf = [None, None]                               # ("S", u) or ("P", u, set of (half, group))
+    cinfo = [None] * nci
+    xm = [[None, None], [None, None]]
+    o_applied = [0]                                   # PVs applied to O
+    rescale = [rng.random() < rescale_p for _ in range(n)]
+    tma_events, mma_fifo = [], []                     # pending asynchronous completions
 
-    def loader():
-        for j in range(n):
-            ci, sk, sv = j % nci, (2 * j) % ns, (2 * j + 1) % ns
-            while not ci_empty[ci].done(((j // nci) & 1) ^ 1):
+    # ---- producer (one thread) -------------------------------------------------------------
+    def producer():
+        kpar = vpar = 0
+        for u in range(n):
+            sk, sv = u % nk, u % nv
+            while not producer_skips_empty_wait and not k_empty[sk].done(((u // nk) & 1) ^ 1):
                 yield False
-            while not kv_empty[sk].done((((2 * j) // ns) & 1) ^ 1):
+            if kinds[u]:
+                tma_events.append(("k8", sk, u))
+            else:
+                tma_events.append(("k16", sk, u))
+            while not v_empty[sv].done(((u // nv) & 1) ^ 1):
                 yield False
-            slot[sk] = ("K", j)
+            tma_events.append(("v8" if kinds[u] else "v16", sv, u))
+            yield True
+
+    def land(ev):
+        kind, s, u = ev
+        if kind == "k16":
+            kslot[s] = (u, "fp16")
+            k_full[s].arrive(4)           # expect_tx arrival + the three stand-in arrivals
+        elif kind == "k8":
+            kslot[s] = (u, 0)
+            k_tma[s].arrive()
+        elif kind == "v16":
+            vslot[s] = (u, "fp16")
+            v_full[s].arrive(4)
+        else:
+            vslot[s] = (u, 0)
+            v_tma[s].arrive()
+
+    # ---- converter warps -------------------------------------------------------------------
+    def converter(w):
+        kpar = vpar = 0
+        for u in range(n):
+            ci = u % nci
+            while not ci_empty[ci].done(((u // nci) & 1) ^ 1):
+                yield False
+            cinfo[ci] = u
             ci_full[ci].arrive()
-            kv_full[sk].arrive()
             yield True
-            while not kv_empty[sv].done((((2 * j + 1) // ns) & 1) ^ 1):
-                yield False
-            slot[sv] = ("V", j)
-            kv_full[sv].arrive()
-            yield True
-
-    def adv(j, q):
-        while j < n and not uses(j, q):
-            j += 1
-        return j
-
-    def mma():
-        nxt, pend, last_s, last_pv, pc, rel = [adv(0, 0), adv(0, 1)], [-1, -1], [-1, -1], [-1, -1], [0, 0], [0] * ns
-        while nxt[0] < n or nxt[1] < n or pend[0] >= 0 or pend[1] >= 0:
-            prog = False
-            for q in (0, 1):
-                o = 1 - q
-                if pend[q] >= 0:
-                    j = pend[q]
-                    sv, u = (2 * j + 1) % ns, (2 * j + 1) // ns
-                    if (not guard or rel[sv] == u) and p_full[q].done(pc[q] & 1) and kv_full[sv].done(u & 1):
-                        if slot[sv] != ("V", j):
-                            stale.append(("V", j))
-                        pc[q] += 1
-                        last_pv[q] = j
-                        if not uses(j, o) or last_pv[o] >= j:
-                            commits.append(kv_empty[sv])
-                            rel[sv] = u + 1
-                        pend[q] = -1
-                        prog = True
-                if pend[q] < 0 and nxt[q] < n:
-                    j = nxt[q]
-                    sk, u = (2 * j) % ns, (2 * j) // ns
-                    if (not guard or rel[sk] == u) and kv_full[sk].done(u & 1):
-                        if slot[sk] != ("K", j):
-                            stale.append(("K", j))
-                        commits.append(s_full[q])
-                        last_s[q] = j
-                        if not uses(j, o) or last_s[o] >= j:
-                            commits.append(kv_empty[sk])
-                            rel[sk] = u + 1
-                        pend[q] = j
-                        nxt[q] = adv(j + 1, q)
-                        prog = True
-            yield prog
-
-    def softmax(q):
-        k = 0
-        for j in range(n):
-            ci = j % nci
-            while not ci_full[ci].done((j // nci) & 1):
-                yield False
-            if uses(j, q):
-                while not s_full[q].done(k & 1):
+            if kinds[u]:
+                sk, sv = u % nk, u % nv
+                while not k_tma[sk].done((kpar >> sk) & 1):
                     yield False
-                p_full[q].arrive(4)
-                k += 1
-            ci_empty[ci].arrive(4)
+                kpar ^= 1 << sk
+                check(kslot[sk] is not None and kslot[sk][0] == u and kslot[sk][1] != "fp16", f"K8 slot {sk} for {u}")
+                kslot[sk] = (u, kslot[sk][1] + 1)
+                while not v_tma[sv].done((vpar >> sv) & 1):
+                    yield False
+                vpar ^= 1 << sv
+                check(vslot[sv] is not None and vslot[sv][0] == u and vslot[sv][1] != "fp16", f"V8 slot {sv} for {u}")
+                vslot[sv] = (u, vslot[sv][1] + 1)
+                k_full[sk].arrive()
+                v_full[sv].arrive()
+                yield True
+
+    def ready(slot, u):
+        return slot is not None and slot[0] == u and (slot[1] == "fp16" or slot[1] == 4)
+
+    # ---- MMA issuer (one thread; operations complete in issue order) --------------------------
+    def mma():
+        def issue_s(u):
+            sk = u % nk
+            while not k_full[sk].done((u // nk) & 1):
+                yield False
+            check(ready(kslot[sk], u), f"S{u} issued on K slot {kslot[sk]}")
+            mma_fifo.append(("S", u))
             yield True
 
-    roles = [loader(), mma(), softmax(0), softmax(1)]
+        def issue_pv(v):
+            sv = v % nv
+            while not p_full[v & 1].done((v >> 1) & 1):
+                yield False
+            while not v_full[sv].done((v // nv) & 1):
+                yield False
+            check(ready(vslot[sv], v), f"PV{v} issued on V slot {vslot[sv]}")
+            b = sbuf[v & 1]
+            check(b is not None and b[0] == "P" and b[1] == v and len(b[2]) == 8, f"PV{v} issued on {b}")
+            mma_fifo.append(("PV", v))
+            yield True
+
+        for u in range(n):
+            if swap_order and u >= 1:
+                yield from issue_pv(u - 1)
+                yield from issue_s(u)
+            else:
+                yield from issue_s(u)
+                if u >= 1:
+                    yield from issue_pv(u - 1)
+        if n:
+            yield from issue_pv(n - 1)
+        mma_fifo.append(("END", n))
+        yield True
+
+    def complete(op):
+        kind, u = op
+        if kind == "S":
+            sk = u % nk
+            check(ready(kslot[sk], u), f"S{u} completed on K slot {kslot[sk]}")
+            b = sbuf[u & 1]
+            check(b is None or (b[0] == "P" and o_applied[0] > b[1]), f"S{u} overwrote unread {b}")
+            sbuf[u & 1] = ("S", u)
+            s_full[u & 1].arrive()
+            k_empty[sk].arrive()
+        elif kind == "PV":
+            sv = u % nv
+            check(ready(vslot[sv], u), f"PV{u} completed on V slot {vslot[sv]}")
+            b = sbuf[u & 1]
+            check(b is not None and b[0] == "P" and b[1] == u and len(b[2]) == 8, f"PV{u} read {b}")
+            check(o_applied[0] == u, f"PV{u} applied out of order")
+            o_applied[0] = u + 1
+            v_empty[sv].arrive()
+            pv_done.arrive()
+        else:
+            o_final.arrive()
+
+    # ---- softmax warps ----------------------------------------------------------------------
+    def softmax(half, g):
+        for u in range(n):
+            ci, b = u % nci, u & 1
+            while not ci_full[ci].done((u // nci) & 1):
+                yield False
+            while not s_full[b].done((u >> 1) & 1):
+                yield False
+            check(sbuf[b] == ("S", u) or (sbuf[b] and sbuf[b][0] == "P" and sbuf[b][1] == u), f"softmax {u} read {sbuf[b]}")
+            check(cinfo[ci] == u, f"softmax {u} read column info of {cinfo[ci]}")
+            if g == 0:
+                xm[b][half] = u
+            xm_bar[b].arrive()
+            while not xm_bar[b].done((u >> 1) & 1):
+                yield False
+            check(xm[b][half ^ 1] == u, f"softmax {u} half {half} read partner max of {xm[b][half ^ 1]}")
+            if sbuf[b][0] == "S":
+                sbuf[b] = ("P", u, set())
+            sbuf[b][2].add((half, g))
+            if rescale[u] and u >= 1:
+                par = ((u - 1) & 1) ^ rescale_parity_shift
+                while not pv_done.done(par):
+                    yield False
+                check(o_applied[0] == u, f"rescale at {u} with {o_applied[0]} PVs applied")
+            ci_empty[ci].arrive()
+            p_full[b].arrive()
+            yield True
+        while not o_final.done(0):
+            yield False
+        check(o_applied[0] == n, "epilogue before every PV")
+
+    roles = [producer(), mma()] + [converter(w) for w in range(4)] + [softmax(h, g) for h in (0, 1) for g in range(4)]
     idle = 0
     while roles:
-        while commits and rng.random() < 0.6:
-            commits.pop(0).arrive()
+        # fire some asynchronous completions: TMA landings in any order, MMAs in issue order
+        while tma_events and rng.random() < 0.5:
+            land(tma_events.pop(rng.randrange(len(tma_events))))
+        while mma_fifo and rng.random() < 0.5:
+            complete(mma_fifo.pop(0))
         prog = False
-        for r in list(roles):
+        for r in rng.sample(roles, len(roles)):
             try:
                 prog |= next(r)
             except StopIteration:
                 roles.remove(r)
                 prog = True
-        idle = 0 if (prog or commits) else idle + 1
-        if idle > 20 or stale:
-            return False, stale
-    return True, stale
+        idle = 0 if (prog or tma_events or mma_fifo) else idle + 1
+        if idle > 50:
+            return False
+    while mma_fifo:
+        complete(mma_fifo.pop(0))
+    return True
 
 
 def _patterns():
     rng = random.Random(11)
-    pats = [[USE0 | USE1] * 40, [USE0] * 30, [USE0, USE1] * 20]
-    for _ in range(60):
-        n = rng.randint(1, 80)
-        p0 = rng.random()
-        pats.append([rng.choice([USE0, USE1, USE0 | USE1]) if rng.random() < p0 else USE0 | USE1 for _ in range(n)])
-    # long one-sided runs: query tile 0 jumps far ahead of query tile 1
-    pats.append([USE0 | USE1] + [USE1] * 50 + [USE0] + [USE1] * 7 + [USE0 | USE1])
-    pats.append([USE0] * 3 + [USE1] * 40 + [USE0] * 3)
+    pats = [[False] * 40, [True] * 40, [True, False] * 20, [True] * 3 + [False] * 30 + [True] * 2, [True], [False]]
+    for _ in range(40):
+        k = rng.randint(1, 60)
+        p = rng.random()
+        pats.append([rng.random() < p for _ in range(k)])
     return pats
 
 
-@pytest.mark.parametrize("ns", [4, 8])
-def test_protocol_never_deadlocks_or_reads_stale_slots(ns):
+@pytest.mark.parametrize("nk", [3, 6])
+def test_protocol_finishes_and_keeps_every_invariant(nk):
     for i, pat in enumerate(_patterns()):
         for seed in range(3):
-            ok, stale = run(pat, ns=ns, seed=seed)
-            assert ok and not stale, (i, pat, stale)
+            assert run(pat, nk=nk, nv=nk, seed=seed), (i, pat, seed)
 
 
-def test_unguarded_slot_test_reads_stale_data():
-    # Without the per-slot release count, a query tile that looks several tiles ahead tests a slot
-    # barrier two phases early and issues an MMA on the previous occupant of the slot.
-    pat = [USE0 | USE1] + [USE1] * 50 + [USE0] + [USE1] * 7 + [USE0 | USE1]
-    results = [run(pat, seed=s, guard=False) for s in range(5)]
-    assert any(stale for _, stale in results)
+def test_issuing_pv_before_the_next_s_still_holds():
+    # the issue order S_u, PV_{u-1} is the kernel's; PV_{u-1}, S_u is also safe (only slower)
+    for seed in range(5):
+        assert run([True, False] * 12, seed=seed, swap_order=True)
+
+
+def test_wrong_rescale_parity_is_caught():
+    # waiting for the PV completion of the wrong phase either deadlocks or rescales too early
+    bad = 0
+    for seed in range(20):
+        try:
+            ok = run([False] * 30, seed=seed, rescale_p=0.5, rescale_parity_shift=1)
+        except Violation:
+            ok = False
+        bad += not ok
+    assert bad > 0
+
+
+def test_model_detects_a_slot_reused_too_early():
+    # a producer that skips the empty-slot wait overwrites a K tile before its MMA has consumed it
+    caught = 0
+    for seed in range(10):
+        try:
+            ok = run([False] * 20, nk=2, nv=2, seed=seed, producer_skips_empty_wait=True)
+        except AssertionError:
+            ok = False
+        caught += not ok
+    assert caught > 0

@@ -165,11 +165,10 @@ __global__ void qmean_kernel(MaskParams p) {
     reinterpret_cast<float *>(p.buf + p.lay.off_qmean)[idx] = __fdiv_rn(acc, (float)nv);
 }
 
-// kmean[h][cand][c]: history candidates dequantise with one fp32 multiply (code * scale).
-__global__ void kmean_kernel(MaskParams p) {
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t n = (int64_t)p.H * p.n_cand * p.D;
-    if (idx >= n) return;
+// kmean[h][cand][c]: history candidates dequantise with one fp32 multiply (code * scale); sums in
+// ascending token order from +0, one division.  The ring row advances incrementally (no modulo per
+// token).
+__device__ __forceinline__ float kmean_value(const MaskParams &p, int64_t idx) {
     const int c = (int)(idx % p.D);
     const int64_t hc = idx / p.D;
     const int cand = (int)(hc % p.n_cand);
@@ -179,10 +178,12 @@ __global__ void kmean_kernel(MaskParams p) {
     if (cand < p.n_hist_tiles) {
         const int64_t a0 = (int64_t)cand * kTile;
         nv = (int)((a0 + kTile < p.Lh) ? kTile : p.Lh - a0);
+        int64_t phys = (p.first_tok + a0) % p.ring_tokens;
+        const int64_t base = (int64_t)h * p.ring_tokens;
         for (int i = 0; i < nv; ++i) {
-            const int64_t phys = (p.first_tok + a0 + i) % p.ring_tokens;
-            const int64_t r = (int64_t)h * p.ring_tokens + phys;
+            const int64_t r = base + phys;
             acc = __fadd_rn(acc, __fmul_rn((float)p.k8[r * p.D + c], p.ks[r]));
+            if (++phys == p.ring_tokens) phys = 0;
         }
     } else {
         const int64_t a0 = (int64_t)(cand - p.n_hist_tiles) * kTile;
@@ -190,7 +191,13 @@ __global__ void kmean_kernel(MaskParams p) {
         for (int i = 0; i < nv; ++i)
             acc = __fadd_rn(acc, bf16_at(p.kcur, (a0 + i) * p.tok_stride + (int64_t)h * p.head_stride + c));
     }
-    reinterpret_cast<float *>(p.buf + p.lay.off_kmean)[idx] = __fdiv_rn(acc, (float)nv);
+    return __fdiv_rn(acc, (float)nv);
+}
+
+__global__ void kmean_kernel(MaskParams p) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)p.H * p.n_cand * p.D) return;
+    reinterpret_cast<float *>(p.buf + p.lay.off_kmean)[idx] = kmean_value(p, idx);
 }
 
 // score[h][b][cand] = fmaf chain over channels in ascending order from +0.0f.  One block covers
@@ -420,29 +427,8 @@ __global__ void qmean_to_kernel(MaskParams p, float *qmean) {
 
 __global__ void kmean_to_kernel(MaskParams p, float *kmean) {
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t n = (int64_t)p.H * p.n_cand * p.D;
-    if (idx >= n) return;
-    const int c = (int)(idx % p.D);
-    const int64_t hc = idx / p.D;
-    const int cand = (int)(hc % p.n_cand);
-    const int h = (int)(hc / p.n_cand);
-    float acc = 0.0f;
-    int nv;
-    if (cand < p.n_hist_tiles) {
-        const int64_t a0 = (int64_t)cand * kTile;
-        nv = (int)((a0 + kTile < p.Lh) ? kTile : p.Lh - a0);
-        for (int i = 0; i < nv; ++i) {
-            const int64_t phys = (p.first_tok + a0 + i) % p.ring_tokens;
-            const int64_t r = (int64_t)h * p.ring_tokens + phys;
-            acc = __fadd_rn(acc, __fmul_rn((float)p.k8[r * p.D + c], p.ks[r]));
-        }
-    } else {
-        const int64_t a0 = (int64_t)(cand - p.n_hist_tiles) * kTile;
-        nv = (int)((a0 + kTile < p.Nq) ? kTile : p.Nq - a0);
-        for (int i = 0; i < nv; ++i)
-            acc = __fadd_rn(acc, bf16_at(p.kcur, (a0 + i) * p.tok_stride + (int64_t)h * p.head_stride + c));
-    }
-    kmean[idx] = __fdiv_rn(acc, (float)nv);
+    if (idx >= (int64_t)p.H * p.n_cand * p.D) return;
+    kmean[idx] = kmean_value(p, idx);
 }
 
 __global__ void __launch_bounds__(32 * kScoreQB) score_from_kernel(MaskParams p, const float *qmean_all,

@@ -39,10 +39,14 @@ ATTN_SOURCE = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc", "attn.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_dense_production_traffic.json")
 
 
-def source_digest(path=ATTN_SOURCE):
+def source_digest(paths=(ATTN_SOURCE, os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc", "common.cuh"))):
+    """Digest of the attention kernel's sources (the kernel file and the device helpers it includes)."""
     import hashlib
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def measured_traffic(path=TRAFFIC_FILE):

@@ -255,6 +255,15 @@ const char *nomas_status_string(int status);
  * failed and its error string ("" if none).  Valid until the next failing call on this thread. */
 const char *nomas_last_error(void);
 
+/* Test and diagnostic hook: the limit, in nanoseconds, of every bounded wait inside the attention
+ * kernel (process-wide, default 2 000 000 000 = 2 s; it applies to later nomas_attn_fwd calls).  A
+ * wait that runs out records NOMAS_ETIMEOUT in the cache's device error word, and every role of the
+ * CTA then leaves its loop, lets its in-flight copies and MMAs complete and releases TMEM, so the
+ * device stays usable; the call's output is then undefined.  A limit of 0 makes a wait that its
+ * first poll does not satisfy give up at once, which exercises that path.  Returns the previous
+ * limit. */
+uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,8 @@ NOMAS_STATIC_POOL_FLOATS = 2 << 20
 EXPORTED = ["nomas_kv_cache_bytes", "nomas_kv_cache_init", "nomas_kv_cache_destroy", "nomas_kv_cache_state",
             "nomas_kv_append", "nomas_mask_layout_query", "nomas_mask_bytes", "nomas_mask_build",
             "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string",
-            "nomas_last_error", "nomas_mask_build_static", "nomas_attn_workspace_bytes"]
+            "nomas_last_error", "nomas_mask_build_static", "nomas_attn_workspace_bytes",
+            "nomas_set_wait_limit_ns"]
 
 
 class nomas_cache_dims(ctypes.Structure):
@@ -82,6 +83,7 @@ _sigs = {
     "nomas_device_status": (ctypes.c_int, [_p, _p]),
     "nomas_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nomas_last_error": (ctypes.c_char_p, []),
+    "nomas_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(lib, _name)
@@ -107,6 +109,11 @@ def nomas_status_string(status: int) -> str:
 
 def nomas_last_error() -> str:
     return lib.nomas_last_error().decode()
+
+
+def nomas_set_wait_limit_ns(limit_ns: int) -> int:
+    """Set the attention kernel's bounded-wait limit (ns); returns the previous one."""
+    return int(lib.nomas_set_wait_limit_ns(int(limit_ns)))
 
 
 def make_dims(heads, head_dim, tokens_per_frame, window_frames, capacity_frames, head_store_tokens):

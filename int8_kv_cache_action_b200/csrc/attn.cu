@@ -953,6 +953,12 @@ static int launch_attn(const AttnParams &p, dim3 grid, const CUtensorMap *maps, 
 
 using namespace nomas;
 
+extern "C" uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns) {
+    const uint64_t prev = g_timeout_ns;
+    g_timeout_ns = limit_ns;
+    return prev;
+}
+
 extern "C" size_t nomas_attn_workspace_bytes(const nomas_kv_cache *c, const nomas_segment_text *seg) {
     nomas_mask_layout lay;
     if (compute_mask_layout(c, seg, NOMAS_MODE_DENSE, 0.25f, &lay) != NOMAS_OK) return 0;

@@ -68,22 +68,27 @@ struct Watchdog {
     int where;
 };
 
-// Wait for phase `parity` of `bar` to complete, giving up after wd.limit_ns.  The limit is checked
-// after the first unsuccessful poll and then every 32 polls (a limit of 0 gives up after one poll).
+// Wait for phase `parity` of `bar` to complete, giving up after wd.limit_ns (checked every 32 polls;
+// a limit of 0 gives up right after the first unsuccessful poll, without reading the timer).
 // Returns false when the CTA is aborting (this wait or another one ran out).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const Watchdog &wd, int site) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (wd.limit_ns == 0) {
+        set_device_error(wd.err, NOMAS_ETIMEOUT, wd.where * 100 + site);
+        *wd.abort = 1;
+        return false;
+    }
     const uint64_t t0 = globaltimer_ns();
     while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (*wd.abort) return false;
-        if (globaltimer_ns() - t0 >= wd.limit_ns) {
+        if (globaltimer_ns() - t0 > wd.limit_ns) {
             set_device_error(wd.err, NOMAS_ETIMEOUT, wd.where * 100 + site);
             *wd.abort = 1;
             return false;
         }
-#pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
     }
 }
 

@@ -202,32 +202,36 @@ def run_ours(args, rank, world, local_rank):
         if rc != 0:
             raise N.NomasError(rc, what)
 
-    def step(ev=None):
+    bufs0 = {"q": q, "kc": kc, "vc": vc, "kt": kt, "vt": vt, "pk": pk, "pv": pv, "out_d": out_d, "out_s": out_s}
+
+    def step(ev=None, b=bufs0, stream=None):
+        sh = s if stream is None else stream.cuda_stream
+        rs = st if stream is None else stream
         if ev is not None:
-            ev[0].record(st)
-        check(N.nomas_kv_append(cache.handle, pk.data_ptr(), pv.data_ptr(), pk.stride(0), pk.stride(1),
-                                n_frames_prev, 0, 0, 0, s), "append")
+            ev[0].record(rs)
+        check(N.nomas_kv_append(cache.handle, b["pk"].data_ptr(), b["pv"].data_ptr(), b["pk"].stride(0),
+                                b["pk"].stride(1), n_frames_prev, 0, 0, 0, sh), "append")
         if ev is not None:
-            ev[1].record(st)
-        check(N.nomas_mask_build(cache.handle, seg, 0, 0.25, 0, 0, ts, hs, mbuf_d.data_ptr(), s), "mask dense")
+            ev[1].record(rs)
+        check(N.nomas_mask_build(cache.handle, seg, 0, 0.25, 0, 0, ts, hs, mbuf_d.data_ptr(), sh), "mask dense")
         if ev is not None:
-            ev[2].record(st)
-        check(N.nomas_attn_fwd(cache.handle, seg, 0, 0.25, mbuf_d.data_ptr(), q.data_ptr(), kc.data_ptr(),
-                               vc.data_ptr(), kt.data_ptr(), vt.data_ptr(), ts, hs, scale, out_d.data_ptr(), 0,
-                               ws.data_ptr(), s),
+            ev[2].record(rs)
+        check(N.nomas_attn_fwd(cache.handle, seg, 0, 0.25, mbuf_d.data_ptr(), b["q"].data_ptr(), b["kc"].data_ptr(),
+                               b["vc"].data_ptr(), b["kt"].data_ptr(), b["vt"].data_ptr(), ts, hs, scale,
+                               b["out_d"].data_ptr(), 0, ws.data_ptr(), sh),
               "attn dense")
         if ev is not None:
-            ev[3].record(st)
-        check(N.nomas_mask_build(cache.handle, seg, 1, 0.25, q.data_ptr(), kc.data_ptr(), ts, hs,
-                                 mbuf_s.data_ptr(), s), "mask sparse")
+            ev[3].record(rs)
+        check(N.nomas_mask_build(cache.handle, seg, 1, 0.25, b["q"].data_ptr(), b["kc"].data_ptr(), ts, hs,
+                                 mbuf_s.data_ptr(), sh), "mask sparse")
         if ev is not None:
-            ev[4].record(st)
-        check(N.nomas_attn_fwd(cache.handle, seg, 1, 0.25, mbuf_s.data_ptr(), q.data_ptr(), kc.data_ptr(),
-                               vc.data_ptr(), kt.data_ptr(), vt.data_ptr(), ts, hs, scale, out_s.data_ptr(), 0,
-                               ws.data_ptr(), s),
+            ev[4].record(rs)
+        check(N.nomas_attn_fwd(cache.handle, seg, 1, 0.25, mbuf_s.data_ptr(), b["q"].data_ptr(), b["kc"].data_ptr(),
+                               b["vc"].data_ptr(), b["kt"].data_ptr(), b["vt"].data_ptr(), ts, hs, scale,
+                               b["out_s"].data_ptr(), 0, ws.data_ptr(), sh),
               "attn sparse")
         if ev is not None:
-            ev[5].record(st)
+            ev[5].record(rs)
 
     for _ in range(args.warmup):
         step()
@@ -271,32 +275,55 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ph = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(n_ph)) for i in range(5)]
 
-    # end to end: pinned host inputs -> device, the same C-ABI calls, device -> host of the outputs
+    # end to end: every step copies its inputs from pinned host memory, runs the same C-ABI calls and
+    # copies both outputs back.  Like a serving loop, the copies of one step overlap the compute of
+    # its neighbours: two device buffer sets, an H2D stream, the compute stream and a D2H stream,
+    # ordered by events (inputs of set i are rewritten only after the compute that read them, outputs
+    # of set i only after their D2H).  The timed region runs from before the first H2D copy to after
+    # the last D2H copy.
     e2e = None
     if rank == 0 or world > 1:
-        host = {n: t.cpu().pin_memory() for n, t in (("q", q), ("kc", kc), ("vc", vc), ("kt", kt), ("vt", vt),
-                                                     ("pk", pk), ("pv", pv))}
-        hout = torch.empty(out_d.shape, dtype=torch.float32).pin_memory()
-        hout2 = torch.empty(out_s.shape, dtype=torch.float32).pin_memory()
+        names = ("q", "kc", "vc", "kt", "vt", "pk", "pv")
+        host = {n: bufs0[n].cpu().pin_memory() for n in names}
+        bufs1 = {n: torch.empty_like(bufs0[n]) for n in names + ("out_d", "out_s")}
+        sets = [bufs0, bufs1]
+        hout = [[torch.empty(out_d.shape, dtype=torch.float32).pin_memory() for _ in range(2)] for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = 2 * hout.numel() * 4
-        dst = {"q": q, "kc": kc, "vc": vc, "kt": kt, "vt": vt, "pk": pk, "pv": pv}
-        n_e2e = max(2, min(args.steps, 5))
+        d2h = 2 * out_d.numel() * 4
+        s_h2d, s_d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        done = [torch.cuda.Event() for _ in range(2)]
+        ready = [torch.cuda.Event() for _ in range(2)]
+        out_free = [torch.cuda.Event() for _ in range(2)]
+        n_e2e = max(4, min(args.steps, 12))
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        e0.record(st)
-        for _ in range(n_e2e):
-            for n, t in host.items():
-                dst[n].copy_(t, non_blocking=True)
-            step()
-            hout.copy_(out_d, non_blocking=True)
-            hout2.copy_(out_s, non_blocking=True)
-        e1.record(st)
+        e0.record(s_h2d)
+        for k in range(n_e2e):
+            i = k % 2
+            b = sets[i]
+            if k >= 2:
+                s_h2d.wait_event(done[i])          # step k-2 has finished reading set i
+            with torch.cuda.stream(s_h2d):
+                for n in names:
+                    b[n].copy_(host[n], non_blocking=True)
+            ready[i].record(s_h2d)
+            st.wait_event(ready[i])
+            if k >= 2:
+                st.wait_event(out_free[i])         # the D2H of step k-2 has read set i's outputs
+            step(b=b, stream=st)
+            done[i].record(st)
+            s_d2h.wait_event(done[i])
+            with torch.cuda.stream(s_d2h):
+                hout[i][0].copy_(b["out_d"], non_blocking=True)
+                hout[i][1].copy_(b["out_s"], non_blocking=True)
+            out_free[i].record(s_d2h)
+        e1.record(s_d2h)
         torch.cuda.synchronize()
         ems = e0.elapsed_time(e1) / n_e2e
         e2e = {"value": (flops_dense + flops_sparse) / (ems * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": n_e2e,
+               "pipelined": "H2D / compute / D2H on three streams, two buffer sets"}
     return dict(ms=ms, phases=ph, flops_dense=flops_dense, flops_sparse=flops_sparse, append_bytes=append_bytes,
                 clocks=clk.summary(), e2e=e2e, cfg=cfg)
 

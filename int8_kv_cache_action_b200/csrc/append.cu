@@ -43,13 +43,37 @@ __device__ __forceinline__ void unpack16(const uint4 &w0, const uint4 &w1, float
     }
 }
 
+// s = RN(a / 127) for a = absmax of bf16 values, without the division routine: q0 = RN(a c) with
+// c = RN(1/127), the remainder a - 127 q0 is exact by FMA, and s = RN(q0 + (a - 127 q0) c) is
+// Markstein's correction step ("Computation of elementary functions on the IBM RISC System/6000
+// processor", 1990).  Checked by exact rational arithmetic against RN(a / 127) for every bf16 a in
+// [2^-110, max finite], where q0 and s are normals and the remainder (a subnormal at the low end) is
+// exact; zero gives zero, and subnormal or non-finite a take the IEEE division.
+__device__ __forceinline__ float div127(float a) {
+    constexpr float c = 0x1.020408p-7f;                   // RN(1/127)
+    const float q0 = __fmul_rn(a, c);
+    const float s = __fmaf_rn(__fmaf_rn(-q0, 127.0f, a), c, q0);
+    if (!(a >= 0x1p-110f && a <= 0x1.fffffep127f) && a != 0.0f) return __fdiv_rn(a, 127.0f);
+    return s;
+}
+
+// 1/s for normal s: the hardware approximation (PTX rcp.approx.f32, relative error about 2^-23)
+// refined by one Newton-Raphson step r = r0 + r0 (1 - s r0), both by FMA, leaves a relative error
+// below 2^-24 + 2^-40.
+__device__ __forceinline__ float recip_nr(float s) {
+    float r0;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r0) : "f"(s));
+    return __fmaf_rn(r0, __fmaf_rn(-s, r0, 1.0f), r0);
+}
+
 // Codes rint(x / s) in fp32 with IEEE division and round-half-even for the 16 channels this lane
 // holds; s = RN(absmax / 127) over the group's D channels, so |x / s| <= 127 (1 + 2^-23) and every
 // code lies in [-127, 127].
-// y = x * RN(1/s) is within 2^-16 + 2^-17 of RN(x/s) for |x/s| <= 127 (two roundings of relative
-// size 2^-24 each, one more for RN(x/s) itself), so when y is farther than 2^-15 from the nearest
-// half-integer both round to the same integer.  Otherwise (rare, and always when 1/s overflows) the
-// exact quotient decides; the warp takes that branch only when one of its lanes needs it.
+// y = x * r with r = 1/s to relative 2^-24 + 2^-40 is within 2^-16 + 2^-17 of RN(x/s) for
+// |x/s| <= 127 (about 127 * 2^-23 from r and the rounding of y, 2^-18 for RN(x/s) itself), so when y
+// is farther than 2^-15 from the nearest half-integer both round to the same integer.  Otherwise
+// the exact quotient decides: rarely, and always for s below 2^-125, where r is a NaN.  The warp
+// takes that branch only when one of its lanes needs it.
 // Rounding uses t = y + 1.5 * 2^23: the fp32 add rounds y half-to-even to an integer and leaves it,
 // as a two's-complement byte, in the low byte of t's bit pattern; y - (t - 1.5 * 2^23) is exact.
 template <int LPV>
@@ -60,10 +84,10 @@ __device__ __forceinline__ uint4 quant16(const float (&x)[16], float &s_out) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
     a = group_max<LPV>(a);
-    const float s = __fdiv_rn(a, 127.0f);
+    const float s = div127(a);
     s_out = s;
     const bool nz = s > 0.0f;
-    const float r = nz ? __frcp_rn(s) : 0.0f;
+    const float r = s >= 0x1p-125f ? recip_nr(s) : (nz ? __int_as_float(0x7fffffff) : 0.0f);
     const float2 r2 = make_float2(r, r), m2 = make_float2(kMagic, kMagic), nm2 = make_float2(-kMagic, -kMagic);
     const float2 neg1 = make_float2(-1.0f, -1.0f);
     uint32_t tb[16];
@@ -74,7 +98,7 @@ __device__ __forceinline__ uint4 quant16(const float (&x)[16], float &s_out) {
         const float2 t = __fadd2_rn(y, m2);
         const float2 q = __fadd2_rn(t, nm2);
         const float2 d = __ffma2_rn(q, neg1, y);          // y - rint(y), exact
-        slow |= !(fabsf(d.x) < kFar) || !(fabsf(d.y) < kFar);   // NaN (1/s overflowed) counts as near
+        slow |= !(fabsf(d.x) < kFar) || !(fabsf(d.y) < kFar);   // NaN (tiny s) counts as near
         tb[2 * i] = __float_as_uint(t.x);
         tb[2 * i + 1] = __float_as_uint(t.y);
     }

@@ -111,3 +111,52 @@ def test_capacity_and_argument_errors_leave_cache_unchanged():
     assert rc == N.NOMAS_EINVAL
     st = gc.state()
     assert st["frames_appended"] == 2 and st["head_tokens"] == 0 and st["segments"] == 1
+
+
+def _adversarial_rows(D, seed=5):
+    """bf16 rows (float32 values) whose absmax runs over every positive finite bf16 value, each with
+    random other channels below it, plus rows of zeros, single subnormals, exact half-integer ties at a
+    power-of-two scale and values at the bf16 maximum."""
+    rng = np.random.default_rng(seed)
+    bits = np.arange(0x0001, 0x7F80, dtype=np.uint32)                 # subnormals and normals
+    a = (bits << 16).view(np.float32)
+    n = a.shape[0]
+    frac = rng.uniform(-1.0, 1.0, size=(n, D)).astype(np.float32)
+    rows = (frac * a[:, None]).astype(np.float32)
+    rows[np.arange(n), rng.integers(0, D, n)] = a * rng.choice([-1.0, 1.0], n).astype(np.float32)
+    extra = []
+    extra.append(np.zeros(D, np.float32))
+    z = np.zeros(D, np.float32)
+    z[3] = np.float32(2.0 ** -133)
+    extra.append(z)
+    for k in (-100, -20, 0, 3, 50, 120):                           # s = 2^k, x = (j + 1/2) 2^k: ties
+        j = rng.integers(-127, 127, D).astype(np.float32)
+        x = ((j + np.float32(0.5)) * np.float32(2.0 ** k)).astype(np.float32)
+        x[0] = np.float32(127 * 2.0 ** k)
+        extra.append(x)
+    big = np.float32((np.uint32(0x7F7F) << 16).view(np.float32))
+    extra.append(rng.choice([-1.0, 1.0], D).astype(np.float32) * big)
+    rows = np.concatenate([rows, np.stack(extra)])
+    # round to bf16 (the half-integer ties and the powers of two above are exact in bf16)
+    rows = torch.from_numpy(rows).bfloat16()
+    return rows
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_append_every_bf16_absmax(D):
+    """Codes and scales bit-exact for groups whose absmax is each positive bf16 value in turn."""
+    from int8_kv_cache_action_b200.runtime import KVCache
+    from oracle.ring import OracleCache
+    rows = _adversarial_rows(D)
+    H, T = 4, 64
+    n_tok = (rows.shape[0] + H * T - 1) // (H * T) * T
+    pad = torch.zeros(n_tok * H - rows.shape[0], D, dtype=torch.bfloat16)
+    k = torch.cat([rows, pad]).reshape(n_tok, H, D)
+    v = torch.flip(k, dims=[0])                                      # a different row order for V
+    frames = n_tok // T
+    gc = KVCache(H, D, T, 0, frames, 8)
+    oc = OracleCache(H, D, T, 0, frames, 8)
+    gc.append(k.cuda(), v.cuda(), frames)
+    oc.append(f32(k), f32(v), frames, None, None)
+    _compare_cache(gc, oc)
+    assert gc.status() == 0

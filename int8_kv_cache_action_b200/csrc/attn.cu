@@ -5,9 +5,8 @@
 //   warps 0-3   softmax over key columns 0-63 of every S tile (TMEM lanes 0-127, one thread per row)
 //   warps 4-7   softmax over key columns 64-127; the two halves of a row swap their maxima through
 //               shared memory, so both apply the same offset
-//   warps 8-11  converter: per-column key scale, value scale and visibility window; an INT8 tile,
-//               which TMA lands in the upper half of its slot, becomes exact fp16 codes in place;
-//               each warp converts its own rows
+//   warps 8-11  column info: per-column key scale, value scale and visibility window of every
+//               tile, one tile ahead, in a four-deep shared-memory ring
 //   warp 12     tcgen05.mma issuer (one thread) and TMEM owner
 //   warp 13     TMA producer (one thread); warps 14-15 idle
 // The register file is split per SM sub-partition (one warp of each warpgroup on each), so the
@@ -26,6 +25,14 @@
 // two batches in flight, which the S -> softmax -> PV dependency does not allow.  The issue order
 // S_0, S_1, PV_0, S_2, PV_1, ... computes S_{j+1} while the softmax works on S_j; S_{j+2} reuses
 // the buffer of S_j after PV_j, which tcgen05's in-order execution makes safe.
+//
+// Every tile reaches shared memory by TMA alone.  The pre-pass writes the operands in the layouts
+// the boxes read: fp16 keys [H][n][D] and transposed fp16 values [H][D][n] for the current segment
+// and the text (converted from bf16), and for the retained history and the description heads the
+// INT8 codes as exact fp16 integers in the same layouts (-127..127 are exact in fp16), with their
+// scales in age order.  Converting the codes once per call in the pre-pass costs one HBM pass over
+// the history; converting them in shared memory inside this kernel took issue slots from the
+// softmax warps on every history tile of every query block.
 //
 // Precision: every MMA operand is fp16 with fp32 accumulation.  bf16 inputs convert to fp16
 // exactly for magnitudes in [2^-14, 65504] (the supported input range; smaller values keep 2^-24
@@ -55,11 +62,9 @@ struct AttnCfg {
     static constexpr int NK = (D == 128) ? 3 : 6;          // K tile slots
     static constexpr int NV = NK;                          // V^T tile slots
     static constexpr int SLOT = kTile * D * 2;             // one fp16 tile
-    static constexpr int HALF = SLOT / 2;                  // an INT8 tile lands in the upper half
     static constexpr int KPANEL = kTile * 128;             // K: 64 columns (128 B) of 128 rows
     static constexpr int VPANEL = D * 128;                 // V^T: 64 keys (128 B) of D rows
     static constexpr int KSTEPS = D / 16;
-    static constexpr int CHUNKS = kTile * D / 16 / 128;    // 16-byte INT8 chunks per converter thread
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + NK * SLOT;
     static constexpr int OFF_CS = OFF_V + NV * SLOT;       // float [kNCI][128] key scale x log2 e
@@ -68,13 +73,12 @@ struct AttnCfg {
     static constexpr int OFF_XM = OFF_CW + kNCI * 1024;    // float [2 buffers][2 halves][128] maxima
     static constexpr int OFF_XL = OFF_XM + 2048;           // float [2 halves][128] row sums
     static constexpr int OFF_BAR = OFF_XL + 1024;
-    // q_ready; k_full, k_empty, k_tma [NK]; v_full, v_empty, v_tma [NV]; ci_full, ci_empty [kNCI];
+    // q_ready; k_full, k_empty [NK]; v_full, v_empty [NV]; ci_full, ci_empty [kNCI];
     // s_full, p_full, xm_bar [2]; pv_done; o_final; xl_bar
-    static constexpr int NBAR = 1 + 3 * NK + 3 * NV + 2 * kNCI + 6 + 3;
+    static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 * kNCI + 6 + 3;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int SMEM = BYTES + 1024;              // slack for 1024-byte alignment
-    static_assert(CHUNKS * 128 * 16 == kTile * D, "converter chunk split");
 };
 
 struct AttnParams {
@@ -204,9 +208,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float *sXL = reinterpret_cast<float *>(sm + C::OFF_XL);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
     uint64_t *q_ready = bars;
-    uint64_t *k_full = bars + 1, *k_empty = k_full + C::NK, *k_tma = k_empty + C::NK;
-    uint64_t *v_full = k_tma + C::NK, *v_empty = v_full + C::NV, *v_tma = v_empty + C::NV;
-    uint64_t *ci_full = v_tma + C::NV, *ci_empty = ci_full + kNCI;
+    uint64_t *k_full = bars + 1, *k_empty = k_full + C::NK;
+    uint64_t *v_full = k_empty + C::NK, *v_empty = v_full + C::NV;
+    uint64_t *ci_full = v_empty + C::NV, *ci_empty = ci_full + kNCI;
     uint64_t *s_full = ci_empty + kNCI, *p_full = s_full + 2, *xm_bar = p_full + 2;
     uint64_t *pv_done = xm_bar + 2, *o_final = pv_done + 1, *xl_bar = o_final + 1;
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC);
@@ -237,14 +241,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(q_ready, 8);
         for (int i = 0; i < C::NK; ++i) {
-            mbar_init(&k_full[i], 4);
+            mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], 1);
-            mbar_init(&k_tma[i], 1);
         }
         for (int i = 0; i < C::NV; ++i) {
-            mbar_init(&v_full[i], 4);
+            mbar_init(&v_full[i], 1);
             mbar_init(&v_empty[i], 1);
-            mbar_init(&v_tma[i], 1);
         }
         for (int i = 0; i < kNCI; ++i) {
             mbar_init(&ci_full[i], 4);
@@ -274,18 +276,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int64_t qrow0 = (int64_t)qb * kTile;
 
     if (warp >= 8 && warp < 12) {
-        // ------------------------------------------------------------------ converter warpgroup
-        // Each warp works on its own rows and signals the barriers itself (full barriers count four
-        // converter warps; the producer adds three arrivals when TMA alone fills a slot).  An INT8
-        // row and the second fp16 panel of the same row occupy the same 128 bytes of the slot, and
-        // the first panel lies below the INT8 half, so for D = 128 (and for V^T at any D) the eight
-        // lanes that share a row only need __syncwarp between reading it and writing over it.  Keys
-        // at D = 64 overlap across warps and take a named barrier, followed by a read of the shared
-        // abort decision so that all converter warps leave together.
+        // ------------------------------------------------------------------ column-info warpgroup
+        // Thread t writes column t of every tile's entry in the ring; each warp arrives on ci_full
+        // for its 32 columns.
         setmaxnreg_dec<kRegLoader>();
         wd.where = 3;
         const int t = threadIdx.x - 256;   // 0..127
-        const int kc = t % 8;               // V^T: this thread's 16-key chunk in every row it converts
         struct ColInfo {
             float ks, vs;   // raw key / value scale (cached tiles), 1 / 0 otherwise
             int2 w;
@@ -313,88 +309,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             return ci;
         };
-        // Waits are warp-wide for D = 128; at D = 64 the key conversion needs all four warps, so there
-        // every wait ends in a named barrier whose OR-reduced abort flag all four warps agree on.
-        auto conv_wait = [&](uint64_t *bar, uint32_t par, int site) -> bool {
-            if constexpr (D == 64) {
-                mbar_wait(bar, par, wd, site);
-                return !named_bar_or(1, 128, *abort_flag != 0);
-            } else {
-                return __all_sync(0xffffffffu, mbar_wait(bar, par, wd, site));
-            }
-        };
         ListCursor cursor(list, n_tiles);
-        uint32_t kpar = 0, vpar = 0;        // per slot: parity of the next INT8 landing
         int u = 0;                          // index among this block's tiles
         int4 en;
         bool have = cursor.next(use_bit, en);
         ColInfo nxt;
         if (have) nxt = col_info(en);
-        bool ok = true;
         while (have) {
-            const int4 e = en;
-            const bool cached = is_cached(e.x & 3);
             const ColInfo cur = nxt;
             have = cursor.next(use_bit, en);
             if (have) nxt = col_info(en);
             const int ci = u % kNCI;
-            ok = conv_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, 1);
-            if (!ok) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, wd, 1))) break;
             sCS[ci * 128 + t] = p.scale_log2 * cur.ks;
             sCV[ci * 128 + t] = cur.vs;
             sCW[ci * 128 + t] = cur.w;
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_full[ci]);
-            if (cached) {
-                // keys: INT8 codes in the upper half of the slot -> exact fp16 codes over the slot
-                const int sk = u % C::NK;
-                uint8_t *slot = sK + sk * C::SLOT;
-                uint4 raw[C::CHUNKS];
-                ok = conv_wait(&k_tma[sk], (kpar >> sk) & 1u, 2);
-                if (!ok) break;
-                kpar ^= 1u << sk;
-#pragma unroll
-                for (int i = 0; i < C::CHUNKS; ++i) raw[i] = reinterpret_cast<const uint4 *>(slot + C::HALF)[t + 128 * i];
-                if constexpr (D == 64) {
-                    named_bar_sync(1, 128);   // every code is in registers before any fp16 lands on it
-                } else {
-                    __syncwarp();             // the row's eight chunks are read before its panel 1 is written
-                }
-#pragma unroll
-                for (int i = 0; i < C::CHUNKS; ++i) {
-                    const int idx = t + 128 * i;
-                    const int row = idx / (D / 16), c = idx % (D / 16);
-                    uint4 lo, hi;
-                    i8x16_to_f16(raw[i], lo, hi);
-                    uint8_t *base = slot + (c / 4) * C::KPANEL;
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(row, (c % 4) * 2)) = lo;
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(row, (c % 4) * 2 + 1)) = hi;
-                }
-                // values: V^T INT8 rows -> exact fp16 codes (the softmax multiplies P by the value scale)
-                const int sv = u % C::NV;
-                ok = conv_wait(&v_tma[sv], (vpar >> sv) & 1u, 3);
-                if (!ok) break;
-                vpar ^= 1u << sv;
-                slot = sV + sv * C::SLOT;
-#pragma unroll
-                for (int i = 0; i < C::CHUNKS; ++i) raw[i] = reinterpret_cast<const uint4 *>(slot + C::HALF)[t + 128 * i];
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < C::CHUNKS; ++i) {
-                    const int d = (t + 128 * i) / 8;
-                    uint4 lo, hi;
-                    i8x16_to_f16(raw[i], lo, hi);
-                    uint8_t *base = slot + (kc / 4) * C::VPANEL;
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(d, (kc % 4) * 2)) = lo;
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(d, (kc % 4) * 2 + 1)) = hi;
-                }
-                fence_proxy_async_smem();   // one fence publishes both tiles to the tensor core
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&k_full[sk]);
-                    mbar_arrive(&v_full[sv]);
-                }
-            }
             ++u;
         }
     } else if (warp >= 12) {
@@ -453,66 +384,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             prefetch_tmap(&tm_vc);
             prefetch_tmap(&tm_kh);
             prefetch_tmap(&tm_vh);
-            uint32_t kpar = 0, vpar = 0;             // per slot: parity of the next INT8 landing
             uint32_t kpend = 0, vpend = 0;           // per slot: a copy was issued
-            uint32_t kwait8 = 0, vwait8 = 0;         // per slot: it signals the INT8 barrier
-            uint32_t kwpar = 0, vwpar = 0;           // per slot: parity of that signal
+            uint32_t kwpar = 0, vwpar = 0;           // per slot: parity of the phase it completes
             int u = 0;
             ListCursor cursor(list, n_tiles);
             int4 e;
             while (cursor.next(use_bit, e)) {
                 const int kind = e.x & 3;
                 const int start = e.y;
-                const bool cached = is_cached(kind);
-                const bool hist = kind == kKindHist;
+                const CUtensorMap *mk = kind == kKindCur ? &tm_kc : kind == kKindText ? &tm_kt
+                                      : kind == kKindHist ? &tm_kh : &tm_kp;
+                const CUtensorMap *mv = kind == kKindCur ? &tm_vc : kind == kKindText ? &tm_vt
+                                      : kind == kKindHist ? &tm_vh : &tm_vp;
                 const int sk = u % C::NK;
                 if (!mbar_wait(&k_empty[sk], ((u / C::NK) & 1) ^ 1, wd, 1)) break;
                 uint8_t *dk = sK + sk * C::SLOT;
-                if (!cached) {
-                    mbar_arrive_expect_tx(&k_full[sk], C::SLOT);
-                    mbar_arrive_cnt(&k_full[sk], 3);   // stands in for the converter warps
+                mbar_arrive_expect_tx(&k_full[sk], C::SLOT);
 #pragma unroll
-                    for (int hh = 0; hh < D / 64; ++hh)
-                        tma_load_3d(dk + hh * C::KPANEL, kind == kKindCur ? &tm_kc : &tm_kt, &k_full[sk], hh * 64,
-                                    start, h);
-                    kwait8 &= ~(1u << sk);
-                    kwpar = (kwpar & ~(1u << sk)) | ((uint32_t)((u / C::NK) & 1) << sk);
-                } else {
-                    mbar_arrive_expect_tx(&k_tma[sk], C::HALF);
-                    tma_load_3d(dk + C::HALF, hist ? &tm_kh : &tm_kp, &k_tma[sk], 0, start, h);
-                    kwait8 |= 1u << sk;
-                    kwpar = (kwpar & ~(1u << sk)) | (((kpar >> sk) & 1u) << sk);
-                    kpar ^= 1u << sk;
-                }
+                for (int hh = 0; hh < D / 64; ++hh) tma_load_3d(dk + hh * C::KPANEL, mk, &k_full[sk], hh * 64, start, h);
                 kpend |= 1u << sk;
+                kwpar = (kwpar & ~(1u << sk)) | ((uint32_t)((u / C::NK) & 1) << sk);
                 const int sv = u % C::NV;
                 if (!mbar_wait(&v_empty[sv], ((u / C::NV) & 1) ^ 1, wd, 2)) break;
                 uint8_t *dv = sV + sv * C::SLOT;
-                if (!cached) {
-                    mbar_arrive_expect_tx(&v_full[sv], C::SLOT);
-                    mbar_arrive_cnt(&v_full[sv], 3);
+                mbar_arrive_expect_tx(&v_full[sv], C::SLOT);
 #pragma unroll
-                    for (int pp = 0; pp < 2; ++pp)
-                        tma_load_3d(dv + pp * C::VPANEL, kind == kKindCur ? &tm_vc : &tm_vt, &v_full[sv],
-                                    start + 64 * pp, 0, h);
-                    vwait8 &= ~(1u << sv);
-                    vwpar = (vwpar & ~(1u << sv)) | ((uint32_t)((u / C::NV) & 1) << sv);
-                } else {
-                    mbar_arrive_expect_tx(&v_tma[sv], C::HALF);
-                    tma_load_3d(dv + C::HALF, hist ? &tm_vh : &tm_vp, &v_tma[sv], start, 0, h);
-                    vwait8 |= 1u << sv;
-                    vwpar = (vwpar & ~(1u << sv)) | (((vpar >> sv) & 1u) << sv);
-                    vpar ^= 1u << sv;
-                }
+                for (int pp = 0; pp < 2; ++pp) tma_load_3d(dv + pp * C::VPANEL, mv, &v_full[sv], start + 64 * pp, 0, h);
                 vpend |= 1u << sv;
+                vwpar = (vwpar & ~(1u << sv)) | ((uint32_t)((u / C::NV) & 1) << sv);
                 ++u;
             }
             // the bulk copies must land before the CTA's shared memory is released (a no-op unless
             // this CTA is aborting)
             for (int i = 0; i < C::NK; ++i)
-                if ((kpend >> i) & 1u) mbar_drain(((kwait8 >> i) & 1u) ? &k_tma[i] : &k_full[i], (kwpar >> i) & 1u, 100000000ull);
+                if ((kpend >> i) & 1u) mbar_drain(&k_full[i], (kwpar >> i) & 1u, 100000000ull);
             for (int i = 0; i < C::NV; ++i)
-                if ((vpend >> i) & 1u) mbar_drain(((vwait8 >> i) & 1u) ? &v_tma[i] : &v_full[i], (vwpar >> i) & 1u, 100000000ull);
+                if ((vpend >> i) & 1u) mbar_drain(&v_full[i], (vwpar >> i) & 1u, 100000000ull);
         }
         __syncwarp();
     } else {
@@ -784,14 +691,16 @@ __global__ void __launch_bounds__(256) values_t16_kernel(VtJobs jobs) {
     }
 }
 
-// INT8 history in age order for the attention kernel's TMA boxes:
-//   z = 0: ring rows of the retained history -> K8 rows [H][Lh][D], V^T [H][D][lhp] (lhp = Lh rounded
-//          up to 16, zero padding), key / value scales [H][lhp];
-//   z = 1: description-head store rows [0, Lp) -> V^T [H][D][lpp] (keys and scales are read in place).
+// INT8 codes of the cache as exact fp16 integers, in the layouts of the attention kernel's TMA boxes:
+//   z = 0: ring rows of the retained history in age order -> keys [H][Lh][D], V^T [H][D][lhp] (lhp =
+//          Lh rounded up to 16, zero padding), key / value scales [H][lhp];
+//   z = 1: description-head store rows [0, Lp) -> keys [H][Lp][D], V^T [H][D][lpp] (its scales are
+//          read in place).
+// One block converts 64 tokens x D of one head; values are transposed through shared memory.
 struct HistPrep {
-    const int8_t *k8, *v8, *hv8;
+    const int8_t *k8, *v8, *hk8, *hv8;
     const float *ks, *vs;
-    int8_t *k8l, *v8t, *hv8t;
+    __half *kh, *vht, *kp, *vpt;
     float *ksl, *vsl;
     int64_t ring_tokens, first_tok, Lh, lhp, Lp, lpp, head_rows;
     int32_t H, D;
@@ -806,6 +715,8 @@ __global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
     if (t0 >= np) return;
     const int D = P.D;
     const int cpr = D / 16;
+    const int8_t *ksrc = heads ? P.hk8 : P.k8, *vsrc = heads ? P.hv8 : P.v8;
+    __half *kdst = heads ? P.kp : P.kh;
     auto src_row = [&](int64_t a) -> int64_t {
         return heads ? (int64_t)h * P.head_rows + a : (int64_t)h * P.ring_tokens + (P.first_tok + a) % P.ring_tokens;
     };
@@ -815,10 +726,12 @@ __global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
         uint4 v = make_uint4(0, 0, 0, 0);
         if (a < n) {
             const int64_t sr = src_row(a);
-            v = __ldg(reinterpret_cast<const uint4 *>((heads ? P.hv8 : P.v8) + sr * D) + c);
-            if (!heads)
-                reinterpret_cast<uint4 *>(P.k8l + ((int64_t)h * P.Lh + a) * D)[c] =
-                    __ldg(reinterpret_cast<const uint4 *>(P.k8 + sr * D) + c);
+            v = __ldg(reinterpret_cast<const uint4 *>(vsrc + sr * D) + c);
+            uint4 lo, hi;
+            i8x16_to_f16(__ldg(reinterpret_cast<const uint4 *>(ksrc + sr * D) + c), lo, hi);
+            uint4 *kd = reinterpret_cast<uint4 *>(kdst + ((int64_t)h * n + a) * D) + 2 * c;
+            kd[0] = lo;
+            kd[1] = hi;
         }
         *reinterpret_cast<uint4 *>(&tile[r][c * 16]) = v;
     }
@@ -836,7 +749,7 @@ __global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
         }
     }
     __syncthreads();
-    int8_t *dst = heads ? P.hv8t : P.v8t;
+    __half *dst = heads ? P.vpt : P.vht;
     for (int i = threadIdx.x; i < D * 4; i += blockDim.x) {
         const int d = i / 4, c = i % 4;   // row d, tokens [t0 + 16c, t0 + 16c + 16)
         const int64_t t = t0 + c * 16;
@@ -847,7 +760,11 @@ __global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
             w[k] = (uint32_t)(uint8_t)tile[c * 16 + 4 * k][d] | ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 1][d] << 8) |
                    ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 2][d] << 16) |
                    ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 3][d] << 24);
-        *reinterpret_cast<uint4 *>(dst + ((int64_t)h * D + d) * np + t) = make_uint4(w[0], w[1], w[2], w[3]);
+        uint4 lo, hi;
+        i8x16_to_f16(make_uint4(w[0], w[1], w[2], w[3]), lo, hi);
+        uint4 *vd = reinterpret_cast<uint4 *>(dst + ((int64_t)h * D + d) * np + t);
+        vd[0] = lo;
+        vd[1] = hi;
     }
 }
 
@@ -900,12 +817,13 @@ static int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 // the size does not depend on the cache state:
 //   kc, kt   fp16 [H][n][D]       current-segment / text keys
 //   vc, vt   fp16 [H][D][np8]     current-segment / text values, transposed
-//   k8l      int8 [H][Lh][D]      retained-history keys in age order
-//   v8t      int8 [H][D][lhp]     retained-history values, transposed
+//   kh       fp16 [H][Lh][D]      retained-history key codes in age order
+//   vht      fp16 [H][D][lhp]     retained-history value codes, transposed
 //   ksl, vsl fp32 [H][lhp]        their scales
-//   hv8t     int8 [H][D][lpp]     description-head values, transposed
+//   kp       fp16 [H][Lp][D]      description-head key codes
+//   vpt      fp16 [H][D][lpp]     description-head value codes, transposed
 struct WsLayout {
-    size_t kc, kt, vc, vt, k8l, v8t, ksl, vsl, hv8t, total;
+    size_t kc, kt, vc, vt, kh, vht, ksl, vsl, kp, vpt, total;
 };
 static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
     const auto &d = c->d;
@@ -924,11 +842,12 @@ static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
     w.kt = take((size_t)H * lt * D * 2);
     w.vc = take((size_t)H * D * round_up(nq, 8) * 2);
     w.vt = take((size_t)H * D * round_up(lt, 8) * 2);
-    w.k8l = take((size_t)H * lh * D);
-    w.v8t = take((size_t)H * D * lhp);
+    w.kh = take((size_t)H * lh * D * 2);
+    w.vht = take((size_t)H * D * lhp * 2);
     w.ksl = take((size_t)H * lhp * 4);
     w.vsl = take((size_t)H * lhp * 4);
-    w.hv8t = take((size_t)H * D * lpp);
+    w.kp = take((size_t)H * d.head_store_tokens * D * 2);
+    w.vpt = take((size_t)H * D * lpp * 2);
     w.total = off;
     return w;
 }
@@ -988,7 +907,7 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     const int64_t Nq = lay.n_query, Lt = lay.text_tokens, Lh = lay.history_tokens, Lp = lay.head_tokens;
     const int64_t nqp = round_up(Nq, 8), ltp = round_up(Lt, 8), lhp = round_up(Lh, 16), lpp = round_up(Lp, 16);
 
-    // ---- pre-pass: fp16 keys, transposed fp16 values, INT8 history in age order
+    // ---- pre-pass: fp16 keys, transposed fp16 values, the history's and heads' codes as fp16
     const WsLayout ws = ws_layout(c, Nq, Lt);
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
     {
@@ -1023,12 +942,14 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
         HistPrep hp{};
         hp.k8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_K8]);
         hp.v8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_V8]);
+        hp.hk8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_HK8]);
         hp.hv8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_HV8]);
         hp.ks = static_cast<const float *>(c->buf[NOMAS_BUF_KS]);
         hp.vs = static_cast<const float *>(c->buf[NOMAS_BUF_VS]);
-        hp.k8l = reinterpret_cast<int8_t *>(wsb + ws.k8l);
-        hp.v8t = reinterpret_cast<int8_t *>(wsb + ws.v8t);
-        hp.hv8t = reinterpret_cast<int8_t *>(wsb + ws.hv8t);
+        hp.kh = reinterpret_cast<__half *>(wsb + ws.kh);
+        hp.vht = reinterpret_cast<__half *>(wsb + ws.vht);
+        hp.kp = reinterpret_cast<__half *>(wsb + ws.kp);
+        hp.vpt = reinterpret_cast<__half *>(wsb + ws.vpt);
         hp.ksl = reinterpret_cast<float *>(wsb + ws.ksl);
         hp.vsl = reinterpret_cast<float *>(wsb + ws.vsl);
         hp.ring_tokens = hv.ring_tokens;
@@ -1049,11 +970,9 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     // ---- tensor maps (an extent of zero gets a one-row map that no tile reads)
     CUtensorMap maps[8];
     {
-        const CUtensorMapDataType F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16, U8 = CU_TENSOR_MAP_DATA_TYPE_UINT8;
+        const CUtensorMapDataType F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
         const cuuint32_t bk[3] = {64, (cuuint32_t)kTile, 1};        // K: 64 columns x 128 keys
         const cuuint32_t bv[3] = {64, (cuuint32_t)D, 1};            // V^T: 64 keys x D rows
-        const cuuint32_t bk8[3] = {(cuuint32_t)D, (cuuint32_t)kTile, 1};
-        const cuuint32_t bv8[3] = {(cuuint32_t)kTile, (cuuint32_t)D, 1};
         auto kmap16 = [&](CUtensorMap *m, size_t off, int64_t n) {
             const int64_t nn = n > 0 ? n : 1;
             const cuuint64_t dm[3] = {(cuuint64_t)D, (cuuint64_t)nn, (cuuint64_t)H};
@@ -1066,22 +985,9 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
             const cuuint64_t sd[2] = {(cuuint64_t)pp * 2, (cuuint64_t)D * pp * 2};
             return make_map(m, F16, wsb + off, dm, sd, bv, CU_TENSOR_MAP_SWIZZLE_128B);
         };
-        auto kmap8 = [&](CUtensorMap *m, const void *base, int64_t n, int64_t head_stride_rows) {
-            const int64_t nn = n > 0 ? n : 1;
-            const cuuint64_t dm[3] = {(cuuint64_t)D, (cuuint64_t)nn, (cuuint64_t)H};
-            const cuuint64_t sd[2] = {(cuuint64_t)D, (cuuint64_t)(head_stride_rows > 0 ? head_stride_rows : 1) * D};
-            return make_map(m, U8, base, dm, sd, bk8, CU_TENSOR_MAP_SWIZZLE_NONE);
-        };
-        auto vmap8 = [&](CUtensorMap *m, size_t off, int64_t n, int64_t np) {
-            const int64_t nn = n > 0 ? n : 1, pp = np > 0 ? np : 16;
-            const cuuint64_t dm[3] = {(cuuint64_t)nn, (cuuint64_t)D, (cuuint64_t)H};
-            const cuuint64_t sd[2] = {(cuuint64_t)pp, (cuuint64_t)D * pp};
-            return make_map(m, U8, wsb + off, dm, sd, bv8, CU_TENSOR_MAP_SWIZZLE_NONE);
-        };
         if (!kmap16(&maps[0], ws.kc, Nq) || !kmap16(&maps[1], ws.kt, Lt) || !vmap16(&maps[2], ws.vc, Nq, nqp) ||
-            !vmap16(&maps[3], ws.vt, Lt, ltp) || !kmap8(&maps[4], wsb + ws.k8l, Lh, Lh) ||
-            !kmap8(&maps[5], c->buf[NOMAS_BUF_HK8], Lp, d.head_store_tokens) || !vmap8(&maps[6], ws.v8t, Lh, lhp) ||
-            !vmap8(&maps[7], ws.hv8t, Lp, lpp))
+            !vmap16(&maps[3], ws.vt, Lt, ltp) || !kmap16(&maps[4], ws.kh, Lh) || !kmap16(&maps[5], ws.kp, Lp) ||
+            !vmap16(&maps[6], ws.vht, Lh, lhp) || !vmap16(&maps[7], ws.vpt, Lp, lpp))
             return NOMAS_ECUDA;
     }
     AttnParams p{};

@@ -11,7 +11,7 @@
 //   warp 13     TMA producer (one thread); warps 14-15 idle
 // The register file is split per SM sub-partition (one warp of each warpgroup on each), so the
 // kernel launches at 128 registers per thread and moves them with setmaxnreg: softmax 168 each,
-// converter 112, MMA / producer warpgroup 64 -- 2*168 + 112 + 64 = 512 = 4 x 128.
+// column info 112, MMA / producer warpgroup 64 -- 2*168 + 112 + 64 = 512 = 4 x 128.
 //
 // TMEM (512 columns): Q (fp16 pairs) at [0, D/2), S double buffer at [128, 256) and [256, 384),
 // O at [384, 384 + D).  P (fp16) overwrites the first 32 columns of each 64-column half of its S

@@ -47,6 +47,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "prep.cuh"
 
 namespace nomas {
 
@@ -117,17 +118,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     return d;
 }
 
-__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
-__device__ __forceinline__ uint32_t f16x2_of(float lo, float hi) {
-    __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
 template <int N>
 __device__ __forceinline__ void setmaxnreg_inc() {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
@@ -135,30 +125,6 @@ __device__ __forceinline__ void setmaxnreg_inc() {
 template <int N>
 __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
-// 16 int8 codes -> 16 exact fp16 values (two 16-byte chunks).  Each biased byte u = b + 128 becomes
-// the low byte of the fp16 pattern 0x64uu = 1024 + u; one packed add of -1152 leaves b exactly.
-__device__ __forceinline__ void i8x16_to_f16(const uint4 &w, uint4 &lo, uint4 &hi) {
-    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-    uint32_t o[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t x = in[i] ^ 0x80808080u;
-        o[2 * i] = hadd2_u32(__byte_perm(x, 0x64646464u, 0x4140), 0xE480E480u);
-        o[2 * i + 1] = hadd2_u32(__byte_perm(x, 0x64646464u, 0x4342), 0xE480E480u);
-    }
-    lo = make_uint4(o[0], o[1], o[2], o[3]);
-    hi = make_uint4(o[4], o[5], o[6], o[7]);
-}
-
-// 8 bf16 -> 8 fp16 (16 bytes in, 16 bytes out).
-__device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 &v) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) o[i] = f16x2_of(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ bool is_cached(int kind) { return kind == kKindHist || kind == kKindPriorHead; }
@@ -611,163 +577,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 }
 
-// ---------------------------------------------------------------------------------------------
-// Pre-pass (HBM-bound): operand copies in the layouts the attention kernel's TMA boxes read.
-// ---------------------------------------------------------------------------------------------
-
-// bf16 [n][H][D] (token / head strides in elements) -> fp16 [H][n][D], for up to two tensors.
-struct F16Job {
-    const __nv_bfloat16 *src;
-    __half *dst;
-    int64_t n;
-};
-struct F16Jobs {
-    F16Job job[2];
-    int32_t n_jobs;
-    int32_t H, D;
-    int64_t tok_stride, head_stride;
-};
-
-__global__ void __launch_bounds__(256) keys_f16_kernel(F16Jobs jobs) {
-    const int cpr = jobs.D / 8;   // 16-byte chunks per row
-    for (int jb = 0; jb < jobs.n_jobs; ++jb) {
-        const F16Job J = jobs.job[jb];
-        const int64_t total = J.n * jobs.H * cpr;
-        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-             i += (int64_t)gridDim.x * blockDim.x) {
-            const int c = (int)(i % cpr);
-            const int64_t rowi = i / cpr;              // = h * n + t  (destination order)
-            const int64_t t = rowi % J.n;
-            const int h = (int)(rowi / J.n);
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(J.src + t * jobs.tok_stride +
-                                                                  (int64_t)h * jobs.head_stride) + c);
-            reinterpret_cast<uint4 *>(J.dst + rowi * jobs.D)[c] = bf16x8_to_f16(v);
-        }
-    }
-}
-
-// bf16 [n][H][D] -> fp16 V^T [H][D][np] (np = n rounded up to 8; the padding is zero), for up to
-// two tensors.  One block transposes 64 tokens x D of one head through shared memory.
-struct VtJob {
-    const __nv_bfloat16 *src;
-    __half *dst;
-    int64_t n, np;
-};
-struct VtJobs {
-    VtJob job[2];
-    int32_t H, D;
-    int64_t tok_stride, head_stride;
-};
-
-__global__ void __launch_bounds__(256) values_t16_kernel(VtJobs jobs) {
-    __shared__ __align__(16) __half tile[64][128 + 8];
-    const VtJob J = jobs.job[blockIdx.z];
-    const int h = blockIdx.y;
-    const int64_t t0 = (int64_t)blockIdx.x * 64;
-    if (t0 >= J.np) return;
-    const int D = jobs.D;
-    const int cpr = D / 8;
-    for (int i = threadIdx.x; i < 64 * cpr; i += blockDim.x) {
-        const int r = i / cpr, c = i % cpr;
-        const int64_t t = t0 + r;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (t < J.n)
-            v = bf16x8_to_f16(__ldg(reinterpret_cast<const uint4 *>(J.src + t * jobs.tok_stride +
-                                                                    (int64_t)h * jobs.head_stride) + c));
-        *reinterpret_cast<uint4 *>(&tile[r][c * 8]) = v;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < D * 8; i += blockDim.x) {
-        const int d = i / 8, c = i % 8;   // row d, tokens [t0 + 8c, t0 + 8c + 8)
-        const int64_t t = t0 + c * 8;
-        if (t >= J.np) continue;
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const __half a = tile[c * 8 + 2 * k][d], b = tile[c * 8 + 2 * k + 1][d];
-            w[k] = (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
-        }
-        *reinterpret_cast<uint4 *>(J.dst + ((int64_t)h * D + d) * J.np + t) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
-// INT8 codes of the cache as exact fp16 integers, in the layouts of the attention kernel's TMA boxes:
-//   z = 0: ring rows of the retained history in age order -> keys [H][Lh][D], V^T [H][D][lhp] (lhp =
-//          Lh rounded up to 16, zero padding), key / value scales [H][lhp];
-//   z = 1: description-head store rows [0, Lp) -> keys [H][Lp][D], V^T [H][D][lpp] (its scales are
-//          read in place).
-// One block converts 64 tokens x D of one head; values are transposed through shared memory.
-struct HistPrep {
-    const int8_t *k8, *v8, *hk8, *hv8;
-    const float *ks, *vs;
-    __half *kh, *vht, *kp, *vpt;
-    float *ksl, *vsl;
-    int64_t ring_tokens, first_tok, Lh, lhp, Lp, lpp, head_rows;
-    int32_t H, D;
-};
-
-__global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
-    __shared__ __align__(16) int8_t tile[64][128 + 16];
-    const bool heads = blockIdx.z == 1;
-    const int h = blockIdx.y;
-    const int64_t n = heads ? P.Lp : P.Lh, np = heads ? P.lpp : P.lhp;
-    const int64_t t0 = (int64_t)blockIdx.x * 64;
-    if (t0 >= np) return;
-    const int D = P.D;
-    const int cpr = D / 16;
-    const int8_t *ksrc = heads ? P.hk8 : P.k8, *vsrc = heads ? P.hv8 : P.v8;
-    __half *kdst = heads ? P.kp : P.kh;
-    auto src_row = [&](int64_t a) -> int64_t {
-        return heads ? (int64_t)h * P.head_rows + a : (int64_t)h * P.ring_tokens + (P.first_tok + a) % P.ring_tokens;
-    };
-    for (int i = threadIdx.x; i < 64 * cpr; i += blockDim.x) {
-        const int r = i / cpr, c = i % cpr;
-        const int64_t a = t0 + r;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (a < n) {
-            const int64_t sr = src_row(a);
-            v = __ldg(reinterpret_cast<const uint4 *>(vsrc + sr * D) + c);
-            uint4 lo, hi;
-            i8x16_to_f16(__ldg(reinterpret_cast<const uint4 *>(ksrc + sr * D) + c), lo, hi);
-            uint4 *kd = reinterpret_cast<uint4 *>(kdst + ((int64_t)h * n + a) * D) + 2 * c;
-            kd[0] = lo;
-            kd[1] = hi;
-        }
-        *reinterpret_cast<uint4 *>(&tile[r][c * 16]) = v;
-    }
-    if (!heads && threadIdx.x < 64) {
-        const int64_t a = t0 + threadIdx.x;
-        if (a < np) {
-            float ks = 0.0f, vs = 0.0f;
-            if (a < n) {
-                const int64_t sr = src_row(a);
-                ks = __ldg(P.ks + sr);
-                vs = __ldg(P.vs + sr);
-            }
-            P.ksl[(int64_t)h * P.lhp + a] = ks;
-            P.vsl[(int64_t)h * P.lhp + a] = vs;
-        }
-    }
-    __syncthreads();
-    __half *dst = heads ? P.vpt : P.vht;
-    for (int i = threadIdx.x; i < D * 4; i += blockDim.x) {
-        const int d = i / 4, c = i % 4;   // row d, tokens [t0 + 16c, t0 + 16c + 16)
-        const int64_t t = t0 + c * 16;
-        if (t >= np) continue;
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            w[k] = (uint32_t)(uint8_t)tile[c * 16 + 4 * k][d] | ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 1][d] << 8) |
-                   ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 2][d] << 16) |
-                   ((uint32_t)(uint8_t)tile[c * 16 + 4 * k + 3][d] << 24);
-        uint4 lo, hi;
-        i8x16_to_f16(make_uint4(w[0], w[1], w[2], w[3]), lo, hi);
-        uint4 *vd = reinterpret_cast<uint4 *>(dst + ((int64_t)h * D + d) * np + t);
-        vd[0] = lo;
-        vd[1] = hi;
-    }
-}
-
 }  // namespace nomas
 
 // ------------------------------------------------------------------------------------------------
@@ -920,10 +729,7 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
         if (Lt > 0)
             jobs.job[jobs.n_jobs++] =
                 F16Job{static_cast<const __nv_bfloat16 *>(ktxt), reinterpret_cast<__half *>(wsb + ws.kt), Lt};
-        int64_t blocks = ((Nq + Lt) * H * (D / 8) + 255) / 256;
-        if (blocks > 148 * 16) blocks = 148 * 16;
-        keys_f16_kernel<<<(unsigned)blocks, 256, 0, st>>>(jobs);
-        if ((rc = check_launch("keys_f16_kernel launch"))) return rc;
+        if ((rc = launch_keys_f16(jobs, st))) return rc;
 
         VtJobs vj{};
         vj.H = H;
@@ -933,9 +739,7 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
         vj.job[0] = VtJob{static_cast<const __nv_bfloat16 *>(vcur), reinterpret_cast<__half *>(wsb + ws.vc), Nq, nqp};
         vj.job[1] = VtJob{static_cast<const __nv_bfloat16 *>(Lt > 0 ? vtxt : vcur), reinterpret_cast<__half *>(wsb + ws.vt),
                           Lt, ltp};
-        const dim3 vgrid((unsigned)((nqp > ltp ? nqp : ltp) + 63) / 64, (unsigned)H, Lt > 0 ? 2u : 1u);
-        values_t16_kernel<<<vgrid, 256, 0, st>>>(vj);
-        if ((rc = check_launch("values_t16_kernel launch"))) return rc;
+        if ((rc = launch_values_t16(vj, Lt > 0, nqp > ltp ? nqp : ltp, st))) return rc;
     }
     const HistView hv = hist_view(c);
     if (Lh > 0 || Lp > 0) {
@@ -961,10 +765,7 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
         hp.head_rows = d.head_store_tokens;
         hp.H = H;
         hp.D = D;
-        const int64_t nmax = lhp > lpp ? lhp : lpp;
-        const dim3 hgrid((unsigned)((nmax + 63) / 64), (unsigned)H, 2u);
-        hist_prep_kernel<<<hgrid, 256, 0, st>>>(hp);
-        if ((rc = check_launch("hist_prep_kernel launch"))) return rc;
+        if ((rc = launch_hist_prep(hp, st))) return rc;
     }
 
     // ---- tensor maps (an extent of zero gets a one-row map that no tile reads)

@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "nomas_internal.h"
@@ -253,6 +254,20 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bo
 // whose rows are 128 bytes (8 rows = one 1024-byte swizzle atom).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+__device__ __forceinline__ uint32_t f16x2_of(float lo, float hi) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// 8 bf16 -> 8 fp16 (16 bytes in, 16 bytes out).
+__device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 &v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = f16x2_of(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+    return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 }  // namespace nomas

@@ -1,0 +1,52 @@
+// Pre-pass of nomas_attn_fwd (HBM-bound): operand copies in the layouts the attention kernel's TMA
+// boxes read -- fp16 keys [H][n][D], fp16 values transposed [H][D][n], and the cache's INT8 codes
+// widened to exact fp16 in the same layouts.
+#pragma once
+
+#include "common.cuh"
+
+namespace nomas {
+
+// bf16 [n][H][D] (token / head strides in elements) -> fp16 [H][n][D], for up to two tensors.
+struct F16Job {
+    const __nv_bfloat16 *src;
+    __half *dst;
+    int64_t n;
+};
+struct F16Jobs {
+    F16Job job[2];
+    int32_t n_jobs;
+    int32_t H, D;
+    int64_t tok_stride, head_stride;
+};
+
+// bf16 [n][H][D] -> fp16 V^T [H][D][np] (np = n rounded up to 8, zero padding); job[1] is used when
+// `two` is set.
+struct VtJob {
+    const __nv_bfloat16 *src;
+    __half *dst;
+    int64_t n, np;
+};
+struct VtJobs {
+    VtJob job[2];
+    int32_t H, D;
+    int64_t tok_stride, head_stride;
+};
+
+// INT8 ring rows of the retained history (age order) and description-head rows -> fp16 codes; see
+// hist_prep_kernel.
+struct HistPrep {
+    const int8_t *k8, *v8, *hk8, *hv8;
+    const float *ks, *vs;
+    __half *kh, *vht, *kp, *vpt;
+    float *ksl, *vsl;
+    int64_t ring_tokens, first_tok, Lh, lhp, Lp, lpp, head_rows;
+    int32_t H, D;
+};
+
+// Each enqueues one kernel on `st` and returns NOMAS_OK or the launch error.
+int launch_keys_f16(const F16Jobs &jobs, cudaStream_t st);
+int launch_values_t16(const VtJobs &jobs, bool two, int64_t max_np, cudaStream_t st);
+int launch_hist_prep(const HistPrep &P, cudaStream_t st);
+
+}  // namespace nomas

@@ -29,6 +29,15 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "C2"
 METRIC = "masked attention TFLOP/s (dense + 25% block-sparse step, INT8 KV history) on 1 B200"
+
+
+def step_config(cfg, world):
+    """The `config` object of the JSON line; both arms report the same one."""
+    return {"workload": "production_1280x704: 16x128, 30-frame segment (26400 queries), 18-frame INT8 "
+                        "history (15840 keys), 768 head + 8 tails x 64; step = append + dense mask + "
+                        "dense attention + sparse selection (25%) + sparse attention",
+            "seq_len": cfg.n_query, "heads": cfg.heads, "head_dim": cfg.head_dim,
+            "l2": "inputs larger than L2 (324 MB bf16 q/k/v per step)", "parallelism": f"replica x{world}"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -455,6 +464,7 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
+        from int8_kv_cache_action_b200.workloads import CONFIGS
         vals = []
         for i in range(args.warmup + args.steps):
             r = cpu_oracle_sample(seconds_budget=6.0)
@@ -464,7 +474,7 @@ def main():
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "production_1280x704 dense attention (sampled rows)"},
+                "config": step_config(CONFIGS[WORKLOAD], args.gpus),
                 "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": vals[0]["cores"], "kind": "oracle",
                                  "sample": vals[0]["sample"]},
                 "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -506,11 +516,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "production_1280x704: 16x128, 30-frame segment (26400 queries), 18-frame INT8 "
-                               "history (15840 keys), 768 head + 8 tails x 64; step = append + dense mask + "
-                               "dense attention + sparse selection (25%) + sparse attention",
-                   "seq_len": cfg.n_query, "heads": cfg.heads, "head_dim": cfg.head_dim,
-                   "l2": "inputs larger than L2 (324 MB bf16 q/k/v per step)", "parallelism": f"replica x{world}"},
+        "config": step_config(cfg, world),
         "roofline": {"bound": "tensor",
                      "kernel": "nomas_attn_fwd dense (attn_fwd_kernel<128> + its operand-copy pre-pass)",
                      "achieved": dense_tflops,

@@ -64,3 +64,27 @@ def test_traffic_is_dropped_when_the_kernel_changed(tmp_path):
     assert bench.measured_traffic(str(f)) == 123
     f.write_text(json.dumps({"attn_source_sha256_16": "0" * 16, "bytes_per_launch": 123}))
     assert bench.measured_traffic(str(f)) is None
+
+
+def test_reference_arm_line():
+    """`bench.py --impl reference` (the timed CPU oracle) prints one JSON line with the measured arm's
+    config object, a cpu_baseline describing the sample, and an end-to-end entry with no copies."""
+    import json
+    import subprocess
+    import sys
+
+    import bench
+    from int8_kv_cache_action_b200.workloads import CONFIGS
+    root = os.path.dirname(os.path.abspath(bench.__file__))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3"],
+                       cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "TFLOP/s"
+    assert d["config"] == bench.step_config(CONFIGS[bench.WORKLOAD], 1)
+    assert d["steps"] == 1 and d["warmup"] == 3 and d["higher_is_better"] is True and d["value"] > 0
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}

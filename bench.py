@@ -329,7 +329,7 @@ def run_ours(args, rank, world, local_rank):
             out_free[i].record(s_d2h)
         e1.record(s_d2h)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1) / n_e2e
+        ems, _ = aggregate_ranks(e0.elapsed_time(e1) / n_e2e, 0.0, world, reduce_max)   # slowest rank
         e2e = {"value": (flops_dense + flops_sparse) / (ems * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": n_e2e,
                "pipelined": "H2D / compute / D2H on three streams, two buffer sets"}

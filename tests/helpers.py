@@ -1,6 +1,8 @@
 """Shared test helpers: build the CUDA cache and the oracle cache from the same seeded inputs."""
 from __future__ import annotations
 
+from fractions import Fraction
+
 import numpy as np
 import torch
 
@@ -57,3 +59,24 @@ def sample_rows(cfg: Config, n_random=200, seed=7):
     rows.update(rng.integers(0, nq, n_random).tolist())
     rows.add(nq - 1)
     return np.asarray(sorted(rows), np.int64)
+
+
+def rn32(x: Fraction) -> Fraction:
+    """Round a rational below the fp32 overflow threshold to the nearest fp32 (subnormals included),
+    ties to even."""
+    if x == 0:
+        return Fraction(0)
+    neg = x < 0
+    x = -x if neg else x
+    e = x.numerator.bit_length() - x.denominator.bit_length()
+    if x < Fraction(2) ** e:
+        e -= 1
+    assert e <= 127, "overflow"
+    e = max(e, -126)                                    # the subnormal grid is 2^-149
+    m = x / Fraction(2) ** (e - 23)
+    fl = m.numerator // m.denominator
+    rem = m - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl & 1):
+        fl += 1
+    r = Fraction(fl) * Fraction(2) ** (e - 23)
+    return -r if neg else r

@@ -7,26 +7,7 @@ subnormal and non-finite a elsewhere."""
 import struct
 from fractions import Fraction
 
-
-def _rn32(x: Fraction) -> Fraction:
-    """Round a rational below the fp32 overflow threshold to the nearest fp32 (subnormals included),
-    ties to even."""
-    if x == 0:
-        return Fraction(0)
-    neg = x < 0
-    x = -x if neg else x
-    e = x.numerator.bit_length() - x.denominator.bit_length()
-    if x < Fraction(2) ** e:
-        e -= 1
-    assert e <= 127, "overflow"
-    e = max(e, -126)                                    # the subnormal grid is 2^-149
-    m = x / Fraction(2) ** (e - 23)
-    fl = m.numerator // m.denominator
-    rem = m - fl
-    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl & 1):
-        fl += 1
-    r = Fraction(fl) * Fraction(2) ** (e - 23)
-    return -r if neg else r
+from tests.helpers import rn32
 
 
 def _bf16(bits: int) -> Fraction:
@@ -38,20 +19,20 @@ def test_rounding_helper_matches_fp32_casts():
     rng = np.random.default_rng(0)
     for v in np.concatenate([rng.standard_normal(200) * 10.0 ** rng.integers(-30, 30, 200),
                              rng.standard_normal(50) * 1e-40]):                  # fp32 subnormals
-        assert _rn32(Fraction(float(v))) == Fraction(float(np.float32(v)))
+        assert rn32(Fraction(float(v))) == Fraction(float(np.float32(v)))
 
 
 def test_division_by_127_without_division_is_exact():
-    c = _rn32(Fraction(1, 127))
+    c = rn32(Fraction(1, 127))
     assert float(c) == float.fromhex("0x1.020408p-7")
     lo = (127 - 110) << 7                                # bf16 bits of 2^-110
     checked = 0
     for bits in range(lo, 0x7F80):
         a = _bf16(bits)
-        q0 = _rn32(a * c)
-        rem = _rn32(a - 127 * q0)
+        q0 = rn32(a * c)
+        rem = rn32(a - 127 * q0)
         assert rem == a - 127 * q0, "remainder not exact"
-        s = _rn32(rem * c + q0) if rem else q0
-        assert s == _rn32(a / 127) and s >= Fraction(2) ** -126, hex(bits)
+        s = rn32(rem * c + q0) if rem else q0
+        assert s == rn32(a / 127) and s >= Fraction(2) ** -126, hex(bits)
         checked += 1
     assert checked == 0x7F80 - lo

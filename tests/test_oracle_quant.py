@@ -92,3 +92,46 @@ def test_scale_is_per_row_not_per_tensor():
     q, s = quantize(x)
     assert q[0, 0] == 127 and q[1, 0] == 127
     assert s[0] != s[1]
+
+
+def _exact_quantize_row(x):
+    """The quantiser's definition in exact rational arithmetic, with each fp32 rounding done exactly:
+    s = RN32(a / 127), q_c = clamp(round_half_even(RN32(x_c / s)), -127, 127), a = 0 -> s = 0, q = 0."""
+    from fractions import Fraction
+    from tests.helpers import rn32
+    xs = [Fraction(float(v)) for v in x]
+    a = max(abs(v) for v in xs)
+    if a == 0:
+        return [0] * len(xs), Fraction(0)
+    s = rn32(a / 127)
+    return [max(-127, min(127, round(rn32(v / s)))) for v in xs], s
+
+
+def test_matches_exact_rational_definition():
+    """Random, tie-constructed, tiny (subnormal scale) and huge bf16 rows: codes and scale equal the
+    definition evaluated in exact rationals with exact fp32 roundings."""
+    rng = np.random.default_rng(11)
+    rows = [_bf16(rng.standard_normal(64) * 10.0 ** rng.uniform(-30, 30)) for _ in range(120)]
+    for k in (-20, 0, 7):                       # s = 2^k exactly: (j + 1/2) 2^k are exact ties
+        j = rng.integers(-127, 127, 64).astype(np.float32)
+        x = ((j + np.float32(0.5)) * np.float32(2.0 ** k)).astype(np.float32)
+        x[0] = np.float32(127 * 2.0 ** k)
+        rows.append(x)
+    for e in (-133, -128, -120):                # subnormal and near-subnormal absmax
+        rows.append(_bf16(rng.uniform(-1, 1, 64) * 2.0 ** e))
+    rows.append(_bf16(rng.choice([-1.0, 1.0], 64) * 3.3e38))
+    # x = absmax / 2 where x / s lies just below 63.5 but its fp32 quotient is exactly 63.5: the
+    # definition (fp32 division, then half-even) gives 64, a wider division would give 63
+    for a_bits in (0x4238, 0x3F17, 0x423B):
+        a = np.uint32(a_bits << 16).view(np.float32)
+        x = np.zeros(64, np.float32)
+        x[0], x[1], x[2] = a, a / 2, -a / 2
+        rows.append(x)
+    x = np.stack(rows).astype(np.float32)
+    assert np.array_equal(_bf16(x), x)
+    q, s = quantize(x)
+    for i in range(x.shape[0]):
+        codes, scale = _exact_quantize_row(x[i])
+        assert s[i] == float(scale), i
+        assert q[i].tolist() == codes, i
+    assert [q[-3 + k, 1] for k in range(3)] == [64, 64, 64] and [q[-3 + k, 2] for k in range(3)] == [-64, -64, -64]

@@ -17,7 +17,10 @@ of which blocks those are ("parity vs the real system: unpinned"):
         mean = sum / n_valid                      (fp32 IEEE division);
   * score = fmaf chain over channels (see csrc/oracle_score.c);
   * keep k = ceil(n * keep_frac) blocks (clamped to [1, n]), ordered by score
-    descending then candidate index ascending.
+    descending then candidate index ascending;
+  * the order is total: a NaN score (an inf or NaN input reaches the means)
+    ranks as -inf, and -0 ranks equal to +0, so every candidate has exactly
+    one rank (ties between them go to the lower index like any other tie).
 Text, description heads and in-window action tails are always kept.
 """
 from __future__ import annotations
@@ -72,6 +75,12 @@ def scores(qmean: np.ndarray, kmean: np.ndarray) -> np.ndarray:
     return out
 
 
+def rank_key(s: np.ndarray) -> np.ndarray:
+    """Score as a ranking key: NaN -> -inf (and -0 == +0, as float comparison already has it)."""
+    s = np.asarray(s, np.float64)
+    return np.where(np.isnan(s), -np.inf, s)
+
+
 def keep_count(n: int, keep_frac: float) -> int:
     if n == 0:
         return 0
@@ -104,6 +113,6 @@ def select(q: np.ndarray, hist_k8: np.ndarray, hist_ks: np.ndarray, k_cur: np.nd
         sc[h] = s
         idx = np.arange(ncand)
         for b in range(nqb):
-            order = np.lexsort((idx, -s[b].astype(np.float64)))   # primary: score desc; then index asc
+            order = np.lexsort((idx, -rank_key(s[b])))   # primary: score desc; then index asc
             sel[h, b] = order[:k]
     return sel, sc

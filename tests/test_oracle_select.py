@@ -79,3 +79,20 @@ def test_ties_pick_lower_index_and_full_keep():
 @pytest.mark.parametrize("n,f,k", [(331, 0.25, 83), (80, 0.25, 20), (1, 0.25, 1), (7, 0.25, 2), (10, 1.0, 10), (0, 0.25, 0)])
 def test_keep_count(n, f, k):
     assert sel.keep_count(n, f) == k
+
+
+def test_nan_scores_rank_as_minus_infinity():
+    # One inf query channel: its block mean is inf, so candidate scores become inf, -inf or NaN
+    # (inf * 0 in the fmaf chain).  The order is total: NaN ranks as -inf, ties by lower index.
+    q = np.ones((128, 1, 2), np.float32)
+    q[5, 0, 0] = np.inf
+    blocks = [(0.0, 5.0), (-1.0, 0.0), (1.0, 0.0), (0.0, 0.0), (-2.0, 0.0)]   # NaN, -inf, inf, NaN, -inf
+    kc = np.concatenate([np.tile(np.array(b, np.float32), (128, 1))[:, None, :] for b in blocks])
+    k8 = np.zeros((1, 0, 2), np.int8)
+    ks = np.zeros((1, 0), np.float32)
+    s_all, sc = sel.select(q, k8, ks, kc, 1.0)
+    s = sc[0, 0]
+    assert np.isnan(s[0]) and np.isnan(s[3]) and s[1] == -np.inf and s[4] == -np.inf and s[2] == np.inf
+    assert list(s_all[0, 0]) == [2, 0, 1, 3, 4]
+    s_half, _ = sel.select(q, k8, ks, kc, 0.5)
+    assert list(s_half[0, 0]) == [2, 0, 1]

@@ -3,11 +3,13 @@
 One step = one pass of the whole path on the production shape (1280x704 -> 880 tokens per latent
 frame, 30-frame segment, 16 heads x 128, 18-frame INT8 history, 768-token description head + 8 action
 tails of 64):
-  a1  nomas_kv_append   quantise-append the finished previous segment (26400 tokens, 18 frames kept)
-  a2  nomas_mask_build  dense visibility classes and tile lists
-  a4  nomas_attn_fwd    dense masked attention (steps 1-2 of a segment's denoising)
-  a3  nomas_mask_build  sparse selection (25 % of candidate video blocks)
-  a4' nomas_attn_fwd    block-sparse attention (steps 3-8)
+  a1  nomas_kv_append     quantise-append the finished previous segment (26400 tokens, 18 frames kept)
+  a2  nomas_mask_build    dense visibility classes and tile lists
+  a4  nomas_attn_prepare  operand pre-pass: current/text K,V to fp16, INT8 history codes widened to fp16
+      nomas_attn_run      dense masked attention (steps 1-2 of a segment's denoising)
+  a3  nomas_mask_build    sparse selection (25 % of candidate video blocks)
+  a4' nomas_attn_prepare + nomas_attn_run   block-sparse attention (steps 3-8)
+(nomas_attn_fwd is exactly prepare + run; they are called separately so each is timed.)
 `value` = algorithmic attention FLOPs of the step (visible / selected keys only) / step time, on the
 device, inputs resident in HBM.  Inputs (324 MB of bf16 q/k/v per step) exceed the 126 MB L2.
 
@@ -41,15 +43,21 @@ def step_config(cfg, world):
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# Kernel launches of one step: append 1; dense mask 3; dense attention 4 (key copy, transposed values,
-# history in age order, attention); sparse mask 7; sparse attention 4.
-LAUNCHES_PER_STEP = 19
-ATTN_SOURCE = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc", "attn.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_dense_production_traffic.json")
+# Kernel launches of one step: append 1; dense mask 3; prepare 3 (key copy, transposed values, history
+# widening); dense attention 1; sparse mask 5; prepare 3; sparse attention 1.
+LAUNCHES_PER_STEP = 17
+CSRC = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc")
+COMMON = os.path.join(CSRC, "common.cuh")
+TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose digest it was taken with)
+    "attn": (os.path.join(ROOT, "profiles", "attn_dense_production_traffic.json"),
+             (os.path.join(CSRC, "attn.cu"), COMMON)),
+    "append": (os.path.join(ROOT, "profiles", "append_production_traffic.json"),
+               (os.path.join(CSRC, "append.cu"), COMMON)),
+}
 
 
-def source_digest(paths=(ATTN_SOURCE, os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc", "common.cuh"))):
-    """Digest of the attention kernel's sources (the kernel file and the device helpers it includes)."""
+def source_digest(paths):
+    """Digest of a kernel's sources (its file and the device helpers it includes)."""
     import hashlib
     h = hashlib.sha256()
     for path in paths:
@@ -58,16 +66,27 @@ def source_digest(paths=(ATTN_SOURCE, os.path.join(ROOT, "int8_kv_cache_action_b
     return h.hexdigest()[:16]
 
 
-def measured_traffic(path=TRAFFIC_FILE):
-    """DRAM bytes per dense attention launch from an ncu capture, or None when the attention source
-    has changed since the counters were taken."""
+def measured_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from an ncu capture, or None when its sources have changed
+    since the counters were taken."""
+    path, sources = TRAFFIC[kernel]
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("attn_source_sha256_16") != source_digest():
+    if d.get("source_sha256_16") != source_digest(sources):
         return None
     return d.get("bytes_per_launch")
+
+
+def prepare_bytes(cfg, hist_tokens, head_tokens):
+    """Algorithmic bytes of nomas_attn_prepare: current and text K, V read as bf16 and written as fp16;
+    per history (token, head) the K and V codes read (2 D) with both scales (8 B) and written as fp16
+    (4 D) with both scales in age order (8 B); per earlier-head (token, head) the codes read (2 D),
+    checked scales (8 B) and fp16 codes written (4 D)."""
+    H, D = cfg.heads, cfg.head_dim
+    bf = (cfg.n_query + cfg.current.text_len) * H * D * 2 * (2 + 2)
+    return bf + hist_tokens * H * (6 * D + 16) + head_tokens * H * (6 * D + 8)
 
 
 def aggregate_ranks(ms_local, work_per_rank, world, reduce_max=None):
@@ -216,31 +235,34 @@ def run_ours(args, rank, world, local_rank):
     def step(ev=None, b=bufs0, stream=None):
         sh = s if stream is None else stream.cuda_stream
         rs = st if stream is None else stream
-        if ev is not None:
-            ev[0].record(rs)
+
+        def mark(i):
+            if ev is not None:
+                ev[i].record(rs)
+
+        def prepare():
+            check(N.nomas_attn_prepare(cache.handle, seg, b["kc"].data_ptr(), b["vc"].data_ptr(),
+                                       b["kt"].data_ptr(), b["vt"].data_ptr(), ts, hs, ws.data_ptr(), sh), "prepare")
+
+        mark(0)
         check(N.nomas_kv_append(cache.handle, b["pk"].data_ptr(), b["pv"].data_ptr(), b["pk"].stride(0),
                                 b["pk"].stride(1), n_frames_prev, 0, 0, 0, sh), "append")
-        if ev is not None:
-            ev[1].record(rs)
+        mark(1)
         check(N.nomas_mask_build(cache.handle, seg, 0, 0.25, 0, 0, ts, hs, mbuf_d.data_ptr(), sh), "mask dense")
-        if ev is not None:
-            ev[2].record(rs)
-        check(N.nomas_attn_fwd(cache.handle, seg, 0, 0.25, mbuf_d.data_ptr(), b["q"].data_ptr(), b["kc"].data_ptr(),
-                               b["vc"].data_ptr(), b["kt"].data_ptr(), b["vt"].data_ptr(), ts, hs, scale,
-                               b["out_d"].data_ptr(), 0, ws.data_ptr(), sh),
-              "attn dense")
-        if ev is not None:
-            ev[3].record(rs)
+        mark(2)
+        prepare()
+        mark(3)
+        check(N.nomas_attn_run(cache.handle, seg, 0, 0.25, mbuf_d.data_ptr(), b["q"].data_ptr(), ts, hs, scale,
+                               b["out_d"].data_ptr(), 0, ws.data_ptr(), sh), "attn dense")
+        mark(4)
         check(N.nomas_mask_build(cache.handle, seg, 1, 0.25, b["q"].data_ptr(), b["kc"].data_ptr(), ts, hs,
                                  mbuf_s.data_ptr(), sh), "mask sparse")
-        if ev is not None:
-            ev[4].record(rs)
-        check(N.nomas_attn_fwd(cache.handle, seg, 1, 0.25, mbuf_s.data_ptr(), b["q"].data_ptr(), b["kc"].data_ptr(),
-                               b["vc"].data_ptr(), b["kt"].data_ptr(), b["vt"].data_ptr(), ts, hs, scale,
-                               b["out_s"].data_ptr(), 0, ws.data_ptr(), sh),
-              "attn sparse")
-        if ev is not None:
-            ev[5].record(rs)
+        mark(5)
+        prepare()
+        mark(6)
+        check(N.nomas_attn_run(cache.handle, seg, 1, 0.25, mbuf_s.data_ptr(), b["q"].data_ptr(), ts, hs, scale,
+                               b["out_s"].data_ptr(), 0, ws.data_ptr(), sh), "attn sparse")
+        mark(7)
 
     for _ in range(args.warmup):
         step()
@@ -253,6 +275,7 @@ def run_ours(args, rank, world, local_rank):
     flops_sparse = 4.0 * cfg.head_dim * sparse_key_sum(mv["sel"], cfg, st_now["history_tokens"],
                                                        st_now["head_tokens"])
     append_bytes = (cfg.window_frames * cfg.tokens_per_frame) * cfg.heads * APPEND_BYTES_PER_TOKEN_HEAD(cfg.head_dim)
+    prep_bytes = prepare_bytes(cfg, st_now["history_tokens"], st_now["head_tokens"])
 
     # timed region: K steps back to back, events on the launching stream
     if world > 1:
@@ -278,11 +301,11 @@ def run_ours(args, rank, world, local_rank):
     # per-phase breakdown: a separate pass of steps issued back to back with events between the
     # phases (no host synchronisation inside the pass, so no phase includes host launch latency)
     n_ph = max(3, min(args.steps, 10))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(n_ph)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(n_ph)]
     for k in range(n_ph):
         step(evs[k])
     torch.cuda.synchronize()
-    ph = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(n_ph)) for i in range(5)]
+    ph = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(n_ph)) for i in range(7)]
 
     # end to end: every step copies its inputs from pinned host memory, runs the same C-ABI calls and
     # copies both outputs back.  Like a serving loop, the copies of one step overlap the compute of
@@ -333,8 +356,14 @@ def run_ours(args, rank, world, local_rank):
         e2e = {"value": (flops_dense + flops_sparse) / (ems * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": n_e2e,
                "pipelined": "H2D / compute / D2H on three streams, two buffer sets"}
+    ws_bytes = {"production_1280x704": int(ws.numel())}
+    del ws, mbuf_d, mbuf_s
+    big = CONFIGS["C4"]
+    c4 = KVCache.for_config(big, dev)
+    ws_bytes["full_history_7th_of_7"] = int(N.nomas_attn_workspace_bytes(c4.handle, segment_text_of(big.current)))
+    del c4
     return dict(ms=ms, phases=ph, flops_dense=flops_dense, flops_sparse=flops_sparse, append_bytes=append_bytes,
-                clocks=clk.summary(), e2e=e2e, cfg=cfg)
+                prep_bytes=prep_bytes, ws_bytes=ws_bytes, clocks=clk.summary(), e2e=e2e, cfg=cfg)
 
 
 def per_config(args):
@@ -516,30 +545,43 @@ def main():
     flops = r["flops_dense"] + r["flops_sparse"]
     _, value = aggregate_ranks(ms_step, flops, world)
     value /= 1e12
-    ph = r["phases"]
-    dense_tflops = r["flops_dense"] / (ph[2] * 1e-3) / 1e12
-    sparse_tflops = r["flops_sparse"] / (ph[4] * 1e-3) / 1e12
+    ph = r["phases"]   # append, mask dense, prepare, run dense, mask sparse, prepare, run sparse
+    dense_tflops = r["flops_dense"] / (ph[3] * 1e-3) / 1e12
+    sparse_tflops = r["flops_sparse"] / (ph[6] * 1e-3) / 1e12
+    dense_call_tflops = r["flops_dense"] / ((ph[2] + ph[3]) * 1e-3) / 1e12
+    sparse_call_tflops = r["flops_sparse"] / ((ph[5] + ph[6]) * 1e-3) / 1e12
     append_gbs = r["append_bytes"] / (ph[0] * 1e-3) / 1e9
-    peak_t = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    prep_ms = 0.5 * (ph[2] + ph[5])
+    prep_gbs = r["prep_bytes"] / (prep_ms * 1e-3) / 1e9
+    peak_sus = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     hbm = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-    traffic = measured_traffic()
+    traffic = measured_traffic("attn")
+    append_traffic = measured_traffic("append")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": step_config(cfg, world),
         "roofline": {"bound": "tensor",
-                     "kernel": "nomas_attn_fwd dense (attn_fwd_kernel<128> + its operand-copy pre-pass)",
+                     "kernel": "attn_fwd_kernel<128> (nomas_attn_run, dense)",
                      "achieved": dense_tflops,
-                     "peak": peak_t, "unit": "TFLOP/s", "frac": dense_tflops / peak_t,
-                     "peak_kind": f"bf16 dense, sustained ({pk_kind})", "frac_of_burst": dense_tflops / peak_burst,
-                     "traffic": traffic},
+                     "peak": peak_burst, "unit": "TFLOP/s", "frac": dense_tflops / peak_burst,
+                     "peak_kind": f"bf16 dense, burst ({pk_kind}): the kernel runs {ph[3]:.2f} ms at a time",
+                     "frac_of_sustained": dense_tflops / peak_sus, "traffic": traffic},
         "roofline_append": {"bound": "hbm", "kernel": "quant_append_kernel<128>", "achieved": append_gbs,
-                            "peak": hbm, "unit": "GB/s", "frac": append_gbs / hbm, "traffic": None},
-        "breakdown_ms": {"append": ph[0], "mask_dense": ph[1], "attn_dense": ph[2], "mask_sparse": ph[3],
-                         "attn_sparse": ph[4]},
+                            "peak": hbm, "unit": "GB/s", "frac": append_gbs / hbm, "traffic": append_traffic,
+                            "peak_kind": f"HBM copy ({pk_kind})"},
+        "roofline_dequant": {"bound": "hbm",
+                             "kernel": "nomas_attn_prepare (keys_f16 + values_t16 + hist_prep: INT8 history codes "
+                                       "and bf16 current/text K,V widened to fp16)",
+                             "achieved": prep_gbs, "peak": hbm, "unit": "GB/s", "frac": prep_gbs / hbm,
+                             "bytes_per_call": r["prep_bytes"], "ms_per_call": prep_ms, "traffic": None},
+        "breakdown_ms": {"append": ph[0], "mask_dense": ph[1], "prepare_dense": ph[2], "attn_dense": ph[3],
+                         "mask_sparse": ph[4], "prepare_sparse": ph[5], "attn_sparse": ph[6]},
         "attn_dense_tflops": dense_tflops, "attn_sparse_tflops": sparse_tflops,
+        "attn_dense_call_tflops": dense_call_tflops, "attn_sparse_call_tflops": sparse_call_tflops,
+        "attn_workspace_bytes": r["ws_bytes"],
         "flops_per_step": {"dense": r["flops_dense"], "sparse": r["flops_sparse"]},
         "kv_tokens_per_s_append": (cfg.window_frames * cfg.tokens_per_frame) * cfg.heads / (ph[0] * 1e-3),
         "cpu_baseline": cpu_base,

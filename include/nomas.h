@@ -54,7 +54,8 @@ typedef enum {
     NOMAS_ETIMEOUT = -4,      /* a bounded device wait ran out (device error word) */
     NOMAS_EDEVICE = -5,       /* inconsistent device data, e.g. a stale mask buffer */
     NOMAS_EUNSUPPORTED = -6,  /* head_dim or size not supported */
-    NOMAS_ESTATE = -7         /* call order or cache state does not allow the call */
+    NOMAS_ESTATE = -7,        /* call order or cache state does not allow the call */
+    NOMAS_ERANGE = -8         /* an attention operand outside the supported range (device error word) */
 } nomas_status;
 
 /* Device buffers of a cache, all caller-owned; sizes from nomas_kv_cache_bytes.
@@ -169,7 +170,10 @@ typedef struct {
 
 /* Fill `out` for the current cache state and segment text.  keep_frac in (0, 1]
  * (sparse only): keep = clamp(ceil(n_cand * keep_frac), 1, n_cand), ceil taken in
- * double precision of the float value. */
+ * double precision of the float value.  Sparse mode supports at most
+ * NOMAS_MAX_SPARSE_CANDIDATES candidate blocks (about a million history plus current tokens);
+ * more return NOMAS_EUNSUPPORTED. */
+#define NOMAS_MAX_SPARSE_CANDIDATES 8192
 int nomas_mask_layout_query(const nomas_kv_cache *cache, const nomas_segment_text *seg, int mode,
                             float keep_frac, nomas_mask_layout *out);
 
@@ -181,7 +185,8 @@ size_t nomas_mask_bytes(const nomas_kv_cache *cache, const nomas_segment_text *s
  * 单卡 4090 怎么做到的; the ranking rule is this library's own: per head and
  * query block, score = fmaf chain over channels of the fp32 mean of the block's
  * queries and the fp32 mean of the candidate's keys, history keys taken as
- * float(code) * scale, sums in ascending token order, mean = sum / n_valid).
+ * float(code) * scale, sums in ascending token order, mean = sum / n_valid; ranked by
+ * score descending then candidate index ascending, with a NaN score ranked as -inf).
  *   q, kcur   bf16 [n_frames*T][H][D] (sparse mode only; NULL allowed in dense)
  *   mask_buf  device buffer of nomas_mask_bytes bytes, 16-byte aligned
  * The result is valid for this cache state; an append in between makes
@@ -231,7 +236,14 @@ size_t nomas_attn_workspace_bytes(const nomas_kv_cache *cache, const nomas_segme
  * tensor core exactly: the key scale multiplies the fp32 score and the value scale the fp32
  * probability, which is then rounded once to fp16 (so each term p * v^ is fp16(p * scale) * code).
  * The QK^T and PV products run on the tensor cores with fp16 operands and fp32 accumulation; bf16
- * inputs convert to fp16 exactly for magnitudes in [2^-14, 65504] (the supported input range).
+ * inputs convert to fp16 exactly for magnitudes in [2^-14, 65504] (smaller magnitudes keep fp16's
+ * 2^-24 absolute resolution).
+ * Supported range, checked on the device: every q, kcur, vcur, ktxt, vtxt element finite with
+ * magnitude below 65520 (it must not round to an fp16 infinity), and every cached value scale at
+ * most 65504 / 64 = 1023.5 (a (token, head) absmax of about 1.3e5 at append time) with finite key
+ * scales.  A violation records NOMAS_ERANGE in the device error word (read by
+ * nomas_device_status); the call still completes and the outputs of the affected rows are
+ * undefined.
  *   q, kcur, vcur  bf16 [n_frames*T][H][D];  ktxt, vtxt bf16 [text_tokens][H][D]
  *                  (NULL allowed when the segment has no text); all share tok_stride / head_stride
  *   out            fp32 [n_frames*T][H][D], contiguous
@@ -242,6 +254,27 @@ int nomas_attn_fwd(const nomas_kv_cache *cache, const nomas_segment_text *seg, i
                    const void *mask_buf, const void *q, const void *kcur, const void *vcur, const void *ktxt,
                    const void *vtxt, int64_t tok_stride, int64_t head_stride, float softmax_scale, float *out,
                    float *lse, void *workspace, nomas_stream stream);
+
+/* The two halves of nomas_attn_fwd, for callers that time or schedule them separately
+ * (nomas_attn_fwd enqueues exactly nomas_attn_prepare followed by nomas_attn_run).
+ *
+ * nomas_attn_prepare: the HBM-bound pre-pass.  Writes into `workspace` the fp16 copies of kcur, vcur,
+ * ktxt, vtxt (keys [H][n][D], values transposed [H][D][n]) and the retained history's and description
+ * heads' INT8 codes widened to exact fp16 (with the history's scales in age order), plus a header that
+ * records the cache state and segment it was prepared for.  Arguments as nomas_attn_fwd.
+ *
+ * nomas_attn_run: the masked (or block-sparse) attention kernel over a prepared workspace; q is read
+ * here.  The kernel checks the workspace header (and the mask buffer's) against the cache state and
+ * segment of the call: a workspace prepared before a later append, for another segment, or never
+ * prepared records NOMAS_EDEVICE in the device error word and leaves `out` unwritten.  The workspace
+ * holds the K/V values of the last prepare: a caller that changes kcur / vcur / ktxt / vtxt must
+ * prepare again. */
+int nomas_attn_prepare(const nomas_kv_cache *cache, const nomas_segment_text *seg, const void *kcur,
+                       const void *vcur, const void *ktxt, const void *vtxt, int64_t tok_stride,
+                       int64_t head_stride, void *workspace, nomas_stream stream);
+int nomas_attn_run(const nomas_kv_cache *cache, const nomas_segment_text *seg, int mode, float keep_frac,
+                   const void *mask_buf, const void *q, int64_t tok_stride, int64_t head_stride,
+                   float softmax_scale, float *out, float *lse, void *workspace, nomas_stream stream);
 
 /* Diagnostic: retained history in age order, dequantised as fp32 code * scale.
  *   k_out, v_out  fp32 [history_tokens][H][D] */

@@ -16,18 +16,19 @@ if not os.path.exists(_LIB_PATH):
 lib = ctypes.CDLL(_LIB_PATH)
 
 NOMAS_OK, NOMAS_EINVAL, NOMAS_ECAPACITY, NOMAS_ECUDA, NOMAS_ETIMEOUT, NOMAS_EDEVICE, NOMAS_EUNSUPPORTED, \
-    NOMAS_ESTATE = 0, -1, -2, -3, -4, -5, -6, -7
+    NOMAS_ESTATE, NOMAS_ERANGE = 0, -1, -2, -3, -4, -5, -6, -7, -8
 NOMAS_BUF_K8, NOMAS_BUF_V8, NOMAS_BUF_KS, NOMAS_BUF_VS, NOMAS_BUF_HK8, NOMAS_BUF_HV8, NOMAS_BUF_HKS, \
     NOMAS_BUF_HVS, NOMAS_BUF_ERR, NOMAS_NBUF = range(10)
 NOMAS_MODE_DENSE, NOMAS_MODE_SPARSE = 0, 1
 NOMAS_MAX_TAILS = 64
 NOMAS_STATIC_POOL_FLOATS = 2 << 20
+NOMAS_MAX_SPARSE_CANDIDATES = 8192
 
 EXPORTED = ["nomas_kv_cache_bytes", "nomas_kv_cache_init", "nomas_kv_cache_destroy", "nomas_kv_cache_state",
             "nomas_kv_append", "nomas_mask_layout_query", "nomas_mask_bytes", "nomas_mask_build",
             "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string",
             "nomas_last_error", "nomas_mask_build_static", "nomas_attn_workspace_bytes",
-            "nomas_set_wait_limit_ns"]
+            "nomas_set_wait_limit_ns", "nomas_attn_prepare", "nomas_attn_run"]
 
 
 class nomas_cache_dims(ctypes.Structure):
@@ -79,6 +80,10 @@ _sigs = {
     "nomas_attn_workspace_bytes": (_sz, [_p, ctypes.POINTER(nomas_segment_text)]),
     "nomas_attn_fwd": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32, _p, _p, _p,
                                       _p, _p, _p, _i64, _i64, _f32, _p, _p, _p, _p]),
+    "nomas_attn_prepare": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), _p, _p, _p, _p, _i64, _i64,
+                                          _p, _p]),
+    "nomas_attn_run": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32, _p, _p, _i64,
+                                      _i64, _f32, _p, _p, _p, _p]),
     "nomas_kv_dequant": (ctypes.c_int, [_p, _p, _p, _p]),
     "nomas_device_status": (ctypes.c_int, [_p, _p]),
     "nomas_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -186,6 +191,17 @@ def nomas_attn_fwd(handle, seg, mode, keep_frac, mask_buf, q, kcur, vcur, ktxt, 
     return lib.nomas_attn_fwd(handle, ctypes.byref(seg), mode, keep_frac, mask_buf, q, kcur, vcur, ktxt or None,
                               vtxt or None, tok_stride, head_stride, softmax_scale, out, lse or None,
                               workspace or None, stream or None)
+
+
+def nomas_attn_prepare(handle, seg, kcur, vcur, ktxt, vtxt, tok_stride, head_stride, workspace, stream=0):
+    return lib.nomas_attn_prepare(handle, ctypes.byref(seg), kcur, vcur, ktxt or None, vtxt or None, tok_stride,
+                                  head_stride, workspace or None, stream or None)
+
+
+def nomas_attn_run(handle, seg, mode, keep_frac, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse=0,
+                   workspace=0, stream=0):
+    return lib.nomas_attn_run(handle, ctypes.byref(seg), mode, keep_frac, mask_buf, q, tok_stride, head_stride,
+                              softmax_scale, out, lse or None, workspace or None, stream or None)
 
 
 def nomas_kv_dequant(handle, k_out, v_out, stream=0):

@@ -92,6 +92,8 @@ struct AttnParams {
     const int32_t *counts;
     const int2 *txtwin;
     MaskHeader expect;
+    const WsHeader *ws_hdr;     // written by nomas_attn_prepare
+    WsHeader ws_expect;
     int32_t sparse;
     int32_t n_pairs;
     // queries and shapes
@@ -198,8 +200,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         hd->history_tokens == p.expect.history_tokens && hd->head_tokens == p.expect.head_tokens &&
                         hd->frames_appended == p.expect.frames_appended && hd->n_query == p.expect.n_query &&
                         hd->text_tokens == p.expect.text_tokens && hd->list_cap == p.expect.list_cap;
-    if (!hdr_ok) {
-        if (threadIdx.x == 0) set_device_error(p.err, NOMAS_EDEVICE, 1);
+    const WsHeader *wh = p.ws_hdr;
+    const bool ws_ok = wh->magic == p.ws_expect.magic && wh->head_dim == p.ws_expect.head_dim &&
+                       wh->frames_appended == p.ws_expect.frames_appended &&
+                       wh->head_tokens == p.ws_expect.head_tokens &&
+                       wh->history_tokens == p.ws_expect.history_tokens && wh->n_query == p.ws_expect.n_query &&
+                       wh->text_tokens == p.ws_expect.text_tokens;
+    if (!hdr_ok || !ws_ok) {
+        if (threadIdx.x == 0) set_device_error(p.err, NOMAS_EDEVICE, hdr_ok ? 2 : 1);
         return;
     }
     const int n_tiles = p.counts[list_id];
@@ -406,14 +414,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t qp[DH / 2];
             const uint4 *src = reinterpret_cast<const uint4 *>(p.q + (row_ok ? row : 0) * p.tok_stride +
                                                                (int64_t)h * p.head_stride + half * DH);
+            bool bad = false;
 #pragma unroll
             for (int i = 0; i < DH / 8; ++i) {
                 const uint4 v = row_ok ? bf16x8_to_f16(__ldg(src + i)) : make_uint4(0, 0, 0, 0);
+                bad |= f16x8_nonfinite(v);
                 qp[4 * i] = v.x;
                 qp[4 * i + 1] = v.y;
                 qp[4 * i + 2] = v.z;
                 qp[4 * i + 3] = v.w;
             }
+            if (bad) set_device_error(p.err, NOMAS_ERANGE, 33);   // q outside the fp16 range
             const uint32_t tq = tmem + lane_base + kTmQ + (uint32_t)(half * DH / 2);
             if constexpr (DH / 2 == 32) {
                 tmem_st32(tq, qp);
@@ -622,8 +633,8 @@ static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, c
 
 static int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
-// Workspace regions (256-byte aligned), sized for the largest history the cache can retain so that
-// the size does not depend on the cache state:
+// Workspace regions (256-byte aligned) after a 256-byte header, sized for the largest history the
+// cache can retain so that the size does not depend on the cache state:
 //   kc, kt   fp16 [H][n][D]       current-segment / text keys
 //   vc, vt   fp16 [H][D][np8]     current-segment / text values, transposed
 //   kh       fp16 [H][Lh][D]      retained-history key codes in age order
@@ -641,7 +652,7 @@ static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
     const int64_t lh = frames * d.tokens_per_frame, lhp = round_up(lh, 16);
     const int64_t lpp = round_up(d.head_store_tokens, 16);
     WsLayout w;
-    size_t off = 0;
+    size_t off = 256;   // WsHeader
     auto take = [&](size_t bytes) {
         const size_t o = off;
         off += (bytes + 255) / 256 * 256;
@@ -661,6 +672,18 @@ static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
     return w;
 }
 
+static WsHeader ws_header(const nomas_kv_cache *c, const nomas_mask_layout &lay) {
+    WsHeader h{};
+    h.magic = kWsMagic;
+    h.head_dim = c->d.head_dim;
+    h.frames_appended = c->frames_appended;
+    h.head_tokens = lay.head_tokens;
+    h.history_tokens = lay.history_tokens;
+    h.n_query = lay.n_query;
+    h.text_tokens = lay.text_tokens;
+    return h;
+}
+
 static uint64_t g_timeout_ns = 2000000000ull;   // 2 s per wait
 
 template <int D>
@@ -677,72 +700,78 @@ static int launch_attn(const AttnParams &p, dim3 grid, const CUtensorMap *maps, 
     return check_launch("attn_fwd_kernel launch");
 }
 
-}  // namespace nomas
-
-using namespace nomas;
-
-extern "C" uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns) {
-    const uint64_t prev = g_timeout_ns;
-    g_timeout_ns = limit_ns;
-    return prev;
+static bool strides_ok(int64_t tok_stride, int64_t head_stride) {
+    return tok_stride > 0 && head_stride > 0 && tok_stride % 8 == 0 && head_stride % 8 == 0;
 }
 
-extern "C" size_t nomas_attn_workspace_bytes(const nomas_kv_cache *c, const nomas_segment_text *seg) {
-    nomas_mask_layout lay;
-    if (compute_mask_layout(c, seg, NOMAS_MODE_DENSE, 0.25f, &lay) != NOMAS_OK) return 0;
-    return ws_layout(c, lay.n_query, lay.text_tokens).total;
-}
-
-extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text *seg, int mode, float keep_frac,
-                              const void *mask_buf, const void *q, const void *kcur, const void *vcur,
-                              const void *ktxt, const void *vtxt, int64_t tok_stride, int64_t head_stride,
-                              float softmax_scale, float *out, float *lse, void *workspace, nomas_stream stream) {
-    nomas_mask_layout lay;
-    int rc = compute_mask_layout(c, seg, mode, keep_frac, &lay);
+// Validate nomas_attn_prepare's arguments (nothing is enqueued).
+static int check_prepare(const nomas_kv_cache *c, const nomas_segment_text *seg, const void *kcur, const void *vcur,
+                         const void *ktxt, const void *vtxt, int64_t tok_stride, int64_t head_stride,
+                         const void *workspace, nomas_mask_layout &lay) {
+    const int rc = compute_mask_layout(c, seg, NOMAS_MODE_DENSE, 0.25f, &lay);
     if (rc) return rc;
-    if (!mask_buf || !aligned16(mask_buf)) return NOMAS_EINVAL;
-    if (!q || !kcur || !vcur || !out || !workspace) return NOMAS_EINVAL;
-    if (!aligned16(q) || !aligned16(kcur) || !aligned16(vcur) || !aligned16(out) || !aligned16(workspace))
+    if (!kcur || !vcur || !workspace || !aligned16(kcur) || !aligned16(vcur) || !aligned16(workspace))
         return NOMAS_EINVAL;
     if (lay.text_tokens > 0 && (!ktxt || !vtxt || !aligned16(ktxt) || !aligned16(vtxt))) return NOMAS_EINVAL;
+    if (!strides_ok(tok_stride, head_stride)) return NOMAS_EINVAL;
+    return NOMAS_OK;
+}
+
+// Validate nomas_attn_run's arguments (nothing is enqueued).
+static int check_run(const nomas_kv_cache *c, const nomas_segment_text *seg, int mode, float keep_frac,
+                     const void *mask_buf, const void *q, int64_t tok_stride, int64_t head_stride,
+                     float softmax_scale, const float *out, const float *lse, const void *workspace,
+                     nomas_mask_layout &lay) {
+    const int rc = compute_mask_layout(c, seg, mode, keep_frac, &lay);
+    if (rc) return rc;
+    if (!mask_buf || !aligned16(mask_buf)) return NOMAS_EINVAL;
+    if (!q || !out || !workspace || !aligned16(q) || !aligned16(out) || !aligned16(workspace)) return NOMAS_EINVAL;
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return NOMAS_EINVAL;
-    if (tok_stride <= 0 || head_stride <= 0 || tok_stride % 8 || head_stride % 8) return NOMAS_EINVAL;
+    if (!strides_ok(tok_stride, head_stride)) return NOMAS_EINVAL;
     if (!(softmax_scale > 0.0f) || !std::isfinite(softmax_scale)) return NOMAS_EINVAL;
+    return NOMAS_OK;
+}
+
+// The pre-pass: fp16 keys, transposed fp16 values, the history's and heads' codes as fp16, and the
+// workspace header.
+static int enqueue_prepare(const nomas_kv_cache *c, const nomas_mask_layout &lay, const void *kcur,
+                           const void *vcur, const void *ktxt, const void *vtxt, int64_t tok_stride,
+                           int64_t head_stride, void *workspace, cudaStream_t st) {
     const auto &d = c->d;
-    const int D = d.head_dim;
-    const int H = d.heads;
-    if (bind_device(c)) return NOMAS_ECUDA;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int D = d.head_dim, H = d.heads;
     const int64_t Nq = lay.n_query, Lt = lay.text_tokens, Lh = lay.history_tokens, Lp = lay.head_tokens;
     const int64_t nqp = round_up(Nq, 8), ltp = round_up(Lt, 8), lhp = round_up(Lh, 16), lpp = round_up(Lp, 16);
-
-    // ---- pre-pass: fp16 keys, transposed fp16 values, the history's and heads' codes as fp16
     const WsLayout ws = ws_layout(c, Nq, Lt);
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
-    {
-        F16Jobs jobs{};
-        jobs.H = H;
-        jobs.D = D;
-        jobs.tok_stride = tok_stride;
-        jobs.head_stride = head_stride;
-        jobs.job[jobs.n_jobs++] = F16Job{static_cast<const __nv_bfloat16 *>(kcur), reinterpret_cast<__half *>(wsb + ws.kc), Nq};
-        if (Lt > 0)
-            jobs.job[jobs.n_jobs++] =
-                F16Job{static_cast<const __nv_bfloat16 *>(ktxt), reinterpret_cast<__half *>(wsb + ws.kt), Lt};
-        if ((rc = launch_keys_f16(jobs, st))) return rc;
+    int *err = static_cast<int *>(c->buf[NOMAS_BUF_ERR]);
+    int rc;
+    F16Jobs jobs{};
+    jobs.H = H;
+    jobs.D = D;
+    jobs.tok_stride = tok_stride;
+    jobs.head_stride = head_stride;
+    jobs.err = err;
+    jobs.hdr = ws_header(c, lay);
+    jobs.hdr_dst = reinterpret_cast<WsHeader *>(wsb);
+    jobs.job[jobs.n_jobs++] = F16Job{static_cast<const __nv_bfloat16 *>(kcur), reinterpret_cast<__half *>(wsb + ws.kc), Nq};
+    if (Lt > 0)
+        jobs.job[jobs.n_jobs++] =
+            F16Job{static_cast<const __nv_bfloat16 *>(ktxt), reinterpret_cast<__half *>(wsb + ws.kt), Lt};
+    if ((rc = launch_keys_f16(jobs, st))) return rc;
 
-        VtJobs vj{};
-        vj.H = H;
-        vj.D = D;
-        vj.tok_stride = tok_stride;
-        vj.head_stride = head_stride;
-        vj.job[0] = VtJob{static_cast<const __nv_bfloat16 *>(vcur), reinterpret_cast<__half *>(wsb + ws.vc), Nq, nqp};
-        vj.job[1] = VtJob{static_cast<const __nv_bfloat16 *>(Lt > 0 ? vtxt : vcur), reinterpret_cast<__half *>(wsb + ws.vt),
-                          Lt, ltp};
-        if ((rc = launch_values_t16(vj, Lt > 0, nqp > ltp ? nqp : ltp, st))) return rc;
-    }
-    const HistView hv = hist_view(c);
+    VtJobs vj{};
+    vj.H = H;
+    vj.D = D;
+    vj.tok_stride = tok_stride;
+    vj.head_stride = head_stride;
+    vj.err = err;
+    vj.job[0] = VtJob{static_cast<const __nv_bfloat16 *>(vcur), reinterpret_cast<__half *>(wsb + ws.vc), Nq, nqp};
+    vj.job[1] = VtJob{static_cast<const __nv_bfloat16 *>(Lt > 0 ? vtxt : vcur), reinterpret_cast<__half *>(wsb + ws.vt),
+                      Lt, ltp};
+    if ((rc = launch_values_t16(vj, Lt > 0, nqp > ltp ? nqp : ltp, st))) return rc;
+
     if (Lh > 0 || Lp > 0) {
+        const HistView hv = hist_view(c);
         HistPrep hp{};
         hp.k8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_K8]);
         hp.v8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_V8]);
@@ -750,6 +779,9 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
         hp.hv8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_HV8]);
         hp.ks = static_cast<const float *>(c->buf[NOMAS_BUF_KS]);
         hp.vs = static_cast<const float *>(c->buf[NOMAS_BUF_VS]);
+        hp.hks = static_cast<const float *>(c->buf[NOMAS_BUF_HKS]);
+        hp.hvs = static_cast<const float *>(c->buf[NOMAS_BUF_HVS]);
+        hp.err = err;
         hp.kh = reinterpret_cast<__half *>(wsb + ws.kh);
         hp.vht = reinterpret_cast<__half *>(wsb + ws.vht);
         hp.kp = reinterpret_cast<__half *>(wsb + ws.kp);
@@ -767,8 +799,20 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
         hp.D = D;
         if ((rc = launch_hist_prep(hp, st))) return rc;
     }
+    return NOMAS_OK;
+}
 
-    // ---- tensor maps (an extent of zero gets a one-row map that no tile reads)
+// The attention kernel over a prepared workspace.
+static int enqueue_run(const nomas_kv_cache *c, const nomas_mask_layout &lay, int mode, const void *mask_buf,
+                       const void *q, int64_t tok_stride, int64_t head_stride, float softmax_scale, float *out,
+                       float *lse, void *workspace, cudaStream_t st) {
+    const auto &d = c->d;
+    const int D = d.head_dim, H = d.heads;
+    const int64_t Nq = lay.n_query, Lt = lay.text_tokens, Lh = lay.history_tokens, Lp = lay.head_tokens;
+    const int64_t nqp = round_up(Nq, 8), ltp = round_up(Lt, 8), lhp = round_up(Lh, 16), lpp = round_up(Lp, 16);
+    const WsLayout ws = ws_layout(c, Nq, Lt);
+    uint8_t *wsb = static_cast<uint8_t *>(workspace);
+    // tensor maps (an extent of zero gets a one-row map that no tile reads)
     CUtensorMap maps[8];
     {
         const CUtensorMapDataType F16 = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -814,6 +858,8 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     p.expect.text_tokens = lay.text_tokens;
     p.expect.list_cap = lay.list_cap;
     p.expect.keep = lay.keep;
+    p.ws_hdr = reinterpret_cast<const WsHeader *>(wsb);
+    p.ws_expect = ws_header(c, lay);
     p.sparse = mode == NOMAS_MODE_SPARSE;
     p.n_pairs = (lay.n_qblocks + 1) / 2;
     p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -829,4 +875,59 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     p.timeout_ns = g_timeout_ns;
     dim3 grid((unsigned)lay.n_qblocks, (unsigned)H);
     return D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
+}
+
+}  // namespace nomas
+
+using namespace nomas;
+
+extern "C" uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns) {
+    const uint64_t prev = g_timeout_ns;
+    g_timeout_ns = limit_ns;
+    return prev;
+}
+
+extern "C" size_t nomas_attn_workspace_bytes(const nomas_kv_cache *c, const nomas_segment_text *seg) {
+    nomas_mask_layout lay;
+    if (compute_mask_layout(c, seg, NOMAS_MODE_DENSE, 0.25f, &lay) != NOMAS_OK) return 0;
+    return ws_layout(c, lay.n_query, lay.text_tokens).total;
+}
+
+extern "C" int nomas_attn_prepare(const nomas_kv_cache *c, const nomas_segment_text *seg, const void *kcur,
+                                  const void *vcur, const void *ktxt, const void *vtxt, int64_t tok_stride,
+                                  int64_t head_stride, void *workspace, nomas_stream stream) {
+    nomas_mask_layout lay;
+    const int rc = check_prepare(c, seg, kcur, vcur, ktxt, vtxt, tok_stride, head_stride, workspace, lay);
+    if (rc) return rc;
+    if (bind_device(c)) return NOMAS_ECUDA;
+    return enqueue_prepare(c, lay, kcur, vcur, ktxt, vtxt, tok_stride, head_stride, workspace,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int nomas_attn_run(const nomas_kv_cache *c, const nomas_segment_text *seg, int mode, float keep_frac,
+                              const void *mask_buf, const void *q, int64_t tok_stride, int64_t head_stride,
+                              float softmax_scale, float *out, float *lse, void *workspace, nomas_stream stream) {
+    nomas_mask_layout lay;
+    const int rc = check_run(c, seg, mode, keep_frac, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse,
+                             workspace, lay);
+    if (rc) return rc;
+    if (bind_device(c)) return NOMAS_ECUDA;
+    return enqueue_run(c, lay, mode, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse, workspace,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text *seg, int mode, float keep_frac,
+                              const void *mask_buf, const void *q, const void *kcur, const void *vcur,
+                              const void *ktxt, const void *vtxt, int64_t tok_stride, int64_t head_stride,
+                              float softmax_scale, float *out, float *lse, void *workspace, nomas_stream stream) {
+    nomas_mask_layout lay_p, lay_r;
+    int rc = check_prepare(c, seg, kcur, vcur, ktxt, vtxt, tok_stride, head_stride, workspace, lay_p);
+    if (rc) return rc;
+    rc = check_run(c, seg, mode, keep_frac, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse, workspace,
+                   lay_r);
+    if (rc) return rc;
+    if (bind_device(c)) return NOMAS_ECUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = enqueue_prepare(c, lay_p, kcur, vcur, ktxt, vtxt, tok_stride, head_stride, workspace, st))) return rc;
+    return enqueue_run(c, lay_r, mode, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse, workspace, st);
 }

@@ -270,4 +270,18 @@ __device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 &v) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// True when any of the 8 fp16 values is inf or NaN (exponent field all ones): the bf16 source was
+// non-finite or above the fp16 range (|x| >= 65520 rounds to inf).
+__device__ __forceinline__ bool f16x8_nonfinite(const uint4 &h) {
+    const uint32_t w[4] = {h.x, h.y, h.z, h.w};
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bad |= ((w[i] & 0x7C00u) == 0x7C00u) | ((w[i] & 0x7C000000u) == 0x7C000000u);
+    return bad;
+}
+
+// Largest cached value scale the attention kernel supports: the kernel multiplies the scale by a
+// probability of at most 2^6 before rounding to fp16, so 64 * scale must stay within 65504.
+constexpr float kMaxValueScale = 65504.0f / 64.0f;
+
 }  // namespace nomas

@@ -77,6 +77,7 @@ int compute_mask_layout(const nomas_kv_cache *c, const nomas_segment_text *seg, 
     o->n_tiles = o->n_hist_tiles + o->n_head_tiles + o->n_cur_tiles + o->n_text_tiles;
     o->n_cand = o->n_hist_tiles + o->n_cur_tiles;
     if (mode == NOMAS_MODE_SPARSE) {
+        if (o->n_cand > NOMAS_MAX_SPARSE_CANDIDATES) return NOMAS_EUNSUPPORTED;
         if (!(keep_frac > 0.0f && keep_frac <= 1.0f)) return NOMAS_EINVAL;
         double k = std::ceil((double)o->n_cand * (double)keep_frac);
         int64_t kk = (int64_t)k;
@@ -212,6 +213,7 @@ extern "C" const char *nomas_status_string(int s) {
         case NOMAS_EDEVICE: return "inconsistent device data";
         case NOMAS_EUNSUPPORTED: return "unsupported size";
         case NOMAS_ESTATE: return "invalid state";
+        case NOMAS_ERANGE: return "attention operand out of range";
         default: return "unknown status";
     }
 }

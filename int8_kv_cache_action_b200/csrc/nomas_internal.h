@@ -59,6 +59,19 @@ struct MaskHeader {
     int32_t keep;
 };
 
+// Device header written at offset 0 of the attention workspace by nomas_attn_prepare; the attention
+// kernel checks it against the cache state and segment of the call.
+constexpr uint32_t kWsMagic = 0x4E4D5753u;
+struct WsHeader {
+    uint32_t magic;
+    int32_t head_dim;
+    int64_t frames_appended;
+    int64_t head_tokens;
+    int64_t history_tokens;
+    int64_t n_query;
+    int64_t text_tokens;
+};
+
 int compute_mask_layout(const nomas_kv_cache *c, const nomas_segment_text *seg, int mode, float keep_frac,
                         nomas_mask_layout *out);
 

@@ -27,6 +27,7 @@ __device__ __forceinline__ void i8x16_to_f16(const uint4 &w, uint4 &lo, uint4 &h
 // bf16 [n][H][D] (token / head strides in elements) -> fp16 [H][n][D], for up to two tensors.  One
 // block converts 64 tokens x D of one head (a contiguous 64 x D run of the destination).
 __global__ void __launch_bounds__(256) keys_f16_kernel(F16Jobs jobs) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *jobs.hdr_dst = jobs.hdr;
     const F16Job J = blockIdx.z ? jobs.job[1] : jobs.job[0];
     const int h = blockIdx.y;
     const int64_t t0 = (int64_t)blockIdx.x * 64;
@@ -36,10 +37,14 @@ __global__ void __launch_bounds__(256) keys_f16_kernel(F16Jobs jobs) {
     const uint4 *src = reinterpret_cast<const uint4 *>(J.src + t0 * jobs.tok_stride + (int64_t)h * jobs.head_stride);
     uint4 *dst = reinterpret_cast<uint4 *>(J.dst + ((int64_t)h * J.n + t0) * jobs.D);
     const int64_t srow = jobs.tok_stride / 8;   // source row stride in 16-byte chunks
+    bool bad = false;
     for (int i = threadIdx.x; i < rows * cpr; i += blockDim.x) {
         const int r = i / cpr, c = i - r * cpr;
-        dst[i] = bf16x8_to_f16(__ldg(src + r * srow + c));
+        const uint4 h = bf16x8_to_f16(__ldg(src + r * srow + c));
+        bad |= f16x8_nonfinite(h);
+        dst[i] = h;
     }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) set_device_error(jobs.err, NOMAS_ERANGE, 30);
 }
 
 // bf16 [n][H][D] -> fp16 V^T [H][D][np] (np = n rounded up to 8; the padding is zero), for up to
@@ -57,6 +62,7 @@ __global__ void __launch_bounds__(256) values_t16_kernel(VtJobs jobs) {
     const int D = jobs.D;
     const int W = D / 2;                  // words per token row
     const int cpr = D / 8;                // 16-byte chunks per token row
+    bool bad = false;
     for (int i = threadIdx.x; i < 64 * cpr; i += blockDim.x) {
         const int r = i / cpr, k = i % cpr;
         const int64_t t = t0 + r;
@@ -64,9 +70,10 @@ __global__ void __launch_bounds__(256) values_t16_kernel(VtJobs jobs) {
         if (t < J.n)
             v = bf16x8_to_f16(__ldg(reinterpret_cast<const uint4 *>(J.src + t * jobs.tok_stride +
                                                                     (int64_t)h * jobs.head_stride) + k));
+        bad |= f16x8_nonfinite(v);
         *reinterpret_cast<uint4 *>(&tile[r * W + ((4 * k) ^ ((r >> 3) << 2))]) = v;
     }
-    __syncthreads();
+    if (__syncthreads_or(bad) && threadIdx.x == 0) set_device_error(jobs.err, NOMAS_ERANGE, 31);
     for (int i = threadIdx.x; i < W * 8; i += blockDim.x) {
         const int w = (i >> 5) * 4 + (i & 3);   // word: channels 2w, 2w + 1
         const int c = (i >> 2) & 7;             // tokens [t0 + 8c, t0 + 8c + 8)
@@ -123,20 +130,26 @@ __global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
         }
         *reinterpret_cast<uint4 *>(&tile[r][c * 16]) = v;
     }
-    if (!heads && threadIdx.x < 64) {
+    // scales: the history's are copied in age order; every cached value scale must keep
+    // 64 * scale within fp16 and every key scale must be finite (checked for the heads too)
+    bool bad = false;
+    if (threadIdx.x < 64) {
         const int64_t a = t0 + threadIdx.x;
         if (a < np) {
             float ks = 0.0f, vs = 0.0f;
             if (a < n) {
                 const int64_t sr = src_row(a);
-                ks = __ldg(P.ks + sr);
-                vs = __ldg(P.vs + sr);
+                ks = __ldg((heads ? P.hks : P.ks) + sr);
+                vs = __ldg((heads ? P.hvs : P.vs) + sr);
+                bad = !(vs <= kMaxValueScale) || !(fabsf(ks) <= 3.4028235e38f);
             }
-            P.ksl[(int64_t)h * P.lhp + a] = ks;
-            P.vsl[(int64_t)h * P.lhp + a] = vs;
+            if (!heads) {
+                P.ksl[(int64_t)h * P.lhp + a] = ks;
+                P.vsl[(int64_t)h * P.lhp + a] = vs;
+            }
         }
     }
-    __syncthreads();
+    if (__syncthreads_or(bad) && threadIdx.x == 0) set_device_error(P.err, NOMAS_ERANGE, 32);
     __half *dst = heads ? P.vpt : P.vht;
     for (int i = threadIdx.x; i < D * 4; i += blockDim.x) {
         const int d = i / 4, c = i % 4;   // row d, tokens [t0 + 16c, t0 + 16c + 16)

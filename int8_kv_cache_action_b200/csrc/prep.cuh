@@ -18,6 +18,9 @@ struct F16Jobs {
     int32_t n_jobs;
     int32_t H, D;
     int64_t tok_stride, head_stride;
+    int *err;            // device error word: NOMAS_ERANGE for a value outside the fp16 range
+    WsHeader hdr;        // written to *hdr_dst by the first block
+    WsHeader *hdr_dst;
 };
 
 // bf16 [n][H][D] -> fp16 V^T [H][D][np] (np = n rounded up to 8, zero padding); job[1] is used when
@@ -31,6 +34,7 @@ struct VtJobs {
     VtJob job[2];
     int32_t H, D;
     int64_t tok_stride, head_stride;
+    int *err;            // device error word: NOMAS_ERANGE for a value outside the fp16 range
 };
 
 // INT8 ring rows of the retained history (age order) and description-head rows -> fp16 codes; see
@@ -40,8 +44,10 @@ struct HistPrep {
     const float *ks, *vs;
     __half *kh, *vht, *kp, *vpt;
     float *ksl, *vsl;
+    const float *hks, *hvs;   // description-head scales (checked only)
     int64_t ring_tokens, first_tok, Lh, lhp, Lp, lpp, head_rows;
     int32_t H, D;
+    int *err;                 // device error word: NOMAS_ERANGE for a value scale above kMaxValueScale
 };
 
 // Each enqueues one kernel on `st` and returns NOMAS_OK or the launch error.

@@ -56,14 +56,26 @@ def test_single_rank_is_local_time():
     assert ms == 4.0 and value == pytest.approx(2e12 / 4e-3)
 
 
-def test_traffic_is_dropped_when_the_kernel_changed(tmp_path):
+def test_traffic_is_dropped_when_the_kernel_changed(tmp_path, monkeypatch):
     import json
     import bench
     f = tmp_path / "t.json"
-    f.write_text(json.dumps({"attn_source_sha256_16": bench.source_digest(), "bytes_per_launch": 123}))
-    assert bench.measured_traffic(str(f)) == 123
-    f.write_text(json.dumps({"attn_source_sha256_16": "0" * 16, "bytes_per_launch": 123}))
-    assert bench.measured_traffic(str(f)) is None
+    sources = bench.TRAFFIC["append"][1]
+    monkeypatch.setitem(bench.TRAFFIC, "append", (str(f), sources))
+    f.write_text(json.dumps({"source_sha256_16": bench.source_digest(sources), "bytes_per_launch": 123}))
+    assert bench.measured_traffic("append") == 123
+    f.write_text(json.dumps({"source_sha256_16": "0" * 16, "bytes_per_launch": 123}))
+    assert bench.measured_traffic("append") is None
+
+
+def test_prepare_bytes_count():
+    import bench
+    from int8_kv_cache_action_b200.workloads import CONFIGS
+    cfg = CONFIGS["C2"]
+    # 27680 bf16 rows of K and V (26400 current + 1280 text) x 16 heads x 128: 2 B read + 2 B written each;
+    # 15840 history tokens x 16 heads: 2 x 128 codes + 2 scales read, 2 x 128 fp16 + 2 scales written
+    want = 27680 * 16 * 128 * 2 * 4 + 15840 * 16 * (2 * 128 + 8 + 4 * 128 + 8)
+    assert bench.prepare_bytes(cfg, 15840, 0) == want
 
 
 def test_reference_arm_line():

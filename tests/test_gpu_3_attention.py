@@ -137,3 +137,39 @@ def test_full_size_sampled_rows(name, mode, n_random):
     if name == "C4":
         rows = rows[::3]
     _check(cfg, mode=mode, rows=rows)
+
+
+def test_prepare_then_run_equals_fwd_and_a_stale_workspace_is_reported():
+    from int8_kv_cache_action_b200 import _nomas as N
+    from int8_kv_cache_action_b200.runtime import segment_text_of
+    cfg = small_config()
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    d = to_device(inp)
+    seg = segment_text_of(cfg.current)
+    buf, _ = gc.build_mask(seg)
+    ref, _ = gc.attention(seg, buf, d["q"], d["k_cur"], d["v_cur"], d["k_txt"], d["v_txt"])
+    q, kc, vc, kt, vt = d["q"], d["k_cur"], d["v_cur"], d["k_txt"], d["v_txt"]
+    ts, hs = q.stride(0), q.stride(1)
+    s = torch.cuda.current_stream().cuda_stream
+    scale = 1.0 / math.sqrt(cfg.head_dim)
+    ws = gc.workspace(seg)
+
+    def run(workspace, mask):
+        out = torch.full_like(ref, -7.0)
+        assert N.nomas_attn_run(gc.handle, seg, 0, 0.25, mask.data_ptr(), q.data_ptr(), ts, hs, scale,
+                                out.data_ptr(), 0, workspace.data_ptr(), s) == 0
+        torch.cuda.synchronize()
+        return out
+
+    assert N.nomas_attn_prepare(gc.handle, seg, kc.data_ptr(), vc.data_ptr(), kt.data_ptr(), vt.data_ptr(), ts, hs,
+                                ws.data_ptr(), s) == 0
+    assert torch.equal(run(ws, buf), ref) and gc.status() == 0
+    assert torch.equal(run(ws, buf), ref) and gc.status() == 0      # a prepared workspace serves again
+    never = torch.zeros_like(ws)
+    out = run(never, buf)                                           # never prepared
+    assert gc.status() == N.NOMAS_EDEVICE and bool((out == -7.0).all())
+    gc.append(kc[:cfg.tokens_per_frame], vc[:cfg.tokens_per_frame], 1)
+    fresh, _ = gc.build_mask(seg)
+    out = run(ws, fresh)                                            # prepared before the append
+    assert gc.status() == N.NOMAS_EDEVICE and bool((out == -7.0).all())

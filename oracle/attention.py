@@ -23,7 +23,7 @@ from __future__ import annotations
 import numpy as np
 
 from .quant import dequantize
-from .visibility import key_windows, TILE
+from .visibility import key_windows, text_query_mask, TILE
 
 
 def _keys_for_head(cache, h, k_cur, v_cur, k_txt, v_txt):
@@ -78,4 +78,30 @@ def attention(cache, q, k_cur, v_cur, k_txt, v_txt, text, scale, rows=None, sel=
             l = P.sum(axis=1, keepdims=True)
             out[r0:r0 + len(rr), h, :] = (P @ V) / l
             lse[h, r0:r0 + len(rr)] = (m + np.log(l))[:, 0]
+    return out, lse
+
+
+def attention_text(cache, q_txt, k_cur, v_cur, k_txt, v_txt, text, scale, rows=None):
+    """Text query rows of the current segment (visibility: visibility.text_query_mask), dense.
+
+    q_txt: float32 [Lt, H, D].  Returns (out float64 [len(rows), H, D], lse float64 [H, len(rows)]); a
+    row with no visible key has output 0 and LSE -inf.
+    """
+    lt, H, D = q_txt.shape
+    nq = k_cur.shape[0]
+    rows = np.arange(lt) if rows is None else np.asarray(rows, np.int64)
+    vis = text_query_mask(cache.history_tokens(), cache.head_used, nq, cache.T, text)[rows]
+    out = np.zeros((len(rows), H, D), np.float64)
+    lse = np.full((H, len(rows)), -np.inf, np.float64)
+    live = vis.any(axis=1)
+    sc = float(scale)
+    for h in range(H):
+        K, V = _keys_for_head(cache, h, k_cur, v_cur, k_txt, v_txt)
+        Q = q_txt[rows, h, :].astype(np.float64)
+        S = np.where(vis, (Q @ K.T) * sc, -np.inf)
+        m = np.where(live, S.max(axis=1), 0.0)[:, None]
+        P = np.exp(S - m)
+        l = P.sum(axis=1, keepdims=True)
+        out[live, h, :] = ((P @ V) / np.where(l > 0, l, 1.0))[live]
+        lse[h, live] = (m + np.log(np.where(l > 0, l, 1.0)))[live, 0]
     return out, lse

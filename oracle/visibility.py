@@ -19,6 +19,20 @@ Action tails of earlier segments are never cached, so never visible.
 Windows are half-open and counted in segment-local latent frames (reading).
 
 Each key carries a window [lo, hi); it is visible to frame t iff lo <= t < hi.
+
+Text query rows (the text stream of the double-stream joint attention, papers.ananclaw.com "这是什么"
+component list).  The pages state who may see the text, not what the text sees; the reading adopted
+keeps the action lock in both directions and the description head free of actions:
+  * a description-head row of the current segment sees the retained history, earlier heads, all
+    current-segment video and the current head, but no action tail of the segment: the head is cached
+    and visible across segments, so a head that absorbed the tails would carry the segment's actions
+    into later segments -- the cross-segment replay the action-aware mask exists to remove;
+  * a row of tail a (window [f0, f1)) sees the retained history, earlier heads and the current head,
+    the current-segment video frames t with f0 <= t < f1 (the mirror of "tail a is visible to frame t
+    iff f0 <= t < f1"), and the tails b whose window shares a frame with a's
+    (max(f0_b, f0) < min(f1_b, f1)),
+    itself included (a tail with an empty window shares no frame, so it sees no tail and no video).
+A text row with no visible key (possible only in degenerate layouts) has output 0.
 """
 from __future__ import annotations
 
@@ -92,3 +106,31 @@ def visible_counts(history_tokens, prior_head_tokens, n_query, tokens_per_frame,
 
 def visible_mask_row(lo, hi, frame):
     return (lo <= frame) & (frame < hi)
+
+
+def text_row_kinds(text):
+    """Per text row: (is_head, f0, f1); f0 = f1 = 0 for head rows."""
+    out = [(True, 0, 0)] * text.head_len
+    for t in text.tails:
+        out += [(False, t.f0, t.f1)] * t.len
+    return out
+
+
+def text_query_mask(history_tokens, prior_head_tokens, n_query, tokens_per_frame, text):
+    """bool [text_len, n_keys] over the keys in region order (history, earlier heads, current video,
+    current head, current tails): which keys each current-segment text row sees."""
+    lo, hi = key_windows(history_tokens, prior_head_tokens, n_query, text)
+    n_keys = lo.shape[0]
+    c0 = history_tokens + prior_head_tokens              # first current-video key
+    t0 = c0 + n_query + text.head_len                    # first tail key
+    video_frame = np.arange(n_query) // tokens_per_frame
+    m = np.zeros((text.text_len, n_keys), bool)
+    for i, (is_head, f0, f1) in enumerate(text_row_kinds(text)):
+        m[i, :c0] = True                                 # retained history and earlier heads
+        m[i, c0 + n_query:t0] = True                     # the current description head
+        if is_head:
+            m[i, c0:c0 + n_query] = True                 # every current video frame, no tail
+        else:
+            m[i, c0:c0 + n_query] = (f0 <= video_frame) & (video_frame < f1)
+            m[i, t0:] = np.maximum(lo[t0:], f0) < np.minimum(hi[t0:], f1)   # tails sharing a frame
+    return m

@@ -375,7 +375,8 @@ def per_config(args):
     from int8_kv_cache_action_b200.runtime import KVCache, mask_views, segment_text_of
     from int8_kv_cache_action_b200.workloads import CONFIGS, make_inputs, APPEND_BYTES_PER_TOKEN_HEAD
     dev = torch.device("cuda", 0)
-    for name in ("C0", "C1", "C2", "C3", "C4"):
+    names = args.only.split(",") if args.only else ["C0", "C1", "C2", "C3", "C4"]
+    for name in names:
         cfg = CONFIGS[name]
         inp = make_inputs(cfg)
         cache = KVCache.for_config(cfg, dev)
@@ -399,7 +400,7 @@ def per_config(args):
             cache.attention(seg, buf, q, kc, vc, kt, vt, mode=cfg.mode, keep_frac=cfg.keep_frac, workspace=ws,
                             out=out)
 
-        reps = 10 if cfg.n_query > 1000 else 50
+        reps = args.reps if args.reps else (10 if cfg.n_query > 1000 else 50)
         for _ in range(3):
             attn()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -496,6 +497,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--per-config", action="store_true",
                     help="print one line per config (attention call and append) instead of the step line")
+    ap.add_argument("--only", default="", help="with --per-config: comma-separated config names (C0..C4, C3r)")
+    ap.add_argument("--reps", type=int, default=0, help="with --per-config: timed calls per config")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

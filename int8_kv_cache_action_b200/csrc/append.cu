@@ -2,30 +2,18 @@
 // sliding-window ring (fluxbbs.com "单卡 4090 怎么做到的", first and second techniques: INT8
 // storage with float scales; 18 retained history latent frames) and the description-head store.
 //
-// HBM-bound: per (token, head) 2*D bf16 read, 2*D int8 + 2 fp32 written.  One group of D/16 lanes
-// handles one (token, head): each lane holds 16 channels of K and 16 of V (two 16-byte loads each),
-// the absmax is reduced with xor-shuffles inside the group, and each lane stores 16 codes.
+// HBM-bound: per (token, head) 2*D bf16 read, 2*D int8 + 2 fp32 written.  A persistent kernel: in
+// every CTA a producer warp keeps TMA copies of (one head x TC tokens) chunks of K and V in flight
+// through a four-stage shared-memory ring while eight consumer warps quantise the chunks already
+// landed, so loads overlap the arithmetic.  One group of D/16 lanes handles one (token, head): each
+// lane holds 16 channels of K and 16 of V, the absmax is reduced with xor-shuffles inside the group,
+// and each lane stores 16 codes.  The ring rows of the video frames and the description-head rows
+// are two jobs of the same launch.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace nomas {
-
-struct AppendArgs {
-    const __nv_bfloat16 *k;   // first token to write
-    const __nv_bfloat16 *v;
-    int64_t tok_stride, head_stride;
-    int64_t n_tok;            // tokens to write
-    int32_t heads;
-    int32_t tokens_per_frame;
-    int32_t capacity_frames;
-    int32_t first_slot;       // ring slot of the first token's frame (video mode)
-    int32_t head_mode;        // 1: destination rows dst_row0 + t (head store)
-    int64_t dst_row0;
-    int64_t rows_per_head;    // destination rows per head
-    int8_t *k8;
-    int8_t *v8;
-    float *ks;
-    float *vs;
-};
 
 template <int LPV>
 __device__ __forceinline__ float group_max(float a) {
@@ -118,71 +106,141 @@ __device__ __forceinline__ uint4 quant16(const float (&x)[16], float &s_out) {
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Work unit of a warp: one head of a block of kTokBlock consecutive tokens, one token per group of
-// D/16 lanes (16 channels per lane).  The warp issues all its 16-byte loads before quantising and
-// writes kTokBlock consecutive destination rows and scales of that head.  Index arithmetic is one
-// 32-bit division per unit; destination rows advance incrementally across frame boundaries.  At most
-// 64 registers, so four 256-thread blocks share an SM.
 template <int D>
-constexpr int kTokBlock = 32 / (D / 16);    // one token per group of D/16 lanes
+constexpr int kTokBlock = 32 / (D / 16);    // tokens per warp: one token per group of D/16 lanes
+
+constexpr int kAppendConsumers = 8;         // consumer warps; warp 8 is the producer
+constexpr int kAppendThreads = 32 * (kAppendConsumers + 1);
+constexpr int kAppendStages = 4;
 
 template <int D>
-__global__ void __launch_bounds__(256, 4) quant_append_kernel(AppendArgs a) {
+struct AppendCfg {
+    static constexpr int TC = kAppendConsumers * kTokBlock<D>;   // tokens per chunk (32 or 64)
+    static constexpr int TILE = TC * D * 2;                      // bytes of one K (or V) tile: 8 KB
+    static constexpr int STAGE = 2 * TILE;
+    static constexpr int OFF_BAR = kAppendStages * STAGE;
+    static constexpr int SMEM = OFF_BAR + 2 * kAppendStages * 8 + 1024;   // + slack for 1024-byte alignment
+};
+
+// One destination of the append: the newest frames into the ring (video) or the head store.
+struct AppendJob {
+    int64_t n_tok;            // tokens
+    int64_t n_chunks;         // ceil(n_tok / TC) * heads
+    int32_t head_mode;        // 0: ring rows slot(frame) * T + r; 1: rows dst_row0 + t
+    int32_t first_slot;       // ring slot of the job's first frame (video)
+    int32_t tok_outer;        // source maps are (D, heads, tokens) when set, else (D, tokens, heads)
+    int32_t _pad;
+    int64_t dst_row0;
+    int64_t rows_per_head;    // destination rows per head
+    int8_t *k8, *v8;
+    float *ks, *vs;
+};
+
+struct AppendParams {
+    AppendJob job[2];
+    int32_t heads, tokens_per_frame, capacity_frames;
+    int *err;
+    uint64_t timeout_ns;
+};
+
+// Chunk c of the launch: job, head and token block (token blocks outer, heads inner).
+__device__ __forceinline__ void chunk_of(const AppendParams &a, int64_t c, int &job, int &h, int64_t &tb) {
+    job = c < a.job[0].n_chunks ? 0 : 1;
+    if (job) c -= a.job[0].n_chunks;
+    tb = c / a.heads;
+    h = (int)(c - tb * a.heads);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAppendThreads, 3)
+    quant_append_kernel(const __grid_constant__ CUtensorMap tk0, const __grid_constant__ CUtensorMap tv0,
+                        const __grid_constant__ CUtensorMap tk1, const __grid_constant__ CUtensorMap tv1,
+                        const AppendParams a) {
+    using C = AppendCfg<D>;
     constexpr int LPV = D / 16;             // lanes per (token, head) vector
-    constexpr int GPW = 32 / LPV;           // groups per warp
-    constexpr int IPG = kTokBlock<D> / GPW; // tokens per group and unit
-    static_assert(IPG >= 1 && IPG * GPW == kTokBlock<D>, "token block split");
-    const int lane = threadIdx.x & 31;
+    constexpr int TB = kTokBlock<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *sm = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR), *empty = full + kAppendStages;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kAppendStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kAppendConsumers);
+        }
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    Watchdog wd{a.err, &abort_flag, a.timeout_ns, 7};
+    const int64_t total = a.job[0].n_chunks + a.job[1].n_chunks;
+
+    if (warp == kAppendConsumers) {
+        // ---------------------------------------------------------------- producer (one thread)
+        if (lane == 0) {
+            uint32_t pend = 0, wpar = 0;    // per stage: a copy was issued, parity of the phase it completes
+            int i = 0;
+            for (int64_t c = blockIdx.x; c < total; c += gridDim.x, ++i) {
+                const int st = i % kAppendStages;
+                if (!mbar_wait(&empty[st], ((i / kAppendStages) & 1) ^ 1, wd, 1)) break;
+                int job, h;
+                int64_t tb;
+                chunk_of(a, c, job, h, tb);
+                uint8_t *dk = sm + st * C::STAGE;
+                const int y = a.job[job].tok_outer ? h : (int)(tb * C::TC);
+                const int z = a.job[job].tok_outer ? (int)(tb * C::TC) : h;
+                mbar_arrive_expect_tx(&full[st], C::STAGE);
+                tma_load_3d(dk, job ? &tk1 : &tk0, &full[st], 0, y, z);
+                tma_load_3d(dk + C::TILE, job ? &tv1 : &tv0, &full[st], 0, y, z);
+                pend |= 1u << st;
+                wpar = (wpar & ~(1u << st)) | ((uint32_t)((i / kAppendStages) & 1) << st);
+            }
+            // the copies must land before the CTA's shared memory is released (a no-op unless aborting)
+            for (int st = 0; st < kAppendStages; ++st)
+                if ((pend >> st) & 1u) mbar_drain(&full[st], (wpar >> st) & 1u, 100000000ull);
+        }
+        return;
+    }
+    // -------------------------------------------------------------------- consumers
     const int sub = lane % LPV;
     const int grp = lane / LPV;
-    const int n_tok = (int)a.n_tok;
-    const int T = a.tokens_per_frame, C = a.capacity_frames;
-    const int n_units = (n_tok + kTokBlock<D> - 1) / kTokBlock<D> * a.heads;
-    const int warp0 = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
-    const int nwarps = (int)(((int64_t)gridDim.x * blockDim.x) >> 5);
-    for (int unit = warp0; unit < n_units; unit += nwarps) {
-        const int tb = unit / a.heads;
-        const int h = unit - tb * a.heads;
-        const int t0 = tb * kTokBlock<D> + grp * IPG;
-        uint4 rk[IPG][2], rv[IPG][2];
-#pragma unroll
-        for (int i = 0; i < IPG; ++i) {
-            const int t = t0 + i < n_tok ? t0 + i : 0;   // rows past the end read token 0, dropped below
-            const int64_t src = (int64_t)t * a.tok_stride + (int64_t)h * a.head_stride + sub * 16;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                rk[i][c] = __ldg(reinterpret_cast<const uint4 *>(a.k + src) + c);
-                rv[i][c] = __ldg(reinterpret_cast<const uint4 *>(a.v + src) + c);
+    const int T = a.tokens_per_frame, Cf = a.capacity_frames;
+    int i = 0;
+    for (int64_t c = blockIdx.x; c < total; c += gridDim.x, ++i) {
+        const int st = i % kAppendStages;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (i / kAppendStages) & 1, wd, 2))) break;
+        int job, h;
+        int64_t tb;
+        chunk_of(a, c, job, h, tb);
+        const AppendJob &J = a.job[job];
+        const int row_in_chunk = warp * TB + grp;
+        const int64_t t = tb * C::TC + row_in_chunk;   // token within the job
+        const uint4 *sk = reinterpret_cast<const uint4 *>(sm + st * C::STAGE + row_in_chunk * D * 2 + sub * 32);
+        const uint4 *sv = reinterpret_cast<const uint4 *>(sm + st * C::STAGE + C::TILE + row_in_chunk * D * 2 + sub * 32);
+        float x[16];
+        float skale, svale;
+        unpack16(sk[0], sk[1], x);
+        const uint4 qk = quant16<LPV>(x, skale);
+        unpack16(sv[0], sv[1], x);
+        const uint4 qv = quant16<LPV>(x, svale);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);    // this warp's reads of the stage are done
+        if (t < J.n_tok) {
+            int64_t row;
+            if (J.head_mode) {
+                row = J.dst_row0 + t;
+            } else {
+                const int f = (int)(t / T);
+                row = (int64_t)((J.first_slot + f) % Cf) * T + (t - (int64_t)f * T);
             }
-        }
-        // destination row of t0: ring slot of its frame (video) or the head store's next row
-        int r = 0, slot = 0;
-        if (!a.head_mode) {
-            const int f = t0 / T;
-            r = t0 - f * T;
-            slot = (a.first_slot + f) % C;
-        }
-#pragma unroll
-        for (int i = 0; i < IPG; ++i) {
-            float x[16];
-            float sk, sv;
-            unpack16(rk[i][0], rk[i][1], x);
-            const uint4 qk = quant16<LPV>(x, sk);
-            unpack16(rv[i][0], rv[i][1], x);
-            const uint4 qv = quant16<LPV>(x, sv);
-            const int64_t row = a.head_mode ? a.dst_row0 + t0 + i : (int64_t)slot * T + r;
-            const int64_t di = (int64_t)h * a.rows_per_head + row;
-            if (t0 + i < n_tok) {
-                *reinterpret_cast<uint4 *>(a.k8 + di * D + sub * 16) = qk;
-                *reinterpret_cast<uint4 *>(a.v8 + di * D + sub * 16) = qv;
-                if (sub == 0) {
-                    a.ks[di] = sk;
-                    a.vs[di] = sv;
-                }
-            }
-            if (++r == T) {   // next token starts the next frame
-                r = 0;
-                slot = slot + 1 == C ? 0 : slot + 1;
+            const int64_t di = (int64_t)h * J.rows_per_head + row;
+            *reinterpret_cast<uint4 *>(J.k8 + di * D + sub * 16) = qk;
+            *reinterpret_cast<uint4 *>(J.v8 + di * D + sub * 16) = qv;
+            if (sub == 0) {
+                J.ks[di] = skale;
+                J.vs[di] = svale;
             }
         }
     }
@@ -221,16 +279,34 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
     }
 }
 
-static int launch_append(const AppendArgs &a, int D, cudaStream_t st) {
-    if (a.n_tok <= 0) return NOMAS_OK;
-    if (a.n_tok >= (int64_t)1 << 30) return NOMAS_EINVAL;   // 32-bit token indices
-    const int64_t tbk = D == 128 ? kTokBlock<128> : kTokBlock<64>;
-    const int64_t units = (a.n_tok + tbk - 1) / tbk * a.heads;   // one warp each
-    if (units >= (int64_t)1 << 31) return NOMAS_EINVAL;
-    int64_t blocks = (units * 32 + 255) / 256;
-    if (blocks > 148 * 32) blocks = 148 * 32;
-    if (D == 128) quant_append_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(a);
-    else quant_append_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(a);
+// Tensor map over a job's bf16 K (or V): channels innermost, then heads and tokens in order of
+// increasing stride (tokens outermost for [tokens][heads][D] inputs).  The box is D channels of one
+// head and TC tokens, which lands in shared memory as [TC][D] either way.
+static bool source_map(CUtensorMap *m, const void *base, int64_t n_tok, int heads, int D, int64_t tok_stride,
+                       int64_t head_stride, bool tok_outer) {
+    const int tc = D == 128 ? AppendCfg<128>::TC : AppendCfg<64>::TC;
+    const cuuint64_t nt = (cuuint64_t)(n_tok > 0 ? n_tok : 1);
+    const cuuint64_t dims[3] = {(cuuint64_t)D, tok_outer ? (cuuint64_t)heads : nt, tok_outer ? nt : (cuuint64_t)heads};
+    const cuuint64_t strides[2] = {(cuuint64_t)(tok_outer ? head_stride : tok_stride) * 2,
+                                   (cuuint64_t)(tok_outer ? tok_stride : head_stride) * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)D, tok_outer ? 1u : (cuuint32_t)tc, tok_outer ? (cuuint32_t)tc : 1u};
+    return make_tensor_map_3d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, dims, strides, box,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <int D>
+static int launch_append(const CUtensorMap *maps, const AppendParams &a, cudaStream_t st) {
+    using C = AppendCfg<D>;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    std::call_once(once, [] {
+        attr = cudaFuncSetAttribute(quant_append_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    });
+    if (attr != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(append smem)", (int)attr, cudaGetErrorString(attr));
+    const int64_t total = a.job[0].n_chunks + a.job[1].n_chunks;
+    int64_t blocks = (int64_t)sm_count() * 3;
+    if (blocks > total) blocks = total;
+    quant_append_kernel<D><<<(unsigned)blocks, kAppendThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], a);
     return check_launch("quant_append_kernel launch");
 }
 
@@ -252,49 +328,66 @@ extern "C" int nomas_kv_append(nomas_kv_cache *c, const void *k, const void *v, 
     if (c->head_used + head_len > d.head_store_tokens) return NOMAS_ECAPACITY;
     if (d.window_frames == 0 && c->frames_appended + n_frames > d.capacity_frames) return NOMAS_ECAPACITY;
 
-    if (bind_device(c)) return NOMAS_ECUDA;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t T = d.tokens_per_frame;
     const int32_t keep = d.window_frames > 0 ? (n_frames < d.window_frames ? n_frames : d.window_frames) : n_frames;
     const int32_t f0 = n_frames - keep;
     const int64_t g0 = c->frames_appended + f0;
+    const int64_t tc = d.head_dim == 128 ? AppendCfg<128>::TC : AppendCfg<64>::TC;
+    if ((int64_t)keep * T >= ((int64_t)1 << 31) || head_len >= ((int64_t)1 << 31)) return NOMAS_EINVAL;
 
-    AppendArgs a{};
-    a.tok_stride = tok_stride;
-    a.head_stride = head_stride;
+    // both jobs are validated and their maps encoded before the one launch, so a failing call enqueues
+    // nothing and leaves the cache as it was
+    if (bind_device(c)) return NOMAS_ECUDA;
+    AppendParams a{};
     a.heads = d.heads;
     a.tokens_per_frame = d.tokens_per_frame;
     a.capacity_frames = d.capacity_frames;
-    int rc = NOMAS_OK;
+    a.err = static_cast<int *>(c->buf[NOMAS_BUF_ERR]);
+    a.timeout_ns = wait_limit_ns();
+    CUtensorMap maps[4];
+    const void *kv_src[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
+    AppendJob &jv = a.job[0];
+    jv.n_tok = (int64_t)keep * T;
+    jv.n_chunks = (jv.n_tok + tc - 1) / tc * d.heads;
+    jv.head_mode = 0;
+    jv.first_slot = (int32_t)(g0 % d.capacity_frames);
+    jv.rows_per_head = (int64_t)d.capacity_frames * T;
+    jv.k8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_K8]);
+    jv.v8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_V8]);
+    jv.ks = static_cast<float *>(c->buf[NOMAS_BUF_KS]);
+    jv.vs = static_cast<float *>(c->buf[NOMAS_BUF_VS]);
     if (keep > 0) {
-        a.k = static_cast<const __nv_bfloat16 *>(k) + (int64_t)f0 * T * tok_stride;
-        a.v = static_cast<const __nv_bfloat16 *>(v) + (int64_t)f0 * T * tok_stride;
-        a.n_tok = (int64_t)keep * T;
-        a.first_slot = (int32_t)(g0 % d.capacity_frames);
-        a.head_mode = 0;
-        a.rows_per_head = (int64_t)d.capacity_frames * T;
-        a.k8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_K8]);
-        a.v8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_V8]);
-        a.ks = static_cast<float *>(c->buf[NOMAS_BUF_KS]);
-        a.vs = static_cast<float *>(c->buf[NOMAS_BUF_VS]);
-        rc = launch_append(a, d.head_dim, st);
-        if (rc) return rc;
+        kv_src[0][0] = static_cast<const __nv_bfloat16 *>(k) + (int64_t)f0 * T * tok_stride;
+        kv_src[0][1] = static_cast<const __nv_bfloat16 *>(v) + (int64_t)f0 * T * tok_stride;
     }
+    AppendJob &jh = a.job[1];
+    jh.n_tok = head_len;
+    jh.n_chunks = (jh.n_tok + tc - 1) / tc * d.heads;
+    jh.head_mode = 1;
+    jh.dst_row0 = c->head_used;
+    jh.rows_per_head = d.head_store_tokens;
+    jh.k8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_HK8]);
+    jh.v8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_HV8]);
+    jh.ks = static_cast<float *>(c->buf[NOMAS_BUF_HKS]);
+    jh.vs = static_cast<float *>(c->buf[NOMAS_BUF_HVS]);
     if (head_len > 0) {
-        a.k = static_cast<const __nv_bfloat16 *>(head_k);
-        a.v = static_cast<const __nv_bfloat16 *>(head_v);
-        a.n_tok = head_len;
-        a.first_slot = 0;
-        a.head_mode = 1;
-        a.dst_row0 = c->head_used;
-        a.rows_per_head = d.head_store_tokens;
-        a.k8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_HK8]);
-        a.v8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_HV8]);
-        a.ks = static_cast<float *>(c->buf[NOMAS_BUF_HKS]);
-        a.vs = static_cast<float *>(c->buf[NOMAS_BUF_HVS]);
-        rc = launch_append(a, d.head_dim, st);
-        if (rc) return rc;
+        kv_src[1][0] = head_k;
+        kv_src[1][1] = head_v;
     }
+    const bool tok_outer = tok_stride >= head_stride;
+    for (int j = 0; j < 2; ++j) {
+        a.job[j].tok_outer = tok_outer ? 1 : 0;
+        for (int kv = 0; kv < 2; ++kv) {
+            // a job without tokens gets a one-token map over its sibling's memory that no chunk reads
+            const void *base = kv_src[j][kv] ? kv_src[j][kv] : kv_src[j ^ 1][kv];
+            if (!source_map(&maps[2 * j + kv], base, a.job[j].n_tok, d.heads, d.head_dim, tok_stride, head_stride,
+                            tok_outer))
+                return NOMAS_ECUDA;
+        }
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int rc = d.head_dim == 128 ? launch_append<128>(maps, a, st) : launch_append<64>(maps, a, st);
+    if (rc) return rc;
     c->frames_appended += n_frames;
     c->head_used += head_len;
     c->segments += 1;

@@ -2,20 +2,21 @@
 // the visibility; "单卡 4090 怎么做到的" for INT8 storage and the sparse mode).
 //
 // One CTA = one head x one 128-row query block.  Roles (16 warps, one CTA per SM):
-//   warps 0-3   softmax over key columns 0-63 of every S tile (TMEM lanes 0-127, one thread per row)
-//   warps 4-7   softmax over key columns 64-127; the two halves of a row swap their maxima through
-//               shared memory, so both apply the same offset
-//   warps 8-11  column info: per-column key scale, value scale and visibility window of every
-//               tile, one tile ahead, in a four-deep shared-memory ring
-//   warp 12     tcgen05.mma issuer (one thread) and TMEM owner
-//   warp 13     TMA producer (one thread); warps 14-15 idle
-// The register file is split per SM sub-partition (one warp of each warpgroup on each), so the
-// kernel launches at 128 registers per thread and moves them with setmaxnreg: softmax 168 each,
-// column info 112, MMA / producer warpgroup 64 -- 2*168 + 112 + 64 = 512 = 4 x 128.
+//   warps 0-3   softmax of the even-numbered KV tiles of the CTA's list (TMEM lanes 0-127, one thread
+//               per query row over all 128 key columns)
+//   warps 4-7   softmax of the odd-numbered tiles.  The two warpgroups share O and one running
+//               offset per row: each passes the offset it settled on for its tile to the other
+//               through shared memory (a chain in tile order), so while one warpgroup computes its
+//               exponentials the other loads, scales and reduces the next tile
+//   warp 8      tcgen05.mma issuer (one thread) and TMEM owner
+//   warp 9      TMA producer (one thread)
+//   warps 10-11 column info: per-column key scale, value scale and visibility window of every
+//               tile (two columns per thread), one tile ahead, in a four-deep shared-memory ring
+// 384 threads at 168 registers each: a softmax thread holds a whole 128-column score row.
 //
-// TMEM (512 columns): Q (fp16 pairs) at [0, D/2), S double buffer at [128, 256) and [256, 384),
-// O at [384, 384 + D).  P (fp16) overwrites the first 32 columns of each 64-column half of its S
-// buffer, so each softmax half writes only columns it has already read.
+// TMEM (512 columns): Q (fp16 pairs) at [0, D/2), S double buffer at [128, 256) and [256, 384)
+// (tile u uses buffer u % 2, i.e. its softmax warpgroup's), O at [384, 384 + D).  P (fp16)
+// overwrites the first 32 columns of each 64-column half of its S buffer.
 //
 // Both products are TS MMAs (A from TMEM) with a K-major B in 128-byte-swizzled shared memory:
 //   S_b  = Q K_j^T     B = K_j    [128 keys][D]
@@ -51,9 +52,8 @@
 
 namespace nomas {
 
-constexpr int kAttnThreads = 512;
-constexpr int kRegSoftmax = 168, kRegLoader = 112, kRegMma = 64;
-static_assert(2 * kRegSoftmax + kRegLoader + kRegMma == 4 * 128, "register split must equal the launch total");
+constexpr int kAttnThreads = 384;
+constexpr int kWarpMma = 8, kWarpTma = 9, kWarpCi = 10;   // column info: warps 10 and 11
 constexpr int kNCI = 4;                     // column-info ring depth
 constexpr float kRescaleThreshold = 6.0f;   // log2 units: P <= 64
 constexpr uint32_t kTmQ = 0, kTmS = 128, kTmO = 384;
@@ -71,11 +71,12 @@ struct AttnCfg {
     static constexpr int OFF_CS = OFF_V + NV * SLOT;       // float [kNCI][128] key scale x log2 e
     static constexpr int OFF_CV = OFF_CS + kNCI * 512;     // float [kNCI][128] value scale
     static constexpr int OFF_CW = OFF_CV + kNCI * 512;     // int2  [kNCI][128] key frame windows
-    static constexpr int OFF_XM = OFF_CW + kNCI * 1024;    // float [2 buffers][2 halves][128] maxima
-    static constexpr int OFF_XL = OFF_XM + 2048;           // float [2 halves][128] row sums
+    static constexpr int OFF_DEC = OFF_CW + kNCI * 1024;   // float [128] running offset after the last tile
+    static constexpr int OFF_XM = OFF_DEC + 512;           // float [2 warpgroups][128] final offsets
+    static constexpr int OFF_XL = OFF_XM + 1024;           // float [2 warpgroups][128] row sums
     static constexpr int OFF_BAR = OFF_XL + 1024;
     // q_ready; k_full, k_empty [NK]; v_full, v_empty [NV]; ci_full, ci_empty [kNCI];
-    // s_full, p_full, xm_bar [2]; pv_done; o_final; xl_bar
+    // s_full, p_full, dec_full [2]; pv_done; o_final; xl_bar
     static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 * kNCI + 6 + 3;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
@@ -118,15 +119,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
-}
-
-template <int N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ bool is_cached(int kind) { return kind == kKindHist || kind == kKindPriorHead; }
@@ -172,6 +164,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float *sCS = reinterpret_cast<float *>(sm + C::OFF_CS);
     float *sCV = reinterpret_cast<float *>(sm + C::OFF_CV);
     int2 *sCW = reinterpret_cast<int2 *>(sm + C::OFF_CW);
+    float *sDec = reinterpret_cast<float *>(sm + C::OFF_DEC);
     float *sXM = reinterpret_cast<float *>(sm + C::OFF_XM);
     float *sXL = reinterpret_cast<float *>(sm + C::OFF_XL);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
@@ -179,8 +172,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint64_t *k_full = bars + 1, *k_empty = k_full + C::NK;
     uint64_t *v_full = k_empty + C::NK, *v_empty = v_full + C::NV;
     uint64_t *ci_full = v_empty + C::NV, *ci_empty = ci_full + kNCI;
-    uint64_t *s_full = ci_empty + kNCI, *p_full = s_full + 2, *xm_bar = p_full + 2;
-    uint64_t *pv_done = xm_bar + 2, *o_final = pv_done + 1, *xl_bar = o_final + 1;
+    uint64_t *s_full = ci_empty + kNCI, *p_full = s_full + 2, *dec_full = p_full + 2;
+    uint64_t *pv_done = dec_full + 2, *o_final = pv_done + 1, *xl_bar = o_final + 1;
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
 
@@ -223,13 +216,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&v_empty[i], 1);
         }
         for (int i = 0; i < kNCI; ++i) {
-            mbar_init(&ci_full[i], 4);
-            mbar_init(&ci_empty[i], 8);
+            mbar_init(&ci_full[i], 2);      // the 2 column-info warps
+            mbar_init(&ci_empty[i], 4);     // the 4 warps of the tile's softmax warpgroup
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 8);
-            mbar_init(&xm_bar[b], 8);
+            mbar_init(&p_full[b], 4);
+            mbar_init(&dec_full[b], 4);
         }
         mbar_init(pv_done, 1);
         mbar_init(o_final, 1);
@@ -237,7 +230,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         misc[1] = 0;
         fence_mbar_init();
     }
-    if (warp == 12) {
+    if (warp == kWarpMma) {
         tmem_alloc(&misc[0], 512);
         tmem_relinquish();
     }
@@ -249,32 +242,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     Watchdog wd{p.err, abort_flag, p.timeout_ns, 0};
     const int64_t qrow0 = (int64_t)qb * kTile;
 
-    if (warp >= 8 && warp < 12) {
-        // ------------------------------------------------------------------ column-info warpgroup
-        // Thread t writes column t of every tile's entry in the ring; each warp arrives on ci_full
-        // for its 32 columns.
-        setmaxnreg_dec<kRegLoader>();
+    if (warp >= kWarpCi) {
+        // ------------------------------------------------------------------ column-info warps
+        // Thread t writes columns t and t + 64 of every tile's entry in the ring; each warp arrives on
+        // ci_full once its columns are written.
         wd.where = 3;
-        const int t = threadIdx.x - 256;   // 0..127
+        const int t = threadIdx.x - 32 * kWarpCi;   // 0..63
         struct ColInfo {
             float ks, vs;   // raw key / value scale (cached tiles), 1 / 0 otherwise
             int2 w;
         };
         // Column info of a tile (key scale, value scale, frame window), loaded one tile ahead of its
         // use: only loads happen here, so nothing waits for them until the next tile consumes them.
-        auto col_info = [&](const int4 &e) -> ColInfo {
+        auto col_info = [&](const int4 &e, int col) -> ColInfo {
             ColInfo ci{0.0f, 0.0f, make_int2(kAlwaysHi, 0)};
             const int kind = e.x & 3;
             const int64_t start = e.y;
-            if (t < e.z) {
+            if (col < e.z) {
                 if (kind == kKindText) {
-                    ci.w = p.txtwin[start + t];
+                    ci.w = p.txtwin[start + col];
                 } else {
                     ci.w = make_int2(0, kAlwaysHi);
                 }
                 if (is_cached(kind)) {
                     const bool hist = kind == kKindHist;
-                    const int64_t i = (int64_t)h * (hist ? p.hist_stride : p.head_rows) + start + t;
+                    const int64_t i = (int64_t)h * (hist ? p.hist_stride : p.head_rows) + start + col;
                     ci.ks = __ldg((hist ? p.ksl : p.hks) + i);
                     ci.vs = __ldg((hist ? p.vsl : p.hvs) + i);
                 } else {
@@ -287,24 +279,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         int u = 0;                          // index among this block's tiles
         int4 en;
         bool have = cursor.next(use_bit, en);
-        ColInfo nxt;
-        if (have) nxt = col_info(en);
+        ColInfo nxt0, nxt1;
+        if (have) {
+            nxt0 = col_info(en, t);
+            nxt1 = col_info(en, t + 64);
+        }
         while (have) {
-            const ColInfo cur = nxt;
+            const ColInfo c0 = nxt0, c1 = nxt1;
             have = cursor.next(use_bit, en);
-            if (have) nxt = col_info(en);
+            if (have) {
+                nxt0 = col_info(en, t);
+                nxt1 = col_info(en, t + 64);
+            }
             const int ci = u % kNCI;
             if (!__all_sync(0xffffffffu, mbar_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, wd, 1))) break;
-            sCS[ci * 128 + t] = p.scale_log2 * cur.ks;
-            sCV[ci * 128 + t] = cur.vs;
-            sCW[ci * 128 + t] = cur.w;
+            sCS[ci * 128 + t] = p.scale_log2 * c0.ks;
+            sCV[ci * 128 + t] = c0.vs;
+            sCW[ci * 128 + t] = c0.w;
+            sCS[ci * 128 + t + 64] = p.scale_log2 * c1.ks;
+            sCV[ci * 128 + t + 64] = c1.vs;
+            sCW[ci * 128 + t + 64] = c1.w;
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_full[ci]);
             ++u;
         }
-    } else if (warp >= 12) {
-        setmaxnreg_dec<kRegMma>();
-        if (warp == 12 && lane == 0) {
+    } else if (warp >= kWarpMma) {
+        if (warp == kWarpMma && lane == 0) {
             // -------------------------------------------------------------- MMA issuer
             wd.where = 4;
             constexpr uint32_t idesc_s = idesc_f16_f32(128, 128, false, false);
@@ -351,7 +351,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             umma_commit(o_final);
             // the MMAs must be complete before the CTA releases TMEM, also on the abort path
             if (!ok) mbar_drain(o_final, 0, 100000000ull);
-        } else if (warp == 13 && lane == 0) {
+        } else if (warp == kWarpTma && lane == 0) {
             // -------------------------------------------------------------- TMA producer
             wd.where = 5;
             prefetch_tmap(&tm_kc);
@@ -399,21 +399,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else {
         // ------------------------------------------------------------------ softmax warpgroups
         // Waits are made warp-uniform (__all_sync) because tcgen05.ld/st are warp-collective.
-        setmaxnreg_inc<kRegSoftmax>();
-        const int half = warp >> 2;         // key columns [64 * half, 64 * half + 64) of each tile
+        const int wg = warp >> 2;           // tiles u with u % 2 == wg; S buffer wg
         const int g = warp & 3;             // TMEM lane group
-        wd.where = 1 + half;
+        wd.where = 1 + wg;
         const int r = g * 32 + lane;
         const int64_t row = qrow0 + r;
         const bool row_ok = row < p.Nq;
         const int frame = (int)((row_ok ? row : 0) / p.T);
         const uint32_t lane_base = (uint32_t)(g * 32) << 16;
-        constexpr int DH = D / 2;           // head-dim elements of Q and O handled by this half
-        // Q row r, elements [half * DH, half * DH + DH) -> fp16 pairs in TMEM
+        constexpr int DH = D / 2;           // head-dim elements of Q and O this warpgroup loads / stores
+        // Q row r, elements [wg * DH, wg * DH + DH) -> fp16 pairs in TMEM
         {
             uint32_t qp[DH / 2];
             const uint4 *src = reinterpret_cast<const uint4 *>(p.q + (row_ok ? row : 0) * p.tok_stride +
-                                                               (int64_t)h * p.head_stride + half * DH);
+                                                               (int64_t)h * p.head_stride + wg * DH);
             bool bad = false;
 #pragma unroll
             for (int i = 0; i < DH / 8; ++i) {
@@ -425,7 +424,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 qp[4 * i + 3] = v.w;
             }
             if (bad) set_device_error(p.err, NOMAS_ERANGE, 33);   // q outside the fp16 range
-            const uint32_t tq = tmem + lane_base + kTmQ + (uint32_t)(half * DH / 2);
+            const uint32_t tq = tmem + lane_base + kTmQ + (uint32_t)(wg * DH / 2);
             if constexpr (DH / 2 == 32) {
                 tmem_st32(tq, qp);
             } else {
@@ -436,30 +435,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(q_ready);
         }
-        float m_used = -INFINITY;
+        // Running offset (log2 units) of the row: the chain of decisions in tile order.  Tile u's
+        // warpgroup starts from the offset settled after tile u - 1 (written by the other warpgroup),
+        // raises it only when the tile's maximum exceeds it by more than kRescaleThreshold (then O is
+        // rescaled once PV of tile u - 1 has completed), and passes it on.  This warpgroup's partial
+        // row sum l is kept relative to my_m, the offset of its own latest tile.
+        float my_m = -INFINITY;
         float l = 0.0f;
         int u = 0;
         bool ok = true;
         ListCursor cursor(list, n_tiles);
         int4 e;
         while (cursor.next(use_bit, e)) {
+            if ((u & 1) != wg) {
+                ++u;
+                continue;
+            }
             const int ci = u % kNCI;
-            const int b = u & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(&ci_full[ci], (u / kNCI) & 1, wd, 1));
             if (!ok) break;
             const bool masked = (e.x & mask_bit) != 0;
             const bool cached = is_cached(e.x & 3);
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (u >> 1) & 1, wd, 2));
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], (u >> 1) & 1, wd, 2));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tS = tmem + lane_base + kTmS + (uint32_t)(b * 128 + half * 64);
-            float s[64];
-            tmem_ld64f_sync(tS, s);
+            const uint32_t tS = tmem + lane_base + kTmS + (uint32_t)(wg * 128);
+            float s[128];
+            tmem_ld128f_sync(tS, s);
             // cached keys: apply the per-key scale (which carries softmax scale * log2 e) to the score
             if (cached) {
-                const float4 *cs4 = reinterpret_cast<const float4 *>(sCS + ci * 128 + half * 64);
+                const float4 *cs4 = reinterpret_cast<const float4 *>(sCS + ci * 128);
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
+                for (int i = 0; i < 32; ++i) {
                     if ((i & 7) == 0) asm volatile("" ::: "memory");   // bound how far loads are hoisted
                     const float4 v = cs4[i];
                     const float2 a = __fmul2_rn(make_float2(s[4 * i], s[4 * i + 1]), make_float2(v.x, v.y));
@@ -471,45 +478,55 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             }
             if (masked) {
-                const int4 *cw = reinterpret_cast<const int4 *>(sCW + ci * 128 + half * 64);
+                const int4 *cw = reinterpret_cast<const int4 *>(sCW + ci * 128);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 64; ++i) {
                     if ((i & 7) == 0) asm volatile("" ::: "memory");
                     const int4 w = cw[i];   // windows of columns 2i and 2i+1
                     s[2 * i] = (w.x <= frame && frame < w.y) ? s[2 * i] : -INFINITY;
                     s[2 * i + 1] = (w.z <= frame && frame < w.w) ? s[2 * i + 1] : -INFINITY;
                 }
             }
-            // row maximum over this half (two independent max3 chains), then swapped with the other half
-            float m0 = max3(s[0], s[1], s[2]), m1 = max3(s[32], s[33], s[34]);
+            // row maximum over the tile (four independent max3 chains)
+            float mx[4];
 #pragma unroll
-            for (int c = 3; c < 31; c += 2) {
-                m0 = max3(m0, s[c], s[c + 1]);
-                m1 = max3(m1, s[32 + c], s[33 + c]);
-            }
-            const float pm = fmaxf(fmaxf(m0, s[31]), fmaxf(m1, s[63]));
-            sXM[(b * 2 + half) * 128 + r] = pm;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&xm_bar[b]);
-            ok = __all_sync(0xffffffffu, mbar_wait(&xm_bar[b], (u >> 1) & 1, wd, 3));
-            if (!ok) break;
-            const float po = sXM[(b * 2 + (half ^ 1)) * 128 + r];
+            for (int k = 0; k < 4; ++k) mx[k] = max3(s[32 * k], s[32 * k + 1], s[32 * k + 2]);
+#pragma unroll
+            for (int c = 3; c < 31; c += 2)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) mx[k] = max3(mx[k], s[32 * k + c], s[32 * k + c + 1]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], s[32 * k + 31]);
+            const float pm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             // log2 domain: cached scores are already scaled, bf16-source scores take the uniform scale
-            // (a positive factor commutes with the maximum exactly); both halves compute the same values
+            // (a positive factor commutes with the maximum exactly)
             const float cmul = cached ? 1.0f : p.scale_log2;
-            const float mt = fmaxf(pm, po) * cmul;
-            const float m_new = fmaxf(m_used, mt);
-            const bool grow = m_new > m_used + kRescaleThreshold;   // false while both are -inf
-            const bool need_o = grow && m_used != -INFINITY;
-            const float f = need_o ? ex2(m_used - m_new) : 1.0f;
-            if (grow) m_used = m_new;
-            const float off = (m_used == -INFINITY) ? 0.0f : m_used;
+            const float mt = pm * cmul;
+            float m_prev = -INFINITY;
+            if (u > 0) {   // the offset after tile u - 1, settled by the other warpgroup
+                ok = __all_sync(0xffffffffu, mbar_wait(&dec_full[wg ^ 1], ((u - 1) >> 1) & 1, wd, 3));
+                if (!ok) break;
+                m_prev = sDec[r];
+            }
+            const float m_new = fmaxf(m_prev, mt);
+            const bool grow = m_new > m_prev + kRescaleThreshold;   // false while both are -inf
+            const float m_cur = grow ? m_new : m_prev;
+            sDec[r] = m_cur;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dec_full[wg]);
+            if (m_cur != my_m) {   // this warpgroup's partial sum moves to the new offset
+                l = (my_m == -INFINITY) ? 0.0f : l * ex2(my_m - m_cur);
+                my_m = m_cur;
+            }
+            const bool need_o = grow && m_prev != -INFINITY;
+            const float f = need_o ? ex2(m_prev - m_cur) : 1.0f;
+            const float off = (m_cur == -INFINITY) ? 0.0f : m_cur;
             const float2 cm2 = make_float2(cmul, cmul);
             const float2 no2 = make_float2(-off, -off);
             float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-            const float2 *cv2 = reinterpret_cast<const float2 *>(sCV + ci * 128 + half * 64);
+            const float2 *cv2 = reinterpret_cast<const float2 *>(sCV + ci * 128);
 #pragma unroll
-            for (int qt = 0; qt < 2; ++qt) {
+            for (int qt = 0; qt < 4; ++qt) {   // keys 32 qt .. 32 qt + 31 -> P columns (qt / 2) * 64 + (qt % 2) * 16
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
@@ -520,20 +537,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     if (cached) pe = __fmul2_rn(pe, cv2[(qt * 32 + c) / 2]);
                     pk[c / 2] = f16x2_of(pe.x, pe.y);
                 }
-                tmem_st16(tS + qt * 16, pk);
+                tmem_st16(tS + (uint32_t)((qt >> 1) * 64 + (qt & 1) * 16), pk);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_empty[ci]);   // column info no longer needed
-            l = l * f + ((acc[0].x + acc[1].x) + (acc[0].y + acc[1].y));
-            // rescale this half of O (rare: only when some row's maximum grew past the threshold) once
-            // PV of the previous tile is complete; S_u's completion already implies PV_{u-2}'s
+            l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);   // l is already relative to m_cur
+            // rescale O (rare: only when some row's maximum grew past the threshold) once PV of tile
+            // u - 1 is complete; S_u's completion already implies PV_{u-2}'s, and PV_u waits for this
+            // warpgroup's P
             if (__any_sync(0xffffffffu, need_o)) {
                 ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (u - 1) & 1, wd, 4));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(half * DH);
+                const uint32_t tO = tmem + lane_base + kTmO;
 #pragma unroll 1
-                for (int c0 = 0; c0 < DH; c0 += 32) {
+                for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t rr[32];
                     tmem_ld32_sync(tO + c0, rr);
 #pragma unroll
@@ -544,23 +562,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[b]);
+            if (lane == 0) mbar_arrive(&p_full[wg]);
             ++u;
         }
-        // epilogue: the two halves' row sums, then O / l over this half's columns
+        // epilogue: combine the two warpgroups' row sums at the final offset (the later of the two
+        // warpgroups' offsets: the chain never lowers it), then O / l over this warpgroup's columns
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_final, 0, wd, 5));
         if (ok) {
-            sXL[half * 128 + r] = l;
+            sXL[wg * 128 + r] = l;
+            sXM[wg * 128 + r] = my_m;
             __syncwarp();
             if (lane == 0) mbar_arrive(xl_bar);
             ok = __all_sync(0xffffffffu, mbar_wait(xl_bar, 0, wd, 6));
         }
         if (ok) {
             tc_fence_after();
-            const float lt = l + sXL[(half ^ 1) * 128 + r];
+            const float ma = sXM[r], mb = sXM[128 + r];
+            const float mf = fmaxf(ma, mb);
+            const float la = ma == -INFINITY ? 0.0f : sXL[r] * ex2(ma - mf);
+            const float lb = mb == -INFINITY ? 0.0f : sXL[128 + r] * ex2(mb - mf);
+            const float lt = la + lb;
             const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-            float *dst = p.out + (row * p.H + h) * (int64_t)D + half * DH;
-            const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(half * DH);
+            float *dst = p.out + (row * p.H + h) * (int64_t)D + wg * DH;
+            const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(wg * DH);
 #pragma unroll 1
             for (int c0 = 0; c0 < DH; c0 += 32) {
                 uint32_t rr[32];
@@ -575,14 +599,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                 }
             }
-            if (p.lse && row_ok && half == 0)
-                p.lse[(int64_t)h * p.Nq + row] = (m_used + log2f(lt)) * 0.69314718055994530942f;
+            if (p.lse && row_ok && wg == 0)
+                p.lse[(int64_t)h * p.Nq + row] = (mf + log2f(lt)) * 0.69314718055994530942f;
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 12) {
+    if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -595,40 +619,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // ------------------------------------------------------------------------------------------------
 namespace nomas {
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult qr = cudaDriverEntryPointSymbolNotFound;
-        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr);
-        if (e == cudaSuccess && qr == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(ptr);
-        else cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", e != cudaSuccess ? (int)e : (int)qr,
-                       e != cudaSuccess ? cudaGetErrorString(e) : "symbol query failed");
-    }
-    return fn;
-}
-
 // 3-D tiled map.  dims / strides are innermost first (strides in bytes for dims 1 and 2).
 static bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, const cuuint64_t dims[3],
                      const cuuint64_t strides[2], const cuuint32_t box[3], CUtensorMapSwizzle swz) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint32_t es[3] = {1, 1, 1};
-    const CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        char msg[160];
-        std::snprintf(msg, sizeof(msg), "dims %llu x %llu x %llu, strides %llu %llu", (unsigned long long)dims[0],
-                      (unsigned long long)dims[1], (unsigned long long)dims[2], (unsigned long long)strides[0],
-                      (unsigned long long)strides[1]);
-        cuda_fail("cuTensorMapEncodeTiled", (int)r, msg);
-        return false;
-    }
-    return true;
+    return make_tensor_map_3d(m, dt, base, dims, strides, box, swz);
 }
 
 static int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -684,7 +678,6 @@ static WsHeader ws_header(const nomas_kv_cache *c, const nomas_mask_layout &lay)
     return h;
 }
 
-static uint64_t g_timeout_ns = 2000000000ull;   // 2 s per wait
 
 template <int D>
 static int launch_attn(const AttnParams &p, dim3 grid, const CUtensorMap *maps, cudaStream_t st) {
@@ -872,7 +865,7 @@ static int enqueue_run(const nomas_kv_cache *c, const nomas_mask_layout &lay, in
     p.out = out;
     p.lse = lse;
     p.err = static_cast<int *>(c->buf[NOMAS_BUF_ERR]);
-    p.timeout_ns = g_timeout_ns;
+    p.timeout_ns = wait_limit_ns();
     dim3 grid((unsigned)lay.n_qblocks, (unsigned)H);
     return D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
 }
@@ -880,12 +873,6 @@ static int enqueue_run(const nomas_kv_cache *c, const nomas_mask_layout &lay, in
 }  // namespace nomas
 
 using namespace nomas;
-
-extern "C" uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns) {
-    const uint64_t prev = g_timeout_ns;
-    g_timeout_ns = limit_ns;
-    return prev;
-}
 
 extern "C" size_t nomas_attn_workspace_bytes(const nomas_kv_cache *c, const nomas_segment_text *seg) {
     nomas_mask_layout lay;

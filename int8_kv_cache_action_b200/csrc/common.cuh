@@ -69,16 +69,30 @@ struct Watchdog {
     int where;
 };
 
+// Non-blocking test of phase `parity` (try_wait may suspend the thread for a while before it reports).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of `bar` to complete, giving up after wd.limit_ns (checked every 32 polls;
-// a limit of 0 gives up right after the first unsuccessful poll, without reading the timer).
+// a limit of 0 gives up at once unless a first, non-blocking test finds the phase complete).
 // Returns false when the CTA is aborting (this wait or another one ran out).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const Watchdog &wd, int site) {
-    if (mbar_try_wait(bar, parity)) return true;
     if (wd.limit_ns == 0) {
+        if (mbar_test_wait(bar, parity)) return true;
         set_device_error(wd.err, NOMAS_ETIMEOUT, wd.where * 100 + site);
         *wd.abort = 1;
         return false;
     }
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
 #pragma unroll 1
@@ -205,6 +219,25 @@ __device__ __forceinline__ void tmem_ld64f_sync(uint32_t taddr, float *r) {
         "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
         "tcgen05.wait::ld.sync.aligned;"
         : NOMAS_F8(0), NOMAS_F8(8), NOMAS_F8(16), NOMAS_F8(24), NOMAS_F8(32), NOMAS_F8(40), NOMAS_F8(48), NOMAS_F8(56)
+        : "r"(taddr)
+        : "memory");
+}
+// 128 consecutive TMEM columns of this thread's lane in one load, then one wait.
+__device__ __forceinline__ void tmem_ld128f_sync(uint32_t taddr, float *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x128.b32 {"
+        "%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,"
+        "%64,%65,%66,%67,%68,%69,%70,%71,%72,%73,%74,%75,%76,%77,%78,%79,"
+        "%80,%81,%82,%83,%84,%85,%86,%87,%88,%89,%90,%91,%92,%93,%94,%95,"
+        "%96,%97,%98,%99,%100,%101,%102,%103,%104,%105,%106,%107,%108,%109,%110,%111,"
+        "%112,%113,%114,%115,%116,%117,%118,%119,%120,%121,%122,%123,%124,%125,%126,%127}, [%128];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : NOMAS_F8(0), NOMAS_F8(8), NOMAS_F8(16), NOMAS_F8(24), NOMAS_F8(32), NOMAS_F8(40), NOMAS_F8(48), NOMAS_F8(56),
+          NOMAS_F8(64), NOMAS_F8(72), NOMAS_F8(80), NOMAS_F8(88), NOMAS_F8(96), NOMAS_F8(104), NOMAS_F8(112),
+          NOMAS_F8(120)
         : "r"(taddr)
         : "memory");
 }

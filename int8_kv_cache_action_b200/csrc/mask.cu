@@ -154,10 +154,11 @@ __global__ void lists_dense_kernel(MaskParams p) {
 
 constexpr int kPoolAhead = 8;   // rows loaded before they are added (independent loads in flight)
 
-// Block means.  Units [0, H*n_qb) are query blocks (head-major), then H*n_cand key candidates
-// (history blocks in age order, then current-segment blocks).  A unit is handled by D/8 lanes, each
-// summing 8 channels (one 16-byte load per row, so the lanes of a unit read a row of one head
-// contiguously); a warp takes 32/(D/8) consecutive units.  Every channel is summed by one lane over
+// Block means.  Units [0, H*n_qb) are query blocks, then H*n_cand key candidates (history blocks in age
+// order, then current-segment blocks); query and current-key units are numbered block-major (heads
+// inner), so the consecutive units of a CTA read whole [tokens][heads][D] rows together.  A unit is
+// handled by D/8 lanes, each summing 8 channels (one 16-byte load per row); a warp takes 32/(D/8)
+// consecutive units.  Every channel is summed by one lane over
 // the block's valid rows in ascending order from +0 (history keys as fp32(code) * scale, one rounding),
 // then divided once by the number of valid rows.  Loads run kPoolAhead rows ahead of the additions,
 // which keep the row order.
@@ -183,16 +184,25 @@ __global__ void __launch_bounds__(256) pool_kernel(MaskParams p, float *qmean, f
         const __nv_bfloat16 *src = nullptr;
         int64_t h, r0;
         if (u < nq_units) {
-            h = u / p.n_qb;
-            r0 = (u % p.n_qb) * (int64_t)kTile;
+            const int64_t b = u / p.H;
+            h = u - b * p.H;
+            r0 = b * (int64_t)kTile;
             nv = (int)(p.Nq - r0 < kTile ? p.Nq - r0 : kTile);
             src = p.q + r0 * ts + h * p.head_stride + sub * 8;
-            dst = qmean + u * D + sub * 8;
+            dst = qmean + (h * p.n_qb + b) * D + sub * 8;
         } else {
             const int64_t v = u - nq_units;
-            h = v / p.n_cand;
-            const int cand = (int)(v % p.n_cand);
-            dst = kmean + v * D + sub * 8;
+            int cand;
+            if (v < (int64_t)p.H * p.n_hist_tiles) {     // history: head-major (rows of a head are contiguous)
+                h = v / p.n_hist_tiles;
+                cand = (int)(v - h * p.n_hist_tiles);
+            } else {                                     // current keys: block-major like the queries
+                const int64_t w2 = v - (int64_t)p.H * p.n_hist_tiles;
+                const int64_t b = w2 / p.H;
+                h = w2 - b * p.H;
+                cand = p.n_hist_tiles + (int)b;
+            }
+            dst = kmean + (h * p.n_cand + cand) * D + sub * 8;
             if (cand < p.n_hist_tiles) {
                 hist = true;
                 r0 = (int64_t)cand * kTile;
@@ -361,11 +371,12 @@ __global__ void __launch_bounds__(256) select_lists_kernel(MaskParams p, int npo
         keys[i] = k;
     }
     __syncthreads();
-    // bitonic network on each npow2-long segment (pairs never cross a segment: j < npow2)
+    // bitonic network on each npow2-long segment (pairs never cross a segment: j < npow2); j is a
+    // power of two, so the pair index splits with a shift and a mask
     for (int k = 2; k <= npow2; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int j = k >> 1, lj = __ffs(k) - 2; j > 0; j >>= 1, --lj) {
             for (int t = threadIdx.x; t < npow2; t += blockDim.x) {   // 2 * npow2 / 2 pairs
-                const int e = 2 * j * (t / j) + (t % j);              // lower element, bit j clear
+                const int e = ((t >> lj) << (lj + 1)) | (t & (j - 1));  // lower element, bit j clear
                 const bool up = ((e & (npow2 - 1)) & k) == 0;
                 const unsigned long long a = keys[e], b = keys[e + j];
                 if ((a > b) == up) {

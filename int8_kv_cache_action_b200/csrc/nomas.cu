@@ -1,4 +1,5 @@
 // libnomas host entry points: cache handle, buffer sizes, state, status, mask-buffer layout.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -23,11 +24,67 @@ int check_launch(const char *what) {
     return e == cudaSuccess ? NOMAS_OK : cuda_fail(what, (int)e, cudaGetErrorString(e));
 }
 
+static std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};   // 2 s per wait
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+
 int bind_device(const nomas_kv_cache *c) {
     int cur = -1;
     if (cudaGetDevice(&cur) == cudaSuccess && cur == c->device) return NOMAS_OK;
     const cudaError_t e = cudaSetDevice(c->device);
     return e == cudaSuccess ? NOMAS_OK : cuda_fail("cudaSetDevice", (int)e, cudaGetErrorString(e));
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load();
+    if (!f) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult qr = cudaDriverEntryPointSymbolNotFound;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr);
+        if (e == cudaSuccess && qr == cudaDriverEntryPointSuccess) {
+            f = reinterpret_cast<EncodeTiledFn>(ptr);
+            fn.store(f);
+        } else {
+            cuda_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", e != cudaSuccess ? (int)e : (int)qr,
+                      e != cudaSuccess ? cudaGetErrorString(e) : "symbol query failed");
+        }
+    }
+    return f;
+}
+
+bool make_tensor_map_3d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, const cuuint64_t dims[3],
+                        const cuuint64_t strides[2], const cuuint32_t box[3], CUtensorMapSwizzle swz) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint32_t es[3] = {1, 1, 1};
+    const CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char msg[160];
+        std::snprintf(msg, sizeof(msg), "dims %llu x %llu x %llu, strides %llu %llu", (unsigned long long)dims[0],
+                      (unsigned long long)dims[1], (unsigned long long)dims[2], (unsigned long long)strides[0],
+                      (unsigned long long)strides[1]);
+        cuda_fail("cuTensorMapEncodeTiled", (int)r, msg);
+        return false;
+    }
+    return true;
+}
+
+int sm_count() {
+    static std::atomic<int> counts[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int n = counts[dev].load();
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        counts[dev].store(n);
+    }
+    return n;
 }
 
 static size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -202,6 +259,10 @@ extern "C" int nomas_device_status(const nomas_kv_cache *c, nomas_stream stream)
 }
 
 extern "C" const char *nomas_last_error(void) { return g_last_error; }
+
+extern "C" uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns) {
+    return g_wait_limit_ns.exchange(limit_ns, std::memory_order_relaxed);
+}
 
 extern "C" const char *nomas_status_string(int s) {
     switch (s) {

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 
 #include "nomas.h"
 
@@ -83,5 +84,17 @@ int check_launch(const char *what);
 
 // Make the cache's device current for this thread (the library links its own CUDA runtime).
 int bind_device(const nomas_kv_cache *c);
+
+// Limit of every bounded device wait (nomas_set_wait_limit_ns), in nanoseconds.
+uint64_t wait_limit_ns();
+
+// Encode a 3-D tiled TMA map (no interleave, L2 256-byte promotion, zero fill out of bounds).  dims /
+// box are innermost first, strides in bytes for dims 1 and 2.  Records the failure for
+// nomas_last_error and returns false on error.
+bool make_tensor_map_3d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, const cuuint64_t dims[3],
+                        const cuuint64_t strides[2], const cuuint32_t box[3], CUtensorMapSwizzle swz);
+
+// Number of SMs of the current device (queried once per device).
+int sm_count();
 
 }  // namespace nomas

@@ -40,3 +40,33 @@ def test_forced_wait_limit_reports_timeout_and_context_stays_usable():
     torch.cuda.synchronize()
     assert gc.status() == N.NOMAS_OK
     assert torch.equal(again, ref)
+
+
+def test_forced_wait_limit_in_append_reports_timeout_and_the_next_append_is_exact():
+    # The append kernel's consumers wait for each chunk's TMA copy with the same bounded wait: with the
+    # limit at 0 the first wait that is not yet satisfied gives up, the kernel records NOMAS_ETIMEOUT
+    # and unwinds (the producer lets its copies land).  The ring contents of that call are undefined;
+    # a fresh cache on the same context then appends bit for bit as the oracle does.
+    import numpy as np
+    from int8_kv_cache_action_b200.runtime import KVCache
+    from tests.helpers import f32, oracle_cache
+    cfg = small_config(tokens_per_frame=880, n_frames=2, prior_frames=(6,), window=4, heads=16)
+    inp = make_inputs(cfg)
+    kv = inp.prior[0]
+    gc = KVCache.for_config(cfg)
+    prev = N.nomas_set_wait_limit_ns(0)
+    try:
+        gc.append(kv.k.cuda(), kv.v.cuda(), 6, kv.head_k.cuda(), kv.head_v.cuda())
+        torch.cuda.synchronize()
+        st = gc.status()
+    finally:
+        N.nomas_set_wait_limit_ns(prev)
+    assert st == N.NOMAS_ETIMEOUT
+    fresh = gpu_cache(cfg, inp)
+    assert fresh.status() == N.NOMAS_OK
+    oc = oracle_cache(cfg, inp)
+    T = cfg.tokens_per_frame
+    for g in oc.retained_frames():
+        s = slice((g % oc.C) * T, (g % oc.C + 1) * T)
+        assert np.array_equal(fresh.ring_k8().cpu().numpy()[:, s], oc.k8[:, s])
+        assert np.array_equal(fresh.ring_vs().cpu().numpy()[:, s].view(np.uint32), oc.vs[:, s].view(np.uint32))

@@ -7,6 +7,8 @@ tails of 64):
   a2  nomas_mask_build    dense visibility classes and tile lists
   a4  nomas_attn_prepare  operand pre-pass: current/text K,V to fp16, INT8 history codes widened to fp16
       nomas_attn_run      dense masked attention (steps 1-2 of a segment's denoising)
+  a4" nomas_mask_build + nomas_attn_run (NOMAS_MODE_TEXT)   the text query rows of the same joint
+      attention (the text stream), over the workspace the video call prepared (same K/V and cache)
   a3  nomas_mask_build    sparse selection (25 % of candidate video blocks)
   a4' nomas_attn_prepare + nomas_attn_run   block-sparse attention (steps 3-8)
 (nomas_attn_fwd is exactly prepare + run; they are called separately so each is timed.)
@@ -35,17 +37,19 @@ METRIC = "masked attention TFLOP/s (dense + 25% block-sparse step, INT8 KV histo
 
 def step_config(cfg, world):
     """The `config` object of the JSON line; both arms report the same one."""
-    return {"workload": "production_1280x704: 16x128, 30-frame segment (26400 queries), 18-frame INT8 "
-                        "history (15840 keys), 768 head + 8 tails x 64; step = append + dense mask + "
-                        "dense attention + sparse selection (25%) + sparse attention",
+    return {"workload": "production_1280x704: 16x128, 30-frame segment (26400 video + 1280 text queries), "
+                        "18-frame INT8 history (15840 keys), 768 head + 8 tails x 64; step = append + dense "
+                        "mask + dense attention (video rows) + text-row mask + text-row attention + sparse "
+                        "selection (25%) + sparse attention",
             "seq_len": cfg.n_query, "heads": cfg.heads, "head_dim": cfg.head_dim,
             "l2": "inputs larger than L2 (324 MB bf16 q/k/v per step)", "parallelism": f"replica x{world}"}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
 # Kernel launches of one step: append 1; dense mask 3; prepare 3 (key copy, transposed values, history
-# widening); dense attention 1; sparse mask 5; prepare 3; sparse attention 1.
-LAUNCHES_PER_STEP = 17
+# widening); dense attention 1; text mask 3; text attention 1; sparse mask 5; prepare 3; sparse
+# attention 1.
+LAUNCHES_PER_STEP = 21
 CSRC = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc")
 COMMON = os.path.join(CSRC, "common.cuh")
 TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose digest it was taken with)
@@ -112,6 +116,19 @@ def visible_key_sum(cfg, hist_tokens, head_tokens):
     tot = 0
     for t in range(F):
         tot += T * (base + sum(a.len for a in cfg.current.tails if a.f0 <= t < a.f1))
+    return tot
+
+
+def text_key_sum(cfg, hist_tokens, head_tokens):
+    """Sum over the current text rows of visible keys: a head row sees history, earlier heads, all current
+    video and the current head; a row of tail a sees history, earlier heads, the current head, the video
+    frames of its window and the tails whose window shares a frame with its own."""
+    T, seg = cfg.tokens_per_frame, cfg.current
+    ctx = hist_tokens + head_tokens + seg.head_len
+    tot = seg.head_len * (ctx + cfg.n_query)
+    for a in seg.tails:
+        tails = sum(b.len for b in seg.tails if max(a.f0, b.f0) < min(a.f1, b.f1))
+        tot += a.len * (ctx + (a.f1 - a.f0) * T + tails)
     return tot
 
 
@@ -206,7 +223,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     cfg = CONFIGS[WORKLOAD]
     inp = make_inputs(cfg, seed_offset=rank)
-    q, kc, vc, kt, vt = (getattr(inp, n).to(dev) for n in ("q", "k_cur", "v_cur", "k_txt", "v_txt"))
+    q, kc, vc, kt, vt, qt = (getattr(inp, n).to(dev) for n in ("q", "k_cur", "v_cur", "k_txt", "v_txt", "q_txt"))
     prev = inp.prior[-1]
     pk, pv = prev.k.to(dev), prev.v.to(dev)
     cache = KVCache.for_config(cfg, dev)
@@ -217,10 +234,13 @@ def run_ours(args, rank, world, local_rank):
     s = st.cuda_stream
     lay_d = cache.mask_layout(seg, N.NOMAS_MODE_DENSE)
     lay_s = cache.mask_layout(seg, N.NOMAS_MODE_SPARSE, 0.25)
+    lay_t = cache.mask_layout(seg, N.NOMAS_MODE_TEXT)
+    mbuf_t = torch.empty(lay_t["total_bytes"], dtype=torch.uint8, device=dev)
     mbuf_d = torch.empty(lay_d["total_bytes"], dtype=torch.uint8, device=dev)
     mbuf_s = torch.empty(lay_s["total_bytes"], dtype=torch.uint8, device=dev)
     out_d = torch.empty((cfg.n_query, cfg.heads, cfg.head_dim), dtype=torch.float32, device=dev)
     out_s = torch.empty_like(out_d)
+    out_t = torch.empty((cfg.current.text_len, cfg.heads, cfg.head_dim), dtype=torch.float32, device=dev)
     ws = cache.workspace(seg)
     scale = 1.0 / math.sqrt(cfg.head_dim)
     ts, hs = q.stride(0), q.stride(1)
@@ -230,7 +250,8 @@ def run_ours(args, rank, world, local_rank):
         if rc != 0:
             raise N.NomasError(rc, what)
 
-    bufs0 = {"q": q, "kc": kc, "vc": vc, "kt": kt, "vt": vt, "pk": pk, "pv": pv, "out_d": out_d, "out_s": out_s}
+    bufs0 = {"q": q, "kc": kc, "vc": vc, "kt": kt, "vt": vt, "qt": qt, "pk": pk, "pv": pv, "out_d": out_d,
+             "out_t": out_t, "out_s": out_s}
 
     def step(ev=None, b=bufs0, stream=None):
         sh = s if stream is None else stream.cuda_stream
@@ -255,14 +276,19 @@ def run_ours(args, rank, world, local_rank):
         check(N.nomas_attn_run(cache.handle, seg, 0, 0.25, mbuf_d.data_ptr(), b["q"].data_ptr(), ts, hs, scale,
                                b["out_d"].data_ptr(), 0, ws.data_ptr(), sh), "attn dense")
         mark(4)
+        check(N.nomas_mask_build(cache.handle, seg, 2, 0.25, 0, 0, ts, hs, mbuf_t.data_ptr(), sh), "mask text")
+        mark(5)
+        check(N.nomas_attn_run(cache.handle, seg, 2, 0.25, mbuf_t.data_ptr(), b["qt"].data_ptr(), ts, hs, scale,
+                               b["out_t"].data_ptr(), 0, ws.data_ptr(), sh), "attn text")
+        mark(6)
         check(N.nomas_mask_build(cache.handle, seg, 1, 0.25, b["q"].data_ptr(), b["kc"].data_ptr(), ts, hs,
                                  mbuf_s.data_ptr(), sh), "mask sparse")
-        mark(5)
+        mark(7)
         prepare()
-        mark(6)
+        mark(8)
         check(N.nomas_attn_run(cache.handle, seg, 1, 0.25, mbuf_s.data_ptr(), b["q"].data_ptr(), ts, hs, scale,
                                b["out_s"].data_ptr(), 0, ws.data_ptr(), sh), "attn sparse")
-        mark(7)
+        mark(9)
 
     for _ in range(args.warmup):
         step()
@@ -271,6 +297,7 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError("device error during warm-up")
     st_now = cache.state()
     flops_dense = 4.0 * cfg.head_dim * cfg.heads * visible_key_sum(cfg, st_now["history_tokens"], st_now["head_tokens"])
+    flops_text = 4.0 * cfg.head_dim * cfg.heads * text_key_sum(cfg, st_now["history_tokens"], st_now["head_tokens"])
     mv = mask_views(mbuf_s, lay_s)
     flops_sparse = 4.0 * cfg.head_dim * sparse_key_sum(mv["sel"], cfg, st_now["history_tokens"],
                                                        st_now["head_tokens"])
@@ -301,11 +328,11 @@ def run_ours(args, rank, world, local_rank):
     # per-phase breakdown: a separate pass of steps issued back to back with events between the
     # phases (no host synchronisation inside the pass, so no phase includes host launch latency)
     n_ph = max(3, min(args.steps, 10))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(n_ph)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(n_ph)]
     for k in range(n_ph):
         step(evs[k])
     torch.cuda.synchronize()
-    ph = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(n_ph)) for i in range(7)]
+    ph = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(n_ph)) for i in range(9)]
 
     # end to end: every step copies its inputs from pinned host memory, runs the same C-ABI calls and
     # copies both outputs back.  Like a serving loop, the copies of one step overlap the compute of
@@ -315,13 +342,14 @@ def run_ours(args, rank, world, local_rank):
     # the last D2H copy.
     e2e = None
     if rank == 0 or world > 1:
-        names = ("q", "kc", "vc", "kt", "vt", "pk", "pv")
+        names = ("q", "kc", "vc", "kt", "vt", "qt", "pk", "pv")
         host = {n: bufs0[n].cpu().pin_memory() for n in names}
-        bufs1 = {n: torch.empty_like(bufs0[n]) for n in names + ("out_d", "out_s")}
+        bufs1 = {n: torch.empty_like(bufs0[n]) for n in names + ("out_d", "out_t", "out_s")}
         sets = [bufs0, bufs1]
-        hout = [[torch.empty(out_d.shape, dtype=torch.float32).pin_memory() for _ in range(2)] for _ in range(2)]
+        hout = [[torch.empty(bufs0[o].shape, dtype=torch.float32).pin_memory() for o in ("out_d", "out_t", "out_s")]
+                for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in host.values())
-        d2h = 2 * out_d.numel() * 4
+        d2h = (2 * out_d.numel() + out_t.numel()) * 4
         s_h2d, s_d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
         done = [torch.cuda.Event() for _ in range(2)]
         ready = [torch.cuda.Event() for _ in range(2)]
@@ -348,12 +376,13 @@ def run_ours(args, rank, world, local_rank):
             s_d2h.wait_event(done[i])
             with torch.cuda.stream(s_d2h):
                 hout[i][0].copy_(b["out_d"], non_blocking=True)
-                hout[i][1].copy_(b["out_s"], non_blocking=True)
+                hout[i][1].copy_(b["out_t"], non_blocking=True)
+                hout[i][2].copy_(b["out_s"], non_blocking=True)
             out_free[i].record(s_d2h)
         e1.record(s_d2h)
         torch.cuda.synchronize()
         ems, _ = aggregate_ranks(e0.elapsed_time(e1) / n_e2e, 0.0, world, reduce_max)   # slowest rank
-        e2e = {"value": (flops_dense + flops_sparse) / (ems * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
+        e2e = {"value": (flops_dense + flops_text + flops_sparse) / (ems * 1e-3) / 1e12 * world, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": n_e2e,
                "pipelined": "H2D / compute / D2H on three streams, two buffer sets"}
     ws_bytes = {"production_1280x704": int(ws.numel())}
@@ -362,7 +391,8 @@ def run_ours(args, rank, world, local_rank):
     c4 = KVCache.for_config(big, dev)
     ws_bytes["full_history_7th_of_7"] = int(N.nomas_attn_workspace_bytes(c4.handle, segment_text_of(big.current)))
     del c4
-    return dict(ms=ms, phases=ph, flops_dense=flops_dense, flops_sparse=flops_sparse, append_bytes=append_bytes,
+    return dict(ms=ms, phases=ph, flops_dense=flops_dense, flops_text=flops_text, flops_sparse=flops_sparse,
+                append_bytes=append_bytes,
                 prep_bytes=prep_bytes, ws_bytes=ws_bytes, clocks=clk.summary(), e2e=e2e, cfg=cfg)
 
 
@@ -545,16 +575,18 @@ def main():
         return
     cfg = r["cfg"]
     ms_step = r["ms"] / args.steps
-    flops = r["flops_dense"] + r["flops_sparse"]
+    flops = r["flops_dense"] + r["flops_text"] + r["flops_sparse"]
     _, value = aggregate_ranks(ms_step, flops, world)
     value /= 1e12
-    ph = r["phases"]   # append, mask dense, prepare, run dense, mask sparse, prepare, run sparse
+    # append, mask dense, prepare, run dense, mask text, run text, mask sparse, prepare, run sparse
+    ph = r["phases"]
     dense_tflops = r["flops_dense"] / (ph[3] * 1e-3) / 1e12
-    sparse_tflops = r["flops_sparse"] / (ph[6] * 1e-3) / 1e12
+    text_tflops = r["flops_text"] / (ph[5] * 1e-3) / 1e12
+    sparse_tflops = r["flops_sparse"] / (ph[8] * 1e-3) / 1e12
     dense_call_tflops = r["flops_dense"] / ((ph[2] + ph[3]) * 1e-3) / 1e12
-    sparse_call_tflops = r["flops_sparse"] / ((ph[5] + ph[6]) * 1e-3) / 1e12
+    sparse_call_tflops = r["flops_sparse"] / ((ph[7] + ph[8]) * 1e-3) / 1e12
     append_gbs = r["append_bytes"] / (ph[0] * 1e-3) / 1e9
-    prep_ms = 0.5 * (ph[2] + ph[5])
+    prep_ms = 0.5 * (ph[2] + ph[7])
     prep_gbs = r["prep_bytes"] / (prep_ms * 1e-3) / 1e9
     peak_sus = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -581,11 +613,13 @@ def main():
                              "achieved": prep_gbs, "peak": hbm, "unit": "GB/s", "frac": prep_gbs / hbm,
                              "bytes_per_call": r["prep_bytes"], "ms_per_call": prep_ms, "traffic": None},
         "breakdown_ms": {"append": ph[0], "mask_dense": ph[1], "prepare_dense": ph[2], "attn_dense": ph[3],
-                         "mask_sparse": ph[4], "prepare_sparse": ph[5], "attn_sparse": ph[6]},
+                         "mask_text": ph[4], "attn_text": ph[5], "mask_sparse": ph[6], "prepare_sparse": ph[7],
+                         "attn_sparse": ph[8]},
+        "attn_text_tflops": text_tflops,
         "attn_dense_tflops": dense_tflops, "attn_sparse_tflops": sparse_tflops,
         "attn_dense_call_tflops": dense_call_tflops, "attn_sparse_call_tflops": sparse_call_tflops,
         "attn_workspace_bytes": r["ws_bytes"],
-        "flops_per_step": {"dense": r["flops_dense"], "sparse": r["flops_sparse"]},
+        "flops_per_step": {"dense": r["flops_dense"], "text": r["flops_text"], "sparse": r["flops_sparse"]},
         "kv_tokens_per_s_append": (cfg.window_frames * cfg.tokens_per_frame) * cfg.heads / (ph[0] * 1e-3),
         "cpu_baseline": cpu_base,
         "e2e": r["e2e"],

@@ -142,6 +142,17 @@ int nomas_kv_append(nomas_kv_cache *cache, const void *k, const void *v, int64_t
 
 #define NOMAS_MODE_DENSE 0
 #define NOMAS_MODE_SPARSE 1
+/* Text query rows of the current segment (the text stream of the double-stream joint attention,
+ * papers.ananclaw.com "干货攻略", 这是什么), always dense.  The pages say who may see the text, not what
+ * the text sees; this library's reading: a description-head row sees the retained history, earlier
+ * heads, all current video and the current head, but no action tail (the head is cached and visible
+ * across segments, so it must not carry the segment's actions); a row of tail a (window [f0, f1))
+ * sees the history, earlier heads and the current head, the current video frames t with
+ * f0 <= t < f1, and the tails whose window shares a frame with a's (itself included).  In this mode
+ * nomas_mask_build needs no q / kcur, and nomas_attn_run / nomas_attn_fwd read q as the text queries
+ * [text_tokens][H][D] and write out [text_tokens][H][D] and lse [H][text_tokens].  A row with no
+ * visible key (possible only in degenerate layouts) gets output 0. */
+#define NOMAS_MODE_TEXT 2
 
 /* Where mask_build puts its results inside the caller's mask buffer.
  * Key order for tiles and classes: retained history (age order), description

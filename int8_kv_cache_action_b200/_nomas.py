@@ -19,7 +19,7 @@ NOMAS_OK, NOMAS_EINVAL, NOMAS_ECAPACITY, NOMAS_ECUDA, NOMAS_ETIMEOUT, NOMAS_EDEV
     NOMAS_ESTATE, NOMAS_ERANGE = 0, -1, -2, -3, -4, -5, -6, -7, -8
 NOMAS_BUF_K8, NOMAS_BUF_V8, NOMAS_BUF_KS, NOMAS_BUF_VS, NOMAS_BUF_HK8, NOMAS_BUF_HV8, NOMAS_BUF_HKS, \
     NOMAS_BUF_HVS, NOMAS_BUF_ERR, NOMAS_NBUF = range(10)
-NOMAS_MODE_DENSE, NOMAS_MODE_SPARSE = 0, 1
+NOMAS_MODE_DENSE, NOMAS_MODE_SPARSE, NOMAS_MODE_TEXT = 0, 1, 2
 NOMAS_MAX_TAILS = 64
 NOMAS_STATIC_POOL_FLOATS = 2 << 20
 NOMAS_MAX_SPARSE_CANDIDATES = 8192

@@ -139,16 +139,18 @@ struct AppendJob {
 struct AppendParams {
     AppendJob job[2];
     int32_t heads, tokens_per_frame, capacity_frames;
+    FastDiv div_heads, div_frame;     // by heads, by tokens_per_frame
     int *err;
     uint64_t timeout_ns;
 };
 
-// Chunk c of the launch: job, head and token block (token blocks outer, heads inner).
-__device__ __forceinline__ void chunk_of(const AppendParams &a, int64_t c, int &job, int &h, int64_t &tb) {
-    job = c < a.job[0].n_chunks ? 0 : 1;
-    if (job) c -= a.job[0].n_chunks;
-    tb = c / a.heads;
-    h = (int)(c - tb * a.heads);
+// Chunk c of the launch (every count below 2^31): job, head and token block (token blocks outer,
+// heads inner).
+__device__ __forceinline__ void chunk_of(const AppendParams &a, uint32_t c, int &job, int &h, int &tb) {
+    job = c < (uint32_t)a.job[0].n_chunks ? 0 : 1;
+    if (job) c -= (uint32_t)a.job[0].n_chunks;
+    tb = (int)fdiv(c, a.div_heads);
+    h = (int)c - tb * a.heads;
 }
 
 template <int D>
@@ -185,12 +187,11 @@ __global__ void __launch_bounds__(kAppendThreads, 3)
             for (int64_t c = blockIdx.x; c < total; c += gridDim.x, ++i) {
                 const int st = i % kAppendStages;
                 if (!mbar_wait(&empty[st], ((i / kAppendStages) & 1) ^ 1, wd, 1)) break;
-                int job, h;
-                int64_t tb;
-                chunk_of(a, c, job, h, tb);
+                int job, h, tb;
+                chunk_of(a, (uint32_t)c, job, h, tb);
                 uint8_t *dk = sm + st * C::STAGE;
-                const int y = a.job[job].tok_outer ? h : (int)(tb * C::TC);
-                const int z = a.job[job].tok_outer ? (int)(tb * C::TC) : h;
+                const int y = a.job[job].tok_outer ? h : tb * C::TC;
+                const int z = a.job[job].tok_outer ? tb * C::TC : h;
                 mbar_arrive_expect_tx(&full[st], C::STAGE);
                 tma_load_3d(dk, job ? &tk1 : &tk0, &full[st], 0, y, z);
                 tma_load_3d(dk + C::TILE, job ? &tv1 : &tv0, &full[st], 0, y, z);
@@ -211,12 +212,11 @@ __global__ void __launch_bounds__(kAppendThreads, 3)
     for (int64_t c = blockIdx.x; c < total; c += gridDim.x, ++i) {
         const int st = i % kAppendStages;
         if (!__all_sync(0xffffffffu, mbar_wait(&full[st], (i / kAppendStages) & 1, wd, 2))) break;
-        int job, h;
-        int64_t tb;
-        chunk_of(a, c, job, h, tb);
+        int job, h, tb;
+        chunk_of(a, (uint32_t)c, job, h, tb);
         const AppendJob &J = a.job[job];
         const int row_in_chunk = warp * TB + grp;
-        const int64_t t = tb * C::TC + row_in_chunk;   // token within the job
+        const int t = tb * C::TC + row_in_chunk;       // token within the job
         const uint4 *sk = reinterpret_cast<const uint4 *>(sm + st * C::STAGE + row_in_chunk * D * 2 + sub * 32);
         const uint4 *sv = reinterpret_cast<const uint4 *>(sm + st * C::STAGE + C::TILE + row_in_chunk * D * 2 + sub * 32);
         float x[16];
@@ -232,8 +232,12 @@ __global__ void __launch_bounds__(kAppendThreads, 3)
             if (J.head_mode) {
                 row = J.dst_row0 + t;
             } else {
-                const int f = (int)(t / T);
-                row = (int64_t)((J.first_slot + f) % Cf) * T + (t - (int64_t)f * T);
+                // ring slot of the token's frame: first_slot + f < 2 C (f < min(frames, C) -- the job
+                // writes at most C frames), so one conditional subtraction replaces the modulo
+                const int f = (int)fdiv((uint32_t)t, a.div_frame);
+                int slot = J.first_slot + f;
+                if (slot >= Cf) slot -= Cf;
+                row = (int64_t)slot * T + (t - f * T);
             }
             const int64_t di = (int64_t)h * J.rows_per_head + row;
             *reinterpret_cast<uint4 *>(J.k8 + di * D + sub * 16) = qk;
@@ -304,6 +308,7 @@ static int launch_append(const CUtensorMap *maps, const AppendParams &a, cudaStr
     });
     if (attr != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(append smem)", (int)attr, cudaGetErrorString(attr));
     const int64_t total = a.job[0].n_chunks + a.job[1].n_chunks;
+    if (total >= ((int64_t)1 << 31)) return NOMAS_EINVAL;   // chunk ids are 32-bit
     int64_t blocks = (int64_t)sm_count() * 3;
     if (blocks > total) blocks = total;
     quant_append_kernel<D><<<(unsigned)blocks, kAppendThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], a);
@@ -344,6 +349,8 @@ extern "C" int nomas_kv_append(nomas_kv_cache *c, const void *k, const void *v, 
     a.capacity_frames = d.capacity_frames;
     a.err = static_cast<int *>(c->buf[NOMAS_BUF_ERR]);
     a.timeout_ns = wait_limit_ns();
+    a.div_heads = make_fastdiv((uint32_t)d.heads);
+    a.div_frame = make_fastdiv((uint32_t)d.tokens_per_frame);
     CUtensorMap maps[4];
     const void *kv_src[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
     AppendJob &jv = a.job[0];

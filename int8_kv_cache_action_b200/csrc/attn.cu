@@ -70,8 +70,8 @@ struct AttnCfg {
     static constexpr int OFF_V = OFF_K + NK * SLOT;
     static constexpr int OFF_CS = OFF_V + NV * SLOT;       // float [kNCI][128] key scale x log2 e
     static constexpr int OFF_CV = OFF_CS + kNCI * 512;     // float [kNCI][128] value scale
-    static constexpr int OFF_CW = OFF_CV + kNCI * 512;     // int2  [kNCI][128] key frame windows
-    static constexpr int OFF_DEC = OFF_CW + kNCI * 1024;   // float [128] running offset after the last tile
+    static constexpr int OFF_CW = OFF_CV + kNCI * 512;     // int4  [kNCI][128] key visibility codes
+    static constexpr int OFF_DEC = OFF_CW + kNCI * 2048;   // float [128] running offset after the last tile
     static constexpr int OFF_XM = OFF_DEC + 512;           // float [2 warpgroups][128] final offsets
     static constexpr int OFF_XL = OFF_XM + 1024;           // float [2 warpgroups][128] row sums
     static constexpr int OFF_BAR = OFF_XL + 1024;
@@ -91,11 +91,13 @@ struct AttnParams {
     const uint8_t *mask;
     const int4 *lists;
     const int32_t *counts;
-    const int2 *txtwin;
+    const int2 *txtwin;         // per text token: frame window (tails) or [0, kAlwaysHi) (head)
     MaskHeader expect;
     const WsHeader *ws_hdr;     // written by nomas_attn_prepare
     WsHeader ws_expect;
     int32_t sparse;
+    int32_t text_rows;          // query rows are the current text (NOMAS_MODE_TEXT), else the video
+    int32_t head_len;           // description-head tokens at the front of the current text
     int32_t n_pairs;
     // queries and shapes
     const __nv_bfloat16 *q;
@@ -163,7 +165,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint8_t *sV = sm + C::OFF_V;
     float *sCS = reinterpret_cast<float *>(sm + C::OFF_CS);
     float *sCV = reinterpret_cast<float *>(sm + C::OFF_CV);
-    int2 *sCW = reinterpret_cast<int2 *>(sm + C::OFF_CW);
+    int4 *sCW = reinterpret_cast<int4 *>(sm + C::OFF_CW);
     float *sDec = reinterpret_cast<float *>(sm + C::OFF_DEC);
     float *sXM = reinterpret_cast<float *>(sm + C::OFF_XM);
     float *sXL = reinterpret_cast<float *>(sm + C::OFF_XL);
@@ -250,19 +252,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int t = threadIdx.x - 32 * kWarpCi;   // 0..63
         struct ColInfo {
             float ks, vs;   // raw key / value scale (cached tiles), 1 / 0 otherwise
-            int2 w;
+            VisCode w;      // visibility code of the key
         };
-        // Column info of a tile (key scale, value scale, frame window), loaded one tile ahead of its
+        // Column info of a tile (key scale, value scale, visibility code), loaded one tile ahead of its
         // use: only loads happen here, so nothing waits for them until the next tile consumes them.
         auto col_info = [&](const int4 &e, int col) -> ColInfo {
-            ColInfo ci{0.0f, 0.0f, make_int2(kAlwaysHi, 0)};
+            ColInfo ci{0.0f, 0.0f, key_none()};
             const int kind = e.x & 3;
             const int64_t start = e.y;
             if (col < e.z) {
                 if (kind == kKindText) {
-                    ci.w = p.txtwin[start + col];
+                    if (start + col < p.head_len) {
+                        ci.w = key_always();
+                    } else {
+                        const int2 w = p.txtwin[start + col];
+                        ci.w = key_tail(w.x, w.y);
+                    }
+                } else if (kind == kKindCur) {
+                    ci.w = key_video((int)((start + col) / p.T));
                 } else {
-                    ci.w = make_int2(0, kAlwaysHi);
+                    ci.w = key_always();
                 }
                 if (is_cached(kind)) {
                     const bool hist = kind == kKindHist;
@@ -295,10 +304,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (!__all_sync(0xffffffffu, mbar_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, wd, 1))) break;
             sCS[ci * 128 + t] = p.scale_log2 * c0.ks;
             sCV[ci * 128 + t] = c0.vs;
-            sCW[ci * 128 + t] = c0.w;
+            sCW[ci * 128 + t] = make_int4(c0.w.x, c0.w.y, c0.w.z, c0.w.w);
             sCS[ci * 128 + t + 64] = p.scale_log2 * c1.ks;
             sCV[ci * 128 + t + 64] = c1.vs;
-            sCW[ci * 128 + t + 64] = c1.w;
+            sCW[ci * 128 + t + 64] = make_int4(c1.w.x, c1.w.y, c1.w.z, c1.w.w);
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_full[ci]);
             ++u;
@@ -405,7 +414,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int r = g * 32 + lane;
         const int64_t row = qrow0 + r;
         const bool row_ok = row < p.Nq;
-        const int frame = (int)((row_ok ? row : 0) / p.T);
+        // the row's visibility code: a video frame, or a text row of the head or of a tail
+        VisCode rc;
+        if (!p.text_rows) {
+            rc = row_video((int)((row_ok ? row : 0) / p.T));
+        } else if (!row_ok || row < p.head_len) {
+            rc = row_head();
+        } else {
+            const int2 w = p.txtwin[row];
+            rc = row_tail(w.x, w.y);
+        }
         const uint32_t lane_base = (uint32_t)(g * 32) << 16;
         constexpr int DH = D / 2;           // head-dim elements of Q and O this warpgroup loads / stores
         // Q row r, elements [wg * DH, wg * DH + DH) -> fp16 pairs in TMEM
@@ -456,6 +474,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (!ok) break;
             const bool masked = (e.x & mask_bit) != 0;
             const bool cached = is_cached(e.x & 3);
+            // visibility of the tile's keys to this row, as 128 bits, taken before the scores are loaded
+            uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
+            if (masked) {
+                const int4 *cw = sCW + ci * 128;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t bits = 0;
+#pragma unroll 8
+                    for (int i = 0; i < 32; ++i) {
+                        const int4 w = cw[q4 * 32 + i];
+                        bits |= (visible(VisCode{w.x, w.y, w.z, w.w}, rc) ? 1u : 0u) << i;
+                    }
+                    vm[q4] = bits;
+                }
+            }
             ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], (u >> 1) & 1, wd, 2));
             if (!ok) break;
             tc_fence_after();
@@ -478,14 +511,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             }
             if (masked) {
-                const int4 *cw = reinterpret_cast<const int4 *>(sCW + ci * 128);
 #pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    if ((i & 7) == 0) asm volatile("" ::: "memory");
-                    const int4 w = cw[i];   // windows of columns 2i and 2i+1
-                    s[2 * i] = (w.x <= frame && frame < w.y) ? s[2 * i] : -INFINITY;
-                    s[2 * i + 1] = (w.z <= frame && frame < w.w) ? s[2 * i + 1] : -INFINITY;
-                }
+                for (int i = 0; i < 128; ++i) s[i] = ((vm[i >> 5] >> (i & 31)) & 1u) ? s[i] : -INFINITY;
             }
             // row maximum over the tile (four independent max3 chains)
             float mx[4];
@@ -796,9 +823,9 @@ static int enqueue_prepare(const nomas_kv_cache *c, const nomas_mask_layout &lay
 }
 
 // The attention kernel over a prepared workspace.
-static int enqueue_run(const nomas_kv_cache *c, const nomas_mask_layout &lay, int mode, const void *mask_buf,
-                       const void *q, int64_t tok_stride, int64_t head_stride, float softmax_scale, float *out,
-                       float *lse, void *workspace, cudaStream_t st) {
+static int enqueue_run(const nomas_kv_cache *c, const nomas_segment_text *seg, const nomas_mask_layout &lay, int mode,
+                       const void *mask_buf, const void *q, int64_t tok_stride, int64_t head_stride,
+                       float softmax_scale, float *out, float *lse, void *workspace, cudaStream_t st) {
     const auto &d = c->d;
     const int D = d.head_dim, H = d.heads;
     const int64_t Nq = lay.n_query, Lt = lay.text_tokens, Lh = lay.history_tokens, Lp = lay.head_tokens;
@@ -854,13 +881,15 @@ static int enqueue_run(const nomas_kv_cache *c, const nomas_mask_layout &lay, in
     p.ws_hdr = reinterpret_cast<const WsHeader *>(wsb);
     p.ws_expect = ws_header(c, lay);
     p.sparse = mode == NOMAS_MODE_SPARSE;
+    p.text_rows = mode == NOMAS_MODE_TEXT;
+    p.head_len = seg->head_len;
     p.n_pairs = (lay.n_qblocks + 1) / 2;
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.tok_stride = tok_stride;
     p.head_stride = head_stride;
     p.H = H;
     p.T = d.tokens_per_frame;
-    p.Nq = Nq;
+    p.Nq = mode == NOMAS_MODE_TEXT ? Lt : Nq;   // query rows of this call
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.out = out;
     p.lse = lse;
@@ -899,7 +928,7 @@ extern "C" int nomas_attn_run(const nomas_kv_cache *c, const nomas_segment_text 
                              workspace, lay);
     if (rc) return rc;
     if (bind_device(c)) return NOMAS_ECUDA;
-    return enqueue_run(c, lay, mode, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse, workspace,
+    return enqueue_run(c, seg, lay, mode, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse, workspace,
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -916,5 +945,6 @@ extern "C" int nomas_attn_fwd(const nomas_kv_cache *c, const nomas_segment_text 
     if (bind_device(c)) return NOMAS_ECUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if ((rc = enqueue_prepare(c, lay_p, kcur, vcur, ktxt, vtxt, tok_stride, head_stride, workspace, st))) return rc;
-    return enqueue_run(c, lay_r, mode, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse, workspace, st);
+    return enqueue_run(c, seg, lay_r, mode, mask_buf, q, tok_stride, head_stride, softmax_scale, out, lse, workspace,
+                       st);
 }

@@ -303,6 +303,9 @@ __device__ __forceinline__ uint4 bf16x8_to_f16(const uint4 &v) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// n / f.d for n < 2^31 (see make_fastdiv).
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) { return (__umulhi(n, f.m) + n) >> f.l; }
+
 // True when any of the 8 fp16 values is inf or NaN (exponent field all ones): the bf16 source was
 // non-finite or above the fp16 range (|x| >= 65520 rounds to inf).
 __device__ __forceinline__ bool f16x8_nonfinite(const uint4 &h) {

@@ -11,6 +11,7 @@
 //
 // Launches: dense  mask_prep, class_map, lists_dense
 //           sparse mask_prep, class_map, pool (block means), score, select_lists
+//           text   mask_prep, class_map_text, lists_dense (query blocks of the current text)
 #include <cmath>
 #include <mutex>
 
@@ -113,6 +114,40 @@ __global__ void class_map_kernel(MaskParams p) {
         cls = vis == total ? 1 : (vis == 0 ? 0 : 2);
     }
     reinterpret_cast<int8_t *>(p.buf + p.lay.off_class)[idx] = cls;
+}
+
+// Text query blocks (NOMAS_MODE_TEXT): one CTA of 128 threads per (query block, KV tile), a thread per
+// text row testing every key of the tile with the same visibility codes the attention kernel applies.
+__device__ __forceinline__ VisCode key_code(const MaskParams &p, const TileInfo &ti, int k) {
+    if (ti.kind == kKindCur) return key_video((int)((ti.start + k) / p.T));
+    if (ti.kind == kKindText && ti.start + k >= p.head_len) {
+        const int2 w = reinterpret_cast<const int2 *>(p.buf + p.lay.off_txtwin)[ti.start + k];
+        return key_tail(w.x, w.y);
+    }
+    return key_always();
+}
+
+__global__ void __launch_bounds__(128) class_map_text_kernel(MaskParams p) {
+    const int b = blockIdx.x / p.n_tiles, j = blockIdx.x % p.n_tiles;
+    const TileInfo ti = tile_info(p, j);
+    int8_t *cls = reinterpret_cast<int8_t *>(p.buf + p.lay.off_class) + (int64_t)b * p.n_tiles + j;
+    if (ti.kind == kKindHist || ti.kind == kKindPriorHead) {   // always visible
+        if (threadIdx.x == 0) *cls = 1;
+        return;
+    }
+    const int64_t i = (int64_t)b * kTile + threadIdx.x;        // text row
+    const bool row_ok = i < p.Lt;
+    VisCode rc = row_head();
+    if (row_ok && i >= p.head_len) {
+        const int2 w = reinterpret_cast<const int2 *>(p.buf + p.lay.off_txtwin)[i];
+        rc = row_tail(w.x, w.y);
+    }
+    int nvis = 0;
+    if (row_ok)
+        for (int k = 0; k < ti.count; ++k) nvis += visible(key_code(p, ti, k), rc) ? 1 : 0;
+    const bool any = __syncthreads_or(row_ok && nvis > 0);
+    const bool all = __syncthreads_and(!row_ok || nvis == ti.count);
+    if (threadIdx.x == 0) *cls = all ? 1 : (any ? 2 : 0);
 }
 
 __device__ __forceinline__ int mask_flag(int8_t cls, int32_t count) { return (cls == 2 || count < kTile); }
@@ -530,6 +565,11 @@ static int enqueue_mask(const MaskParams &p, float *qmean, float *kmean, cudaStr
     const bool sp = p.hdr.mode == NOMAS_MODE_SPARSE;
     if (sp && select_attr()) return NOMAS_ECUDA;
     mask_prep_kernel<<<nblk(p.Lt > 0 ? p.Lt : 1, 256), 256, 0, st>>>(p);
+    if (p.hdr.mode == NOMAS_MODE_TEXT) {
+        class_map_text_kernel<<<(unsigned)((int64_t)p.n_qb * p.n_tiles), 128, 0, st>>>(p);
+        lists_dense_kernel<<<nblk((int64_t)p.n_lists * 32, 128), 128, 0, st>>>(p);
+        return check_launch("mask_build kernels launch");
+    }
     class_map_kernel<<<nblk((int64_t)p.n_qb * p.n_tiles, 256), 256, 0, st>>>(p);
     if (!sp) {
         lists_dense_kernel<<<nblk((int64_t)p.n_lists * 32, 128), 128, 0, st>>>(p);

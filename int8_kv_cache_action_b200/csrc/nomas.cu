@@ -105,7 +105,7 @@ static int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int compute_mask_layout(const nomas_kv_cache *c, const nomas_segment_text *seg, int mode, float keep_frac,
                         nomas_mask_layout *o) {
     if (!c || !seg || !o) return NOMAS_EINVAL;
-    if (mode != NOMAS_MODE_DENSE && mode != NOMAS_MODE_SPARSE) return NOMAS_EINVAL;
+    if (mode != NOMAS_MODE_DENSE && mode != NOMAS_MODE_SPARSE && mode != NOMAS_MODE_TEXT) return NOMAS_EINVAL;
     if (seg->n_frames < 1 || seg->head_len < 0 || seg->n_tails < 0 || seg->n_tails > NOMAS_MAX_TAILS)
         return NOMAS_EINVAL;
     if (seg->n_tails > 0 && !seg->tails) return NOMAS_EINVAL;
@@ -126,7 +126,9 @@ int compute_mask_layout(const nomas_kv_cache *c, const nomas_segment_text *seg, 
     o->n_query = (int64_t)seg->n_frames * d.tokens_per_frame;
     o->text_tokens = lt;
     if (o->n_query > ((int64_t)1 << 30) || lt > ((int64_t)1 << 24)) return NOMAS_EUNSUPPORTED;
-    o->n_qblocks = (int32_t)cdiv(o->n_query, kTile);
+    if (mode == NOMAS_MODE_TEXT && lt == 0) return NOMAS_EINVAL;   // no text rows to attend from
+    // query blocks: 128 rows of the current video, or of the current text in text mode
+    o->n_qblocks = (int32_t)cdiv(mode == NOMAS_MODE_TEXT ? lt : o->n_query, kTile);
     o->n_hist_tiles = (int32_t)cdiv(hv.tokens, kTile);
     o->n_head_tiles = (int32_t)cdiv(c->head_used, kTile);
     o->n_cur_tiles = (int32_t)cdiv(o->n_query, kTile);

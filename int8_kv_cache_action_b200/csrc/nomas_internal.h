@@ -41,6 +41,57 @@ inline HistView hist_view(const nomas_kv_cache *c) {
     return v;
 }
 
+// Division by an invariant divisor d >= 1 for numerators below 2^31 (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994): l = ceil(log2 d),
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (umulhi(n, m) + n) >> l.
+struct FastDiv {
+    uint32_t d, m, l;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+    uint32_t l = 0;
+    while (l < 32 && ((uint64_t)1 << l) < d) ++l;
+    const uint64_t m = (((uint64_t)1 << 32) * (((uint64_t)1 << l) - d)) / d + 1;
+    return FastDiv{d, (uint32_t)m, l};
+}
+
+// Visibility codes (fluxbbs.com "架构": action tails visible only in their own segment and time
+// window; text query rows: see the reading in nomas.h).  A key and a query row each carry two
+// half-open frame intervals, x..y ("video" interval) and z..w ("tail" interval); the key is visible to
+// the row iff one of the pairs overlaps:  max(k.x, r.x) < min(k.y, r.y) || max(k.z, r.z) < min(k.w, r.w).
+//   key  always visible (history, earlier heads, current head): {-kBig, kBig, kNeg, kBig}
+//        current video frame t:                                 {t, t + 1, 0, 0}
+//        action tail with window [f0, f1):                      {0, 0, f0, f1}
+//        past the end of its tile:                              {0, 0, 0, 0}
+//   row  video frame t:                                         {-kBig, kBig, t, t + 1}
+//        description-head text row:                             {-kBig, kBig, 0, 0}
+//        text row of a tail with window [f0, f1):               {f0, f1, f0, f1}, or {f0, f1, kNeg, kNeg + 1}
+//                                                               when the window is empty
+constexpr int32_t kBig = 1 << 30;
+constexpr int32_t kNeg = -2147483647;   // below every frame and every -kBig
+
+struct VisCode {
+    int32_t x, y, z, w;
+};
+
+#if defined(__CUDACC__)
+#define NOMAS_HD __host__ __device__ __forceinline__
+#else
+#define NOMAS_HD inline
+#endif
+
+NOMAS_HD VisCode key_always() { return VisCode{-kBig, kBig, kNeg, kBig}; }
+NOMAS_HD VisCode key_video(int32_t t) { return VisCode{t, t + 1, 0, 0}; }
+NOMAS_HD VisCode key_tail(int32_t f0, int32_t f1) { return VisCode{0, 0, f0, f1}; }
+NOMAS_HD VisCode key_none() { return VisCode{0, 0, 0, 0}; }
+NOMAS_HD VisCode row_video(int32_t t) { return VisCode{-kBig, kBig, t, t + 1}; }
+NOMAS_HD VisCode row_head() { return VisCode{-kBig, kBig, 0, 0}; }
+NOMAS_HD VisCode row_tail(int32_t f0, int32_t f1) {
+    return f0 < f1 ? VisCode{f0, f1, f0, f1} : VisCode{f0, f1, kNeg, kNeg + 1};
+}
+NOMAS_HD bool visible(const VisCode &k, const VisCode &r) {
+    return (k.x > r.x ? k.x : r.x) < (k.y < r.y ? k.y : r.y) || (k.z > r.z ? k.z : r.z) < (k.w < r.w ? k.w : r.w);
+}
+
 // Per-CTA tile-list entry (int4): x = kind | flags, y = start in its source, z = valid keys, w = spare.
 enum TileKind : int { kKindHist = 0, kKindPriorHead = 1, kKindCur = 2, kKindText = 3 };
 constexpr int kUse0 = 1 << 2, kUse1 = 1 << 3, kMask0 = 1 << 4, kMask1 = 1 << 5;

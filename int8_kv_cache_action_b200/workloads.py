@@ -31,7 +31,7 @@ from typing import List, Optional, Tuple
 import torch
 
 # tensor ids used in the seed formula
-TID_Q, TID_KCUR, TID_VCUR, TID_KHIST, TID_VHIST, TID_KTXT, TID_VTXT, TID_OUTLIER, TID_KHEAD, TID_VHEAD = range(10)
+TID_Q, TID_KCUR, TID_VCUR, TID_KHIST, TID_VHIST, TID_KTXT, TID_VTXT, TID_OUTLIER, TID_KHEAD, TID_VHEAD, TID_QTXT = range(11)
 
 
 @dataclass(frozen=True)
@@ -196,6 +196,7 @@ class Inputs:
     k_txt: torch.Tensor        # [Lt, H, D]
     v_txt: torch.Tensor
     prior: List[SegmentKV] = field(default_factory=list)
+    q_txt: Optional[torch.Tensor] = None   # [Lt, H, D]: text query rows (the text stream of the joint attention)
 
 
 def make_inputs(cfg: Config, device="cpu", seed_offset: int = 0) -> Inputs:
@@ -213,6 +214,7 @@ def make_inputs(cfg: Config, device="cpu", seed_offset: int = 0) -> Inputs:
     vc = _randn_bf16((nq, H, D), s(TID_VCUR))
     kt = _randn_bf16((lt, H, D), s(TID_KTXT))
     vt = _randn_bf16((lt, H, D), s(TID_VTXT))
+    qt = _randn_bf16((lt, H, D), s(TID_QTXT))
     hist_tokens = sum(p.n_frames for p in cfg.prior) * T
     head_tokens = sum(p.head_len for p in cfg.prior)
     kh = _randn_bf16((hist_tokens, H, D), s(TID_KHIST))
@@ -222,6 +224,7 @@ def make_inputs(cfg: Config, device="cpu", seed_offset: int = 0) -> Inputs:
     if cfg.outliers:
         qch, kch = outlier_channels(cfg)
         q = _scale_outliers(q, qch)
+        qt = _scale_outliers(qt, qch)
         kc = _scale_outliers(kc, kch)
         kt = _scale_outliers(kt, kch)
         kh = _scale_outliers(kh, kch)
@@ -235,7 +238,8 @@ def make_inputs(cfg: Config, device="cpu", seed_offset: int = 0) -> Inputs:
                                vhd[h0:h0 + p.head_len].to(device) if p.head_len else None))
         t0 += n
         h0 += p.head_len
-    return Inputs(cfg, q.to(device), kc.to(device), vc.to(device), kt.to(device), vt.to(device), prior)
+    return Inputs(cfg, q.to(device), kc.to(device), vc.to(device), kt.to(device), vt.to(device), prior,
+                  qt.to(device))
 
 
 def attention_flops(cfg: Config, visible_keys_per_row_sum: int) -> float:

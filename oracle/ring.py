@@ -18,6 +18,17 @@ Readings adopted where the pages are silent:
     frame window (they are "always visible across segments");
   * action tails are never cached (they are visible only inside their own
     segment).
+
+Archive and selection (hyphentech.top config table: the GPU keeps at most 18
+history latent frames, earlier history is archived to CPU).  The pages say only
+that; the reading adopted:
+  * a frame that leaves the window can first be copied out of the cache as it
+    stands (its INT8 codes and scales), its "record";
+  * the retained history can be set to any list of at most W frames, each one
+    either retained now or given by its record, in the order the list gives
+    (that order is the history's age order for every later step);
+  * later appends add their frames at the new end and drop from the old end,
+    the same sliding window as before.
 """
 from __future__ import annotations
 
@@ -48,13 +59,13 @@ class OracleCache:
         self.frames_appended = 0
         self.head_used = 0
         self.segments = 0
+        self.retained = []            # global indices of the retained frames, age order
+        self.store = {}               # global index -> record (k8 [H,T,D], ks [H,T], v8, vs) of retained frames
 
     # -- state -----------------------------------------------------------------------------
     def retained_frames(self):
         """Global indices of the retained history frames, oldest first."""
-        g = self.frames_appended
-        lo = max(0, g - self.W) if self.W > 0 else 0
-        return list(range(lo, g))
+        return list(self.retained)
 
     def history_tokens(self) -> int:
         return len(self.retained_frames()) * self.T
@@ -82,6 +93,10 @@ class OracleCache:
             self.v8[:, dst] = qv.transpose(1, 0, 2)
             self.ks[:, dst] = sk.T
             self.vs[:, dst] = sv.T
+            self.store[g] = (qk.transpose(1, 0, 2).copy(), sk.T.copy(), qv.transpose(1, 0, 2).copy(), sv.T.copy())
+            self.retained.append(g)
+            if self.W > 0 and len(self.retained) > self.W:
+                self.store.pop(self.retained.pop(0))
         if head_len:
             qk, sk = quantize(head_k)
             qv, sv = quantize(head_v)
@@ -97,13 +112,36 @@ class OracleCache:
     # -- views -----------------------------------------------------------------------------
     def history(self):
         """Age-ordered retained history: (k8 [H,Lh,D], ks [H,Lh], v8, vs)."""
-        T = self.T
-        idx = []
-        for g in self.retained_frames():
-            s = g % self.C
-            idx.extend(range(s * T, (s + 1) * T))
-        idx = np.asarray(idx, dtype=np.int64)
-        return self.k8[:, idx], self.ks[:, idx], self.v8[:, idx], self.vs[:, idx]
+        if not self.retained:
+            return (np.zeros((self.H, 0, self.D), np.int8), np.zeros((self.H, 0), np.float32),
+                    np.zeros((self.H, 0, self.D), np.int8), np.zeros((self.H, 0), np.float32))
+        recs = [self.store[g] for g in self.retained]
+        return tuple(np.concatenate([r[i] for r in recs], axis=1) for i in range(4))
+
+    # -- archive and selection ---------------------------------------------------------------
+    def archive(self, g):
+        """Record of retained frame g: copies of (k8 [H,T,D], ks [H,T], v8, vs)."""
+        if g not in self.store:
+            raise ValueError(f"frame {g} is not retained")
+        return tuple(x.copy() for x in self.store[g])
+
+    def evicted_by(self, n_frames):
+        """Retained frames (oldest first) that an append of n_frames would drop from the window."""
+        if self.W == 0:
+            return []
+        drop = len(self.retained) + min(n_frames, self.W) - self.W
+        return self.retained[:max(0, drop)]
+
+    def select(self, frames, records):
+        """Make `frames` (global indices, age order, at most W, no repeats) the retained history; a frame
+        not retained now is taken from records[g]."""
+        frames = list(frames)
+        if self.W == 0 or len(frames) > self.W or len(set(frames)) != len(frames):
+            raise ValueError("selection needs a window, at most W frames, no repeats")
+        store = {}
+        for g in frames:
+            store[g] = self.store[g] if g in self.store else tuple(np.asarray(x).copy() for x in records[g])
+        self.store, self.retained = store, frames
 
     def prior_heads(self):
         u = self.head_used

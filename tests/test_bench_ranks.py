@@ -100,3 +100,17 @@ def test_reference_arm_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+@pytest.mark.parametrize("name", ["C1", "C2", "C4"])
+def test_text_row_key_count_matches_the_oracle_mask(name):
+    # the bench's algorithmic FLOPs for the text rows count exactly the keys the oracle's rule shows
+    import bench
+    from int8_kv_cache_action_b200.workloads import CONFIGS
+    from oracle import visibility as vis
+    cfg = CONFIGS[name]
+    frames = sum(p.n_frames for p in cfg.prior)
+    lh = (min(frames, cfg.window_frames) if cfg.window_frames else frames) * cfg.tokens_per_frame
+    lp = sum(p.head_len for p in cfg.prior)
+    m = vis.text_query_mask(lh, lp, cfg.n_query, cfg.tokens_per_frame, cfg.current)
+    assert bench.text_key_sum(cfg, lh, lp) == int(m.sum())

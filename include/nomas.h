@@ -140,6 +140,47 @@ int nomas_kv_append(nomas_kv_cache *cache, const void *k, const void *v, int64_t
                     int64_t head_stride, int32_t n_frames, const void *head_k, const void *head_v,
                     int32_t head_len, nomas_stream stream);
 
+/* ------------------------------------------------------------------------------------------------
+ * Archive of evicted frames and selection of the retained history (hyphentech.top, config table:
+ * in the single-GPU setting the GPU keeps at most 18 history latent frames and earlier history is
+ * archived to CPU).  The pages say no more; this library's reading: a frame about to leave the window
+ * can first be copied out as it stands (its INT8 codes and scales: a "record"), and the retained
+ * history can be set to any list of at most min(W, NOMAS_MAX_SELECT_FRAMES) frames, each retained now
+ * or given by its record, in the order listed -- which is then the history's age order for the mask,
+ * the sparse selection and the attention.  Later appends add frames at the new end and drop from the
+ * old end, the same window as before.  Without a selection nothing changes: frame g stays in ring
+ * slot g mod C.
+ * ------------------------------------------------------------------------------------------------ */
+#define NOMAS_MAX_SELECT_FRAMES 64
+
+/* Bytes of one frame record: K codes int8 [H][T][D], V codes int8 [H][T][D], K scales fp32 [H][T],
+ * V scales fp32 [H][T], in that order (0 on invalid dims). */
+size_t nomas_kv_frame_record_bytes(const nomas_cache_dims *dims);
+
+/* The retained frames (global indices, age order) into frames[0 .. *n), at most max_frames of them
+ * (NOMAS_ECAPACITY if more are retained). */
+int nomas_kv_retained(const nomas_kv_cache *cache, int64_t *frames, int32_t max_frames, int32_t *n);
+
+/* The retained frames (oldest first) that an append of n_frames would drop from the window, into
+ * frames[0 .. *n) (none without a window). */
+int nomas_kv_evicted_by(const nomas_kv_cache *cache, int32_t n_frames, int64_t *frames, int32_t max_frames,
+                        int32_t *n);
+
+/* Copy retained frame `frame` out of the cache into `record` (host memory of
+ * nomas_kv_frame_record_bytes bytes; pinned memory makes the copies asynchronous).  The record is
+ * complete once `stream` has reached this point.  Errors: NOMAS_EINVAL if the frame is not retained. */
+int nomas_kv_archive(const nomas_kv_cache *cache, int64_t frame, void *record, nomas_stream stream);
+
+/* Make frames[0 .. n) the retained history, in that age order.  A frame retained now keeps its data;
+ * any other frame is copied in from records[i] (a host record written by nomas_kv_archive; records[i]
+ * may be NULL for retained frames, and `records` may be NULL when every frame is retained).  Needs a
+ * window (W > 0) with W <= NOMAS_MAX_SELECT_FRAMES and n <= W, no repeated frame: NOMAS_EUNSUPPORTED /
+ * NOMAS_EINVAL before anything is enqueued.  Incoming frames go to slots no kept frame uses; if a copy
+ * fails (NOMAS_ECUDA) the retained history is undefined.  Records are read on `stream` (keep them alive
+ * and unchanged until it has passed this point). */
+int nomas_kv_select(nomas_kv_cache *cache, const int64_t *frames, int32_t n, const void *const *records,
+                    nomas_stream stream);
+
 #define NOMAS_MODE_DENSE 0
 #define NOMAS_MODE_SPARSE 1
 /* Text query rows of the current segment (the text stream of the double-stream joint attention,

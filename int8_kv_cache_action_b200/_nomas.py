@@ -23,12 +23,14 @@ NOMAS_MODE_DENSE, NOMAS_MODE_SPARSE, NOMAS_MODE_TEXT = 0, 1, 2
 NOMAS_MAX_TAILS = 64
 NOMAS_STATIC_POOL_FLOATS = 2 << 20
 NOMAS_MAX_SPARSE_CANDIDATES = 8192
+NOMAS_MAX_SELECT_FRAMES = 64
 
 EXPORTED = ["nomas_kv_cache_bytes", "nomas_kv_cache_init", "nomas_kv_cache_destroy", "nomas_kv_cache_state",
             "nomas_kv_append", "nomas_mask_layout_query", "nomas_mask_bytes", "nomas_mask_build",
             "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string",
             "nomas_last_error", "nomas_mask_build_static", "nomas_attn_workspace_bytes",
-            "nomas_set_wait_limit_ns", "nomas_attn_prepare", "nomas_attn_run"]
+            "nomas_set_wait_limit_ns", "nomas_attn_prepare", "nomas_attn_run", "nomas_kv_frame_record_bytes",
+            "nomas_kv_retained", "nomas_kv_evicted_by", "nomas_kv_archive", "nomas_kv_select"]
 
 
 class nomas_cache_dims(ctypes.Structure):
@@ -84,6 +86,11 @@ _sigs = {
                                           _p, _p]),
     "nomas_attn_run": (ctypes.c_int, [_p, ctypes.POINTER(nomas_segment_text), ctypes.c_int, _f32, _p, _p, _i64,
                                       _i64, _f32, _p, _p, _p, _p]),
+    "nomas_kv_frame_record_bytes": (_sz, [ctypes.POINTER(nomas_cache_dims)]),
+    "nomas_kv_retained": (ctypes.c_int, [_p, ctypes.POINTER(_i64), _i32, ctypes.POINTER(_i32)]),
+    "nomas_kv_evicted_by": (ctypes.c_int, [_p, _i32, ctypes.POINTER(_i64), _i32, ctypes.POINTER(_i32)]),
+    "nomas_kv_archive": (ctypes.c_int, [_p, _i64, _p, _p]),
+    "nomas_kv_select": (ctypes.c_int, [_p, ctypes.POINTER(_i64), _i32, ctypes.POINTER(_p), _p]),
     "nomas_kv_dequant": (ctypes.c_int, [_p, _p, _p, _p]),
     "nomas_device_status": (ctypes.c_int, [_p, _p]),
     "nomas_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -202,6 +209,40 @@ def nomas_attn_run(handle, seg, mode, keep_frac, mask_buf, q, tok_stride, head_s
                    workspace=0, stream=0):
     return lib.nomas_attn_run(handle, ctypes.byref(seg), mode, keep_frac, mask_buf, q, tok_stride, head_stride,
                               softmax_scale, out, lse or None, workspace or None, stream or None)
+
+
+def nomas_kv_frame_record_bytes(dims):
+    return lib.nomas_kv_frame_record_bytes(ctypes.byref(dims))
+
+
+def _frame_list(fn, handle, *args):
+    cap = 4096
+    buf = (_i64 * cap)()
+    n = _i32()
+    _check(fn(handle, *args, buf, cap, ctypes.byref(n)), fn.__name__)
+    return [int(buf[i]) for i in range(n.value)]
+
+
+def nomas_kv_retained(handle):
+    """Retained history frames (global indices), age order."""
+    return _frame_list(lib.nomas_kv_retained, handle)
+
+
+def nomas_kv_evicted_by(handle, n_frames):
+    """Retained frames an append of n_frames would drop, oldest first."""
+    return _frame_list(lib.nomas_kv_evicted_by, handle, n_frames)
+
+
+def nomas_kv_archive(handle, frame, record, stream=0):
+    return lib.nomas_kv_archive(handle, frame, record, stream or None)
+
+
+def nomas_kv_select(handle, frames, records=None, stream=0):
+    """frames: global indices in age order; records: host addresses (0 for retained frames) or None."""
+    n = len(frames)
+    fr = (_i64 * max(1, n))(*frames)
+    rec = None if records is None else (_p * max(1, n))(*[r or None for r in records])
+    return lib.nomas_kv_select(handle, fr, n, rec, stream or None)
 
 
 def nomas_kv_dequant(handle, k_out, v_out, stream=0):

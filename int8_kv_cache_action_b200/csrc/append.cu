@@ -10,6 +10,7 @@
 // and each lane stores 16 codes.  The ring rows of the video frames and the description-head rows
 // are two jobs of the same launch.
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 
@@ -129,7 +130,8 @@ struct AppendJob {
     int32_t head_mode;        // 0: ring rows slot(frame) * T + r; 1: rows dst_row0 + t
     int32_t first_slot;       // ring slot of the job's first frame (video)
     int32_t tok_outer;        // source maps are (D, heads, tokens) when set, else (D, tokens, heads)
-    int32_t _pad;
+    int32_t use_slots;        // video: frame f goes to slots[f] instead of first_slot + f (mod C)
+    int32_t slots[NOMAS_MAX_SELECT_FRAMES];
     int64_t dst_row0;
     int64_t rows_per_head;    // destination rows per head
     int8_t *k8, *v8;
@@ -235,8 +237,13 @@ __global__ void __launch_bounds__(kAppendThreads, 3)
                 // ring slot of the token's frame: first_slot + f < 2 C (f < min(frames, C) -- the job
                 // writes at most C frames), so one conditional subtraction replaces the modulo
                 const int f = (int)fdiv((uint32_t)t, a.div_frame);
-                int slot = J.first_slot + f;
-                if (slot >= Cf) slot -= Cf;
+                int slot;
+                if (J.use_slots) {
+                    slot = J.slots[f];
+                } else {
+                    slot = J.first_slot + f;
+                    if (slot >= Cf) slot -= Cf;
+                }
                 row = (int64_t)slot * T + (t - f * T);
             }
             const int64_t di = (int64_t)h * J.rows_per_head + row;
@@ -253,7 +260,8 @@ __global__ void __launch_bounds__(kAppendThreads, 3)
 struct DequantArgs {
     const int8_t *k8, *v8;
     const float *ks, *vs;
-    int64_t rows_per_head, ring_tokens, first_tok, n_tok;
+    HistView hv;
+    int64_t n_tok;
     int32_t heads;
     float *k_out, *v_out;
 };
@@ -268,8 +276,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
         const int64_t th = i / (D / CPT);
         const int h = (int)(th % a.heads);
         const int64_t t = th / a.heads;
-        const int64_t phys = (a.first_tok + t) % a.ring_tokens;
-        const int64_t r = (int64_t)h * a.rows_per_head + phys;
+        const int64_t r = (int64_t)h * a.hv.ring_tokens + hist_row(a.hv, t);
         const float sk = a.ks[r], sv = a.vs[r];
         const int8_t *pk = a.k8 + r * D + c0;
         const int8_t *pv = a.v8 + r * D + c0;
@@ -337,6 +344,34 @@ extern "C" int nomas_kv_append(nomas_kv_cache *c, const void *k, const void *v, 
     const int32_t keep = d.window_frames > 0 ? (n_frames < d.window_frames ? n_frames : d.window_frames) : n_frames;
     const int32_t f0 = n_frames - keep;
     const int64_t g0 = c->frames_appended + f0;
+    // Retained list after the append: the old frames that still fit the window, then the new ones.  A
+    // new frame g takes slot g mod C unless a kept frame holds it (possible only after a selection),
+    // in which case it takes the lowest free slot.
+    const int64_t Cf = d.capacity_frames;
+    size_t n_old = c->ret_frame.size();
+    if (d.window_frames > 0) {
+        const int64_t room = (int64_t)d.window_frames - keep;
+        if ((int64_t)n_old > room) n_old = (size_t)(room > 0 ? room : 0);
+    }
+    std::vector<int64_t> nf(c->ret_frame.end() - n_old, c->ret_frame.end());
+    std::vector<int32_t> ns(c->ret_slot.end() - n_old, c->ret_slot.end());
+    std::vector<char> used((size_t)Cf, 0);
+    for (int32_t sl : ns) used[sl] = 1;
+    std::vector<int32_t> new_slots((size_t)keep);
+    bool consecutive = true;
+    for (int32_t f = 0; f < keep; ++f) {
+        int32_t sl = (int32_t)((g0 + f) % Cf);
+        if (used[sl]) {
+            sl = 0;
+            while (used[sl]) ++sl;   // a free slot exists: kept + new frames <= W <= C
+        }
+        used[sl] = 1;
+        new_slots[f] = sl;
+        consecutive = consecutive && sl == (int32_t)((g0 + f) % Cf);
+        nf.push_back(g0 + f);
+        ns.push_back(sl);
+    }
+    if (!consecutive && keep > NOMAS_MAX_SELECT_FRAMES) return NOMAS_EUNSUPPORTED;   // not reachable
     const int64_t tc = d.head_dim == 128 ? AppendCfg<128>::TC : AppendCfg<64>::TC;
     if ((int64_t)keep * T >= ((int64_t)1 << 31) || head_len >= ((int64_t)1 << 31)) return NOMAS_EINVAL;
 
@@ -358,6 +393,8 @@ extern "C" int nomas_kv_append(nomas_kv_cache *c, const void *k, const void *v, 
     jv.n_chunks = (jv.n_tok + tc - 1) / tc * d.heads;
     jv.head_mode = 0;
     jv.first_slot = (int32_t)(g0 % d.capacity_frames);
+    jv.use_slots = consecutive ? 0 : 1;
+    for (int32_t f = 0; !consecutive && f < keep; ++f) jv.slots[f] = new_slots[f];
     jv.rows_per_head = (int64_t)d.capacity_frames * T;
     jv.k8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_K8]);
     jv.v8 = static_cast<int8_t *>(c->buf[NOMAS_BUF_V8]);
@@ -398,6 +435,9 @@ extern "C" int nomas_kv_append(nomas_kv_cache *c, const void *k, const void *v, 
     c->frames_appended += n_frames;
     c->head_used += head_len;
     c->segments += 1;
+    c->version += 1;
+    c->ret_frame.swap(nf);
+    c->ret_slot.swap(ns);
     return NOMAS_OK;
 }
 
@@ -412,9 +452,7 @@ extern "C" int nomas_kv_dequant(const nomas_kv_cache *c, float *k_out, float *v_
     a.v8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_V8]);
     a.ks = static_cast<const float *>(c->buf[NOMAS_BUF_KS]);
     a.vs = static_cast<const float *>(c->buf[NOMAS_BUF_VS]);
-    a.rows_per_head = hv.ring_tokens;
-    a.ring_tokens = hv.ring_tokens;
-    a.first_tok = hv.first_tok;
+    a.hv = hv;
     a.n_tok = hv.tokens;
     a.heads = c->d.heads;
     a.k_out = k_out;

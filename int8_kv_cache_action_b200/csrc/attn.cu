@@ -2,21 +2,20 @@
 // the visibility; "单卡 4090 怎么做到的" for INT8 storage and the sparse mode).
 //
 // One CTA = one head x one 128-row query block.  Roles (16 warps, one CTA per SM):
-//   warps 0-3   softmax of the even-numbered KV tiles of the CTA's list (TMEM lanes 0-127, one thread
-//               per query row over all 128 key columns)
-//   warps 4-7   softmax of the odd-numbered tiles.  The two warpgroups share O and one running
-//               offset per row: each passes the offset it settled on for its tile to the other
-//               through shared memory (a chain in tile order), so while one warpgroup computes its
-//               exponentials the other loads, scales and reduces the next tile
-//   warp 8      tcgen05.mma issuer (one thread) and TMEM owner
-//   warp 9      TMA producer (one thread)
-//   warps 10-11 column info: per-column key scale, value scale and visibility window of every
-//               tile (two columns per thread), one tile ahead, in a four-deep shared-memory ring
-// 384 threads at 168 registers each: a softmax thread holds a whole 128-column score row.
+//   warps 0-3   softmax over key columns 0-63 of every S tile (TMEM lanes 0-127, one thread per row)
+//   warps 4-7   softmax over key columns 64-127; the two halves of a row swap their maxima through
+//               shared memory, so both apply the same offset
+//   warps 8-11  column info: per-column key scale, value scale and visibility code of every tile,
+//               one tile ahead, in a four-deep shared-memory ring
+//   warp 12     tcgen05.mma issuer (one thread) and TMEM owner
+//   warp 13     TMA producer (one thread); warps 14-15 idle
+// The register file is split per SM sub-partition (one warp of each warpgroup on each), so the
+// kernel launches at 128 registers per thread and moves them with setmaxnreg: softmax 168 each,
+// column info 112, MMA / producer warpgroup 64 -- 2*168 + 112 + 64 = 512 = 4 x 128.
 //
-// TMEM (512 columns): Q (fp16 pairs) at [0, D/2), S double buffer at [128, 256) and [256, 384)
-// (tile u uses buffer u % 2, i.e. its softmax warpgroup's), O at [384, 384 + D).  P (fp16)
-// overwrites the first 32 columns of each 64-column half of its S buffer.
+// TMEM (512 columns): Q (fp16 pairs) at [0, D/2), S double buffer at [128, 256) and [256, 384),
+// O at [384, 384 + D).  P (fp16) overwrites the first 32 columns of each 64-column half of its S
+// buffer, so each softmax half writes only columns it has already read.
 //
 // Both products are TS MMAs (A from TMEM) with a K-major B in 128-byte-swizzled shared memory:
 //   S_b  = Q K_j^T     B = K_j    [128 keys][D]
@@ -52,8 +51,10 @@
 
 namespace nomas {
 
-constexpr int kAttnThreads = 384;
-constexpr int kWarpMma = 8, kWarpTma = 9, kWarpCi = 10;   // column info: warps 10 and 11
+constexpr int kAttnThreads = 512;
+constexpr int kWarpCi = 8, kWarpMma = 12, kWarpTma = 13;  // column info: warps 8-11
+constexpr int kRegSoftmax = 168, kRegLoader = 112, kRegMma = 64;
+static_assert(2 * kRegSoftmax + kRegLoader + kRegMma == 4 * 128, "register split must equal the launch total");
 constexpr int kNCI = 4;                     // column-info ring depth
 constexpr float kRescaleThreshold = 6.0f;   // log2 units: P <= 64
 constexpr uint32_t kTmQ = 0, kTmS = 128, kTmO = 384;
@@ -71,12 +72,11 @@ struct AttnCfg {
     static constexpr int OFF_CS = OFF_V + NV * SLOT;       // float [kNCI][128] key scale x log2 e
     static constexpr int OFF_CV = OFF_CS + kNCI * 512;     // float [kNCI][128] value scale
     static constexpr int OFF_CW = OFF_CV + kNCI * 512;     // int4  [kNCI][128] key visibility codes
-    static constexpr int OFF_DEC = OFF_CW + kNCI * 2048;   // float [128] running offset after the last tile
-    static constexpr int OFF_XM = OFF_DEC + 512;           // float [2 warpgroups][128] final offsets
-    static constexpr int OFF_XL = OFF_XM + 1024;           // float [2 warpgroups][128] row sums
+    static constexpr int OFF_XM = OFF_CW + kNCI * 2048;    // float [2 buffers][2 halves][128] maxima
+    static constexpr int OFF_XL = OFF_XM + 2048;           // float [2 halves][128] row sums
     static constexpr int OFF_BAR = OFF_XL + 1024;
     // q_ready; k_full, k_empty [NK]; v_full, v_empty [NV]; ci_full, ci_empty [kNCI];
-    // s_full, p_full, dec_full [2]; pv_done; o_final; xl_bar
+    // s_full, p_full, xm_bar [2]; pv_done; o_final; xl_bar
     static constexpr int NBAR = 1 + 2 * NK + 2 * NV + 2 * kNCI + 6 + 3;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
@@ -103,6 +103,7 @@ struct AttnParams {
     const __nv_bfloat16 *q;
     int64_t tok_stride, head_stride;
     int32_t H, T;
+    FastDiv divT;               // token -> frame (every token index here is below 2^31)
     int64_t Nq;
     float scale_log2;           // softmax_scale * log2(e)
     float *out;
@@ -117,10 +118,43 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// 2^x for x <= 6 on the FMA pipe (the MUFU unit's exponential throughput equals the tensor pipe's
+// rate per score at head_dim 128, so part of the exponentials are taken off it): x is clamped at -125,
+// n = rint(x) by the 1.5 * 2^23 add, f = x - n lies in [-1/2, 1/2], 2^f comes from a degree-3
+// polynomial fitted by weighted least squares to the relative error on Chebyshev nodes (maximum
+// relative error 7.5e-5, below fp16's half unit in the last place, 2^-12), and n is added to the
+// exponent field.
+__device__ __forceinline__ float2 exp2_poly(float2 x) {
+    x.x = fmaxf(x.x, -125.0f);
+    x.y = fmaxf(x.y, -125.0f);
+    const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
+    const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
+    const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
+    float2 q = __ffma2_rn(make_float2(0.055171605f, 0.055171605f), f, make_float2(0.24261111f, 0.24261111f));
+    q = __ffma2_rn(q, f, make_float2(0.69326097f, 0.69326097f));
+    q = __ffma2_rn(q, f, make_float2(0.99992806f, 0.99992806f));
+    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
+#ifndef NOMAS_POLY_PAIRS
+#define NOMAS_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = NOMAS_POLY_PAIRS;   // of every 16 column pairs, this many take exp2_poly
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
+}
+
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 __device__ __forceinline__ bool is_cached(int kind) { return kind == kKindHist || kind == kKindPriorHead; }
@@ -166,7 +200,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     float *sCS = reinterpret_cast<float *>(sm + C::OFF_CS);
     float *sCV = reinterpret_cast<float *>(sm + C::OFF_CV);
     int4 *sCW = reinterpret_cast<int4 *>(sm + C::OFF_CW);
-    float *sDec = reinterpret_cast<float *>(sm + C::OFF_DEC);
     float *sXM = reinterpret_cast<float *>(sm + C::OFF_XM);
     float *sXL = reinterpret_cast<float *>(sm + C::OFF_XL);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
@@ -174,8 +207,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint64_t *k_full = bars + 1, *k_empty = k_full + C::NK;
     uint64_t *v_full = k_empty + C::NK, *v_empty = v_full + C::NV;
     uint64_t *ci_full = v_empty + C::NV, *ci_empty = ci_full + kNCI;
-    uint64_t *s_full = ci_empty + kNCI, *p_full = s_full + 2, *dec_full = p_full + 2;
-    uint64_t *pv_done = dec_full + 2, *o_final = pv_done + 1, *xl_bar = o_final + 1;
+    uint64_t *s_full = ci_empty + kNCI, *p_full = s_full + 2, *xm_bar = p_full + 2;
+    uint64_t *pv_done = xm_bar + 2, *o_final = pv_done + 1, *xl_bar = o_final + 1;
     uint32_t *misc = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
 
@@ -193,11 +226,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const bool hdr_ok = hd->magic == p.expect.magic && hd->mode == p.expect.mode &&
                         hd->n_qblocks == p.expect.n_qblocks && hd->n_lists == p.expect.n_lists &&
                         hd->history_tokens == p.expect.history_tokens && hd->head_tokens == p.expect.head_tokens &&
-                        hd->frames_appended == p.expect.frames_appended && hd->n_query == p.expect.n_query &&
+                        hd->cache_version == p.expect.cache_version && hd->n_query == p.expect.n_query &&
                         hd->text_tokens == p.expect.text_tokens && hd->list_cap == p.expect.list_cap;
     const WsHeader *wh = p.ws_hdr;
     const bool ws_ok = wh->magic == p.ws_expect.magic && wh->head_dim == p.ws_expect.head_dim &&
-                       wh->frames_appended == p.ws_expect.frames_appended &&
+                       wh->cache_version == p.ws_expect.cache_version &&
                        wh->head_tokens == p.ws_expect.head_tokens &&
                        wh->history_tokens == p.ws_expect.history_tokens && wh->n_query == p.ws_expect.n_query &&
                        wh->text_tokens == p.ws_expect.text_tokens;
@@ -218,13 +251,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(&v_empty[i], 1);
         }
         for (int i = 0; i < kNCI; ++i) {
-            mbar_init(&ci_full[i], 2);      // the 2 column-info warps
-            mbar_init(&ci_empty[i], 4);     // the 4 warps of the tile's softmax warpgroup
+            mbar_init(&ci_full[i], 4);      // the 4 column-info warps
+            mbar_init(&ci_empty[i], 8);     // the 8 softmax warps
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 4);
-            mbar_init(&dec_full[b], 4);
+            mbar_init(&p_full[b], 8);
+            mbar_init(&xm_bar[b], 8);
         }
         mbar_init(pv_done, 1);
         mbar_init(o_final, 1);
@@ -244,12 +277,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     Watchdog wd{p.err, abort_flag, p.timeout_ns, 0};
     const int64_t qrow0 = (int64_t)qb * kTile;
 
-    if (warp >= kWarpCi) {
-        // ------------------------------------------------------------------ column-info warps
-        // Thread t writes columns t and t + 64 of every tile's entry in the ring; each warp arrives on
-        // ci_full once its columns are written.
+    if (warp >= kWarpCi && warp < kWarpCi + 4) {
+        // ------------------------------------------------------------------ column-info warpgroup
+        // Thread t writes column t of every tile's entry in the ring; each warp arrives on ci_full for
+        // its 32 columns.
+        setmaxnreg_dec<kRegLoader>();
         wd.where = 3;
-        const int t = threadIdx.x - 32 * kWarpCi;   // 0..63
+        const int t = threadIdx.x - 32 * kWarpCi;   // 0..127
         struct ColInfo {
             float ks, vs;   // raw key / value scale (cached tiles), 1 / 0 otherwise
             VisCode w;      // visibility code of the key
@@ -269,7 +303,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                         ci.w = key_tail(w.x, w.y);
                     }
                 } else if (kind == kKindCur) {
-                    ci.w = key_video((int)((start + col) / p.T));
+                    ci.w = key_video((int)fdiv((uint32_t)(start + col), p.divT));
                 } else {
                     ci.w = key_always();
                 }
@@ -288,31 +322,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         int u = 0;                          // index among this block's tiles
         int4 en;
         bool have = cursor.next(use_bit, en);
-        ColInfo nxt0, nxt1;
-        if (have) {
-            nxt0 = col_info(en, t);
-            nxt1 = col_info(en, t + 64);
-        }
+        ColInfo nxt0;
+        if (have) nxt0 = col_info(en, t);
         while (have) {
-            const ColInfo c0 = nxt0, c1 = nxt1;
+            const ColInfo c0 = nxt0;
             have = cursor.next(use_bit, en);
-            if (have) {
-                nxt0 = col_info(en, t);
-                nxt1 = col_info(en, t + 64);
-            }
+            if (have) nxt0 = col_info(en, t);
             const int ci = u % kNCI;
             if (!__all_sync(0xffffffffu, mbar_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, wd, 1))) break;
             sCS[ci * 128 + t] = p.scale_log2 * c0.ks;
             sCV[ci * 128 + t] = c0.vs;
             sCW[ci * 128 + t] = make_int4(c0.w.x, c0.w.y, c0.w.z, c0.w.w);
-            sCS[ci * 128 + t + 64] = p.scale_log2 * c1.ks;
-            sCV[ci * 128 + t + 64] = c1.vs;
-            sCW[ci * 128 + t + 64] = make_int4(c1.w.x, c1.w.y, c1.w.z, c1.w.w);
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_full[ci]);
             ++u;
         }
     } else if (warp >= kWarpMma) {
+        setmaxnreg_dec<kRegMma>();
         if (warp == kWarpMma && lane == 0) {
             // -------------------------------------------------------------- MMA issuer
             wd.where = 4;
@@ -408,29 +434,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else {
         // ------------------------------------------------------------------ softmax warpgroups
         // Waits are made warp-uniform (__all_sync) because tcgen05.ld/st are warp-collective.
-        const int wg = warp >> 2;           // tiles u with u % 2 == wg; S buffer wg
+        setmaxnreg_inc<kRegSoftmax>();
+        const int half = warp >> 2;         // key columns [64 * half, 64 * half + 64) of each tile
         const int g = warp & 3;             // TMEM lane group
-        wd.where = 1 + wg;
+        wd.where = 1 + half;
         const int r = g * 32 + lane;
         const int64_t row = qrow0 + r;
         const bool row_ok = row < p.Nq;
-        // the row's visibility code: a video frame, or a text row of the head or of a tail
-        VisCode rc;
-        if (!p.text_rows) {
-            rc = row_video((int)((row_ok ? row : 0) / p.T));
-        } else if (!row_ok || row < p.head_len) {
-            rc = row_head();
-        } else {
+        // the row's visibility code (a video frame, or a text row of the head or of a tail), needed only
+        // on masked tiles and so rebuilt there instead of held in registers
+        auto row_code = [&]() -> VisCode {
+            if (!p.text_rows) return row_video((int)fdiv(row_ok ? (uint32_t)row : 0u, p.divT));
+            if (!row_ok || row < p.head_len) return row_head();
             const int2 w = p.txtwin[row];
-            rc = row_tail(w.x, w.y);
-        }
+            return row_tail(w.x, w.y);
+        };
         const uint32_t lane_base = (uint32_t)(g * 32) << 16;
-        constexpr int DH = D / 2;           // head-dim elements of Q and O this warpgroup loads / stores
-        // Q row r, elements [wg * DH, wg * DH + DH) -> fp16 pairs in TMEM
+        constexpr int DH = D / 2;           // head-dim elements of Q and O handled by this half
+        // Q row r, elements [half * DH, half * DH + DH) -> fp16 pairs in TMEM
         {
             uint32_t qp[DH / 2];
             const uint4 *src = reinterpret_cast<const uint4 *>(p.q + (row_ok ? row : 0) * p.tok_stride +
-                                                               (int64_t)h * p.head_stride + wg * DH);
+                                                               (int64_t)h * p.head_stride + half * DH);
             bool bad = false;
 #pragma unroll
             for (int i = 0; i < DH / 8; ++i) {
@@ -442,7 +467,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 qp[4 * i + 3] = v.w;
             }
             if (bad) set_device_error(p.err, NOMAS_ERANGE, 33);   // q outside the fp16 range
-            const uint32_t tq = tmem + lane_base + kTmQ + (uint32_t)(wg * DH / 2);
+            const uint32_t tq = tmem + lane_base + kTmQ + (uint32_t)(half * DH / 2);
             if constexpr (DH / 2 == 32) {
                 tmem_st32(tq, qp);
             } else {
@@ -453,53 +478,46 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(q_ready);
         }
-        // Running offset (log2 units) of the row: the chain of decisions in tile order.  Tile u's
-        // warpgroup starts from the offset settled after tile u - 1 (written by the other warpgroup),
-        // raises it only when the tile's maximum exceeds it by more than kRescaleThreshold (then O is
-        // rescaled once PV of tile u - 1 has completed), and passes it on.  This warpgroup's partial
-        // row sum l is kept relative to my_m, the offset of its own latest tile.
-        float my_m = -INFINITY;
+        float m_used = -INFINITY;
         float l = 0.0f;
         int u = 0;
         bool ok = true;
         ListCursor cursor(list, n_tiles);
         int4 e;
         while (cursor.next(use_bit, e)) {
-            if ((u & 1) != wg) {
-                ++u;
-                continue;
-            }
             const int ci = u % kNCI;
+            const int b = u & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(&ci_full[ci], (u / kNCI) & 1, wd, 1));
             if (!ok) break;
             const bool masked = (e.x & mask_bit) != 0;
             const bool cached = is_cached(e.x & 3);
-            // visibility of the tile's keys to this row, as 128 bits, taken before the scores are loaded
-            uint32_t vm[4] = {~0u, ~0u, ~0u, ~0u};
+            // visibility of this half's 64 keys to the row, taken before the scores are loaded
+            uint32_t vm[2] = {~0u, ~0u};
             if (masked) {
-                const int4 *cw = sCW + ci * 128;
+                const VisCode rc = row_code();
+                const int4 *cw = sCW + ci * 128 + half * 64;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
+                for (int q2 = 0; q2 < 2; ++q2) {
                     uint32_t bits = 0;
 #pragma unroll 8
                     for (int i = 0; i < 32; ++i) {
-                        const int4 w = cw[q4 * 32 + i];
+                        const int4 w = cw[q2 * 32 + i];
                         bits |= (visible(VisCode{w.x, w.y, w.z, w.w}, rc) ? 1u : 0u) << i;
                     }
-                    vm[q4] = bits;
+                    vm[q2] = bits;
                 }
             }
-            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[wg], (u >> 1) & 1, wd, 2));
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (u >> 1) & 1, wd, 2));
             if (!ok) break;
             tc_fence_after();
-            const uint32_t tS = tmem + lane_base + kTmS + (uint32_t)(wg * 128);
-            float s[128];
-            tmem_ld128f_sync(tS, s);
+            const uint32_t tS = tmem + lane_base + kTmS + (uint32_t)(b * 128 + half * 64);
+            float s[64];
+            tmem_ld64f_sync(tS, s);
             // cached keys: apply the per-key scale (which carries softmax scale * log2 e) to the score
             if (cached) {
-                const float4 *cs4 = reinterpret_cast<const float4 *>(sCS + ci * 128);
+                const float4 *cs4 = reinterpret_cast<const float4 *>(sCS + ci * 128 + half * 64);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     if ((i & 7) == 0) asm volatile("" ::: "memory");   // bound how far loads are hoisted
                     const float4 v = cs4[i];
                     const float2 a = __fmul2_rn(make_float2(s[4 * i], s[4 * i + 1]), make_float2(v.x, v.y));
@@ -512,73 +530,62 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             if (masked) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i) s[i] = ((vm[i >> 5] >> (i & 31)) & 1u) ? s[i] : -INFINITY;
+                for (int i = 0; i < 64; ++i) s[i] = ((vm[i >> 5] >> (i & 31)) & 1u) ? s[i] : -INFINITY;
             }
-            // row maximum over the tile (four independent max3 chains)
-            float mx[4];
+            // row maximum over this half (two independent max3 chains), then swapped with the other half
+            float m0 = max3(s[0], s[1], s[2]), m1 = max3(s[32], s[33], s[34]);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mx[k] = max3(s[32 * k], s[32 * k + 1], s[32 * k + 2]);
-#pragma unroll
-            for (int c = 3; c < 31; c += 2)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) mx[k] = max3(mx[k], s[32 * k + c], s[32 * k + c + 1]);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) mx[k] = fmaxf(mx[k], s[32 * k + 31]);
-            const float pm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-            // log2 domain: cached scores are already scaled, bf16-source scores take the uniform scale
-            // (a positive factor commutes with the maximum exactly)
-            const float cmul = cached ? 1.0f : p.scale_log2;
-            const float mt = pm * cmul;
-            float m_prev = -INFINITY;
-            if (u > 0) {   // the offset after tile u - 1, settled by the other warpgroup
-                ok = __all_sync(0xffffffffu, mbar_wait(&dec_full[wg ^ 1], ((u - 1) >> 1) & 1, wd, 3));
-                if (!ok) break;
-                m_prev = sDec[r];
+            for (int c = 3; c < 31; c += 2) {
+                m0 = max3(m0, s[c], s[c + 1]);
+                m1 = max3(m1, s[32 + c], s[33 + c]);
             }
-            const float m_new = fmaxf(m_prev, mt);
-            const bool grow = m_new > m_prev + kRescaleThreshold;   // false while both are -inf
-            const float m_cur = grow ? m_new : m_prev;
-            sDec[r] = m_cur;
+            const float pm = fmaxf(fmaxf(m0, s[31]), fmaxf(m1, s[63]));
+            sXM[(b * 2 + half) * 128 + r] = pm;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&dec_full[wg]);
-            if (m_cur != my_m) {   // this warpgroup's partial sum moves to the new offset
-                l = (my_m == -INFINITY) ? 0.0f : l * ex2(my_m - m_cur);
-                my_m = m_cur;
-            }
-            const bool need_o = grow && m_prev != -INFINITY;
-            const float f = need_o ? ex2(m_prev - m_cur) : 1.0f;
-            const float off = (m_cur == -INFINITY) ? 0.0f : m_cur;
+            if (lane == 0) mbar_arrive(&xm_bar[b]);
+            ok = __all_sync(0xffffffffu, mbar_wait(&xm_bar[b], (u >> 1) & 1, wd, 3));
+            if (!ok) break;
+            const float po = sXM[(b * 2 + (half ^ 1)) * 128 + r];
+            // log2 domain: cached scores are already scaled, bf16-source scores take the uniform scale
+            // (a positive factor commutes with the maximum exactly); both halves compute the same values
+            const float cmul = cached ? 1.0f : p.scale_log2;
+            const float mt = fmaxf(pm, po) * cmul;
+            const float m_new = fmaxf(m_used, mt);
+            const bool grow = m_new > m_used + kRescaleThreshold;   // false while both are -inf
+            const bool need_o = grow && m_used != -INFINITY;
+            const float f = need_o ? ex2(m_used - m_new) : 1.0f;
+            if (grow) m_used = m_new;
+            const float off = (m_used == -INFINITY) ? 0.0f : m_used;
             const float2 cm2 = make_float2(cmul, cmul);
             const float2 no2 = make_float2(-off, -off);
             float2 acc[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-            const float2 *cv2 = reinterpret_cast<const float2 *>(sCV + ci * 128);
+            const float2 *cv2 = reinterpret_cast<const float2 *>(sCV + ci * 128 + half * 64);
 #pragma unroll
-            for (int qt = 0; qt < 4; ++qt) {   // keys 32 qt .. 32 qt + 31 -> P columns (qt / 2) * 64 + (qt % 2) * 16
+            for (int qt = 0; qt < 2; ++qt) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const float2 a = __ffma2_rn(make_float2(s[qt * 32 + c], s[qt * 32 + c + 1]), cm2, no2);
-                    float2 pe = make_float2(ex2(a.x), ex2(a.y));
+                    float2 pe = (c / 2) < kPolyPairs ? exp2_poly(a) : make_float2(ex2(a.x), ex2(a.y));
                     acc[(c >> 1) & 1] = __fadd2_rn(acc[(c >> 1) & 1], pe);
                     // cached values enter the tensor core as exact codes: P carries their scale
                     if (cached) pe = __fmul2_rn(pe, cv2[(qt * 32 + c) / 2]);
                     pk[c / 2] = f16x2_of(pe.x, pe.y);
                 }
-                tmem_st16(tS + (uint32_t)((qt >> 1) * 64 + (qt & 1) * 16), pk);
+                tmem_st16(tS + qt * 16, pk);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_empty[ci]);   // column info no longer needed
-            l += (acc[0].x + acc[1].x) + (acc[0].y + acc[1].y);   // l is already relative to m_cur
-            // rescale O (rare: only when some row's maximum grew past the threshold) once PV of tile
-            // u - 1 is complete; S_u's completion already implies PV_{u-2}'s, and PV_u waits for this
-            // warpgroup's P
+            l = l * f + ((acc[0].x + acc[1].x) + (acc[0].y + acc[1].y));
+            // rescale this half of O (rare: only when some row's maximum grew past the threshold) once
+            // PV of the previous tile is complete; S_u's completion already implies PV_{u-2}'s
             if (__any_sync(0xffffffffu, need_o)) {
                 ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (u - 1) & 1, wd, 4));
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t tO = tmem + lane_base + kTmO;
+                const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(half * DH);
 #pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                for (int c0 = 0; c0 < DH; c0 += 32) {
                     uint32_t rr[32];
                     tmem_ld32_sync(tO + c0, rr);
 #pragma unroll
@@ -589,29 +596,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[wg]);
+            if (lane == 0) mbar_arrive(&p_full[b]);
             ++u;
         }
-        // epilogue: combine the two warpgroups' row sums at the final offset (the later of the two
-        // warpgroups' offsets: the chain never lowers it), then O / l over this warpgroup's columns
+        // epilogue: the two halves' row sums, then O / l over this half's columns
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_final, 0, wd, 5));
         if (ok) {
-            sXL[wg * 128 + r] = l;
-            sXM[wg * 128 + r] = my_m;
+            sXL[half * 128 + r] = l;
             __syncwarp();
             if (lane == 0) mbar_arrive(xl_bar);
             ok = __all_sync(0xffffffffu, mbar_wait(xl_bar, 0, wd, 6));
         }
         if (ok) {
             tc_fence_after();
-            const float ma = sXM[r], mb = sXM[128 + r];
-            const float mf = fmaxf(ma, mb);
-            const float la = ma == -INFINITY ? 0.0f : sXL[r] * ex2(ma - mf);
-            const float lb = mb == -INFINITY ? 0.0f : sXL[128 + r] * ex2(mb - mf);
-            const float lt = la + lb;
+            const float lt = l + sXL[(half ^ 1) * 128 + r];
             const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-            float *dst = p.out + (row * p.H + h) * (int64_t)D + wg * DH;
-            const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(wg * DH);
+            float *dst = p.out + (row * p.H + h) * (int64_t)D + half * DH;
+            const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(half * DH);
 #pragma unroll 1
             for (int c0 = 0; c0 < DH; c0 += 32) {
                 uint32_t rr[32];
@@ -626,8 +627,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     }
                 }
             }
-            if (p.lse && row_ok && wg == 0)
-                p.lse[(int64_t)h * p.Nq + row] = (mf + log2f(lt)) * 0.69314718055994530942f;
+            if (p.lse && row_ok && half == 0)
+                p.lse[(int64_t)h * p.Nq + row] = (m_used + log2f(lt)) * 0.69314718055994530942f;
         }
     }
 
@@ -697,7 +698,7 @@ static WsHeader ws_header(const nomas_kv_cache *c, const nomas_mask_layout &lay)
     WsHeader h{};
     h.magic = kWsMagic;
     h.head_dim = c->d.head_dim;
-    h.frames_appended = c->frames_appended;
+    h.cache_version = c->version;
     h.head_tokens = lay.head_tokens;
     h.history_tokens = lay.history_tokens;
     h.n_query = lay.n_query;
@@ -808,8 +809,7 @@ static int enqueue_prepare(const nomas_kv_cache *c, const nomas_mask_layout &lay
         hp.vpt = reinterpret_cast<__half *>(wsb + ws.vpt);
         hp.ksl = reinterpret_cast<float *>(wsb + ws.ksl);
         hp.vsl = reinterpret_cast<float *>(wsb + ws.vsl);
-        hp.ring_tokens = hv.ring_tokens;
-        hp.first_tok = hv.first_tok;
+        hp.hv = hv;
         hp.Lh = Lh;
         hp.lhp = lhp;
         hp.Lp = Lp;
@@ -873,7 +873,7 @@ static int enqueue_run(const nomas_kv_cache *c, const nomas_segment_text *seg, c
     p.expect.n_lists = lay.n_lists;
     p.expect.history_tokens = lay.history_tokens;
     p.expect.head_tokens = lay.head_tokens;
-    p.expect.frames_appended = c->frames_appended;
+    p.expect.cache_version = c->version;
     p.expect.n_query = lay.n_query;
     p.expect.text_tokens = lay.text_tokens;
     p.expect.list_cap = lay.list_cap;
@@ -889,6 +889,7 @@ static int enqueue_run(const nomas_kv_cache *c, const nomas_segment_text *seg, c
     p.head_stride = head_stride;
     p.H = H;
     p.T = d.tokens_per_frame;
+    p.divT = make_fastdiv((uint32_t)d.tokens_per_frame);
     p.Nq = mode == NOMAS_MODE_TEXT ? Lt : Nq;   // query rows of this call
     p.scale_log2 = softmax_scale * 1.4426950408889634f;
     p.out = out;

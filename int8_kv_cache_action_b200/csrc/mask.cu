@@ -35,7 +35,7 @@ struct MaskParams {
     int64_t tok_stride, head_stride;
     const int8_t *k8;
     const float *ks;
-    int64_t ring_tokens, first_tok;
+    HistView hv;              // ring rows of the retained history in age order
 };
 
 struct TileInfo {
@@ -197,7 +197,7 @@ constexpr int kPoolAhead = 8;   // rows loaded before they are added (independen
 // the block's valid rows in ascending order from +0 (history keys as fp32(code) * scale, one rounding),
 // then divided once by the number of valid rows.  Loads run kPoolAhead rows ahead of the additions,
 // which keep the row order.
-template <int D>
+template <int D, bool CONTIG>
 __global__ void __launch_bounds__(256) pool_kernel(MaskParams p, float *qmean, float *kmean) {
     constexpr int LPU = D / 8;             // lanes per unit
     constexpr int UPW = 32 / LPU;          // units per warp
@@ -274,10 +274,21 @@ __global__ void __launch_bounds__(256) pool_kernel(MaskParams p, float *qmean, f
                 src += ts;
             }
         } else {
-            // ring rows of the block in age order; the physical row advances with one wrap check
-            int64_t phys = (p.first_tok + r0) % p.ring_tokens;
-            const int8_t *kb = p.k8 + h * p.ring_tokens * D + sub * 8;
-            const float *sb = p.ks + h * p.ring_tokens;
+            // ring rows of the block in age order; in a contiguous layout the physical row advances with
+            // one wrap check, otherwise every row is looked up in the history map
+            const int64_t ring = p.hv.ring_tokens;
+            int64_t phys = hist_row(p.hv, r0);
+            int64_t a = r0;
+            auto next_row = [&]() {
+                ++a;
+                if (CONTIG) {
+                    if (++phys == ring) phys = 0;
+                } else if (a < r0 + nv) {
+                    phys = hist_row(p.hv, a);
+                }
+            };
+            const int8_t *kb = p.k8 + h * ring * D + sub * 8;
+            const float *sb = p.ks + h * ring;
             auto add_row = [&](const uint2 &r, float sc) {
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
@@ -293,14 +304,14 @@ __global__ void __launch_bounds__(256) pool_kernel(MaskParams p, float *qmean, f
                 for (int k = 0; k < kPoolAhead; ++k) {
                     raw[k] = __ldg(reinterpret_cast<const uint2 *>(kb + phys * D));
                     sc[k] = __ldg(sb + phys);
-                    if (++phys == p.ring_tokens) phys = 0;
+                    next_row();
                 }
 #pragma unroll
                 for (int k = 0; k < kPoolAhead; ++k) add_row(raw[k], sc[k]);
             }
             for (; i < nv; ++i) {
                 add_row(__ldg(reinterpret_cast<const uint2 *>(kb + phys * D)), __ldg(sb + phys));
-                if (++phys == p.ring_tokens) phys = 0;
+                next_row();
             }
         }
         const float n = (float)nv;
@@ -508,7 +519,7 @@ static int prepare_mask(const nomas_kv_cache *c, const nomas_segment_text *seg, 
     p.hdr.n_lists = lay.n_lists;
     p.hdr.history_tokens = lay.history_tokens;
     p.hdr.head_tokens = lay.head_tokens;
-    p.hdr.frames_appended = c->frames_appended;
+    p.hdr.cache_version = c->version;
     p.hdr.n_query = lay.n_query;
     p.hdr.text_tokens = lay.text_tokens;
     p.hdr.list_cap = lay.list_cap;
@@ -542,8 +553,7 @@ static int prepare_mask(const nomas_kv_cache *c, const nomas_segment_text *seg, 
     p.head_stride = head_stride;
     p.k8 = static_cast<const int8_t *>(c->buf[NOMAS_BUF_K8]);
     p.ks = static_cast<const float *>(c->buf[NOMAS_BUF_KS]);
-    p.ring_tokens = hv.ring_tokens;
-    p.first_tok = hv.first_tok;
+    p.hv = hv;
     return NOMAS_OK;
 }
 
@@ -577,8 +587,14 @@ static int enqueue_mask(const MaskParams &p, float *qmean, float *kmean, cudaStr
         const int64_t units = (int64_t)p.H * (p.n_qb + p.n_cand);   // D/8 lanes each
         int64_t blocks = nblk(units * (p.D / 8), 256);
         if (blocks > 148 * 8) blocks = 148 * 8;
-        if (p.D == 128) pool_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(p, qmean, kmean);
-        else pool_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(p, qmean, kmean);
+        const bool contig = p.hv.contiguous != 0;
+        if (p.D == 128) {
+            if (contig) pool_kernel<128, true><<<(unsigned)blocks, 256, 0, st>>>(p, qmean, kmean);
+            else pool_kernel<128, false><<<(unsigned)blocks, 256, 0, st>>>(p, qmean, kmean);
+        } else {
+            if (contig) pool_kernel<64, true><<<(unsigned)blocks, 256, 0, st>>>(p, qmean, kmean);
+            else pool_kernel<64, false><<<(unsigned)blocks, 256, 0, st>>>(p, qmean, kmean);
+        }
         const dim3 sg(nblk(p.n_cand, kScoreTile) * nblk(p.n_qb, kScoreTile), (unsigned)p.H);
         score_kernel<<<sg, 256, 0, st>>>(p, qmean, kmean);
         const int npow2 = pow2_at_least(p.n_cand);

@@ -205,6 +205,7 @@ extern "C" int nomas_kv_cache_init(nomas_kv_cache **out, const nomas_cache_dims 
     c->d = *d;
     for (int i = 0; i < NOMAS_NBUF; ++i) c->buf[i] = bufs[i];
     c->frames_appended = 0;
+    c->version = 0;
     c->head_used = 0;
     c->segments = 0;
     c->device = attr.device;
@@ -226,8 +227,8 @@ extern "C" int nomas_kv_cache_state(const nomas_kv_cache *c, nomas_cache_state *
     const HistView hv = hist_view(c);
     std::memset(o, 0, sizeof(*o));
     o->frames_appended = c->frames_appended;
-    o->retained_frames = (int32_t)(hv.tokens / c->d.tokens_per_frame);
-    o->first_slot = (int32_t)(hv.first_tok / c->d.tokens_per_frame);
+    o->retained_frames = hv.n_frames;
+    o->first_slot = hv.n_frames ? c->ret_slot[0] : 0;
     o->history_tokens = hv.tokens;
     o->head_tokens = c->head_used;
     o->segments = c->segments;

@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda.h>
+#include <vector>
 
 #include "nomas.h"
 
@@ -12,8 +13,11 @@ struct nomas_kv_cache {
     void *buf[NOMAS_NBUF];
     int64_t frames_appended;
     int64_t head_used;
+    int64_t version;                   // changes with every append and selection (checked by the kernels)
     int32_t segments;
-    int32_t device;          // CUDA device owning the buffers; made current on every call
+    int32_t device;                    // CUDA device owning the buffers; made current on every call
+    std::vector<int64_t> ret_frame;    // retained history frames (global index), age order
+    std::vector<int32_t> ret_slot;     // their ring slots
 };
 
 namespace nomas {
@@ -22,23 +26,49 @@ constexpr int kTile = 128;                 // query block and KV tile size
 constexpr uint32_t kMaskMagic = 0x4E4D534Bu;
 constexpr int32_t kAlwaysHi = 1 << 30;      // 'visible to every frame' upper window bound
 
-// Ring view of the retained history (host-computed, passed by value to kernels).
+// Ring view of the retained history in age order (host-computed, passed by value to kernels).  Without
+// a selection the retained frames sit in consecutive slots (frame g in slot g mod C); after
+// nomas_kv_select they may sit anywhere, and the slot of every frame is listed.
 struct HistView {
     int64_t ring_tokens;     // C * T
-    int64_t first_tok;       // physical token of the oldest retained token
+    int64_t first_tok;       // contiguous: physical token of the oldest retained token
     int64_t tokens;          // retained history tokens
+    int32_t T;
+    int32_t contiguous;      // 1: frame i of the history is in slot (first slot + i) mod C
+    int32_t n_frames;
+    int32_t slots[NOMAS_MAX_SELECT_FRAMES];   // otherwise: slot of history frame i (n_frames <= the max)
 };
 
 inline HistView hist_view(const nomas_kv_cache *c) {
     const auto &d = c->d;
-    int64_t g = c->frames_appended;
-    int64_t ret = d.window_frames > 0 ? (g < d.window_frames ? g : d.window_frames) : g;
-    int64_t first_frame = g - ret;
-    HistView v;
+    HistView v{};
+    const int n = (int)c->ret_slot.size();
     v.ring_tokens = (int64_t)d.capacity_frames * d.tokens_per_frame;
-    v.first_tok = (first_frame % d.capacity_frames) * d.tokens_per_frame;
-    v.tokens = ret * d.tokens_per_frame;
+    v.tokens = (int64_t)n * d.tokens_per_frame;
+    v.T = d.tokens_per_frame;
+    v.n_frames = n;
+    v.contiguous = 1;
+    for (int i = 1; i < n; ++i)
+        if (c->ret_slot[i] != (c->ret_slot[0] + i) % d.capacity_frames) v.contiguous = 0;
+    v.first_tok = n ? (int64_t)c->ret_slot[0] * d.tokens_per_frame : 0;
+    if (!v.contiguous)
+        for (int i = 0; i < n && i < NOMAS_MAX_SELECT_FRAMES; ++i) v.slots[i] = c->ret_slot[i];
     return v;
+}
+
+// Physical ring row (within one head) of history token a (age order).
+#if defined(__CUDACC__)
+__host__ __device__ __forceinline__
+#else
+inline
+#endif
+int64_t hist_row(const HistView &v, int64_t a) {
+    if (v.contiguous) {
+        const int64_t p = v.first_tok + a;   // first_tok < C T and a < C T
+        return p >= v.ring_tokens ? p - v.ring_tokens : p;
+    }
+    const int64_t f = a / v.T;
+    return (int64_t)v.slots[f] * v.T + (a - f * v.T);
 }
 
 // Division by an invariant divisor d >= 1 for numerators below 2^31 (Granlund and Montgomery,
@@ -104,7 +134,7 @@ struct MaskHeader {
     int32_t n_lists;
     int64_t history_tokens;
     int64_t head_tokens;
-    int64_t frames_appended;
+    int64_t cache_version;
     int64_t n_query;
     int64_t text_tokens;
     int32_t list_cap;
@@ -117,7 +147,7 @@ constexpr uint32_t kWsMagic = 0x4E4D5753u;
 struct WsHeader {
     uint32_t magic;
     int32_t head_dim;
-    int64_t frames_appended;
+    int64_t cache_version;
     int64_t head_tokens;
     int64_t history_tokens;
     int64_t n_query;

@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
     const int8_t *ksrc = heads ? P.hk8 : P.k8, *vsrc = heads ? P.hv8 : P.v8;
     __half *kdst = heads ? P.kp : P.kh;
     auto src_row = [&](int64_t a) -> int64_t {
-        return heads ? (int64_t)h * P.head_rows + a : (int64_t)h * P.ring_tokens + (P.first_tok + a) % P.ring_tokens;
+        return heads ? (int64_t)h * P.head_rows + a : (int64_t)h * P.hv.ring_tokens + hist_row(P.hv, a);
     };
     for (int i = threadIdx.x; i < 64 * cpr; i += blockDim.x) {
         const int r = i / cpr, c = i % cpr;

@@ -45,7 +45,8 @@ struct HistPrep {
     __half *kh, *vht, *kp, *vpt;
     float *ksl, *vsl;
     const float *hks, *hvs;   // description-head scales (checked only)
-    int64_t ring_tokens, first_tok, Lh, lhp, Lp, lpp, head_rows;
+    HistView hv;              // ring rows of the retained history in age order
+    int64_t Lh, lhp, Lp, lpp, head_rows;
     int32_t H, D;
     int *err;                 // device error word: NOMAS_ERANGE for a value scale above kMaxValueScale
 };

@@ -55,10 +55,12 @@ class KVCache:
         return cls(cfg.heads, cfg.head_dim, cfg.tokens_per_frame, cfg.window_frames, cfg.capacity_frames,
                    cfg.head_store_tokens, device)
 
-    def __del__(self):
+    def __del__(self, _destroy=N.nomas_kv_cache_destroy):
+        # the destroy function is bound at definition time: module globals may already be gone when
+        # the interpreter shuts down
         h = getattr(self, "handle", None)
         if h:
-            N.nomas_kv_cache_destroy(h)
+            _destroy(h)
             self.handle = None
 
     # ---- raw buffer views (for tests and diagnostics) -----------------------------------------
@@ -156,6 +158,29 @@ class KVCache:
                               _stream_handle(stream))
         N._check(rc, "nomas_attn_fwd")
         return out, lse
+
+    # ---- archive of evicted frames and selection of the retained history ------------------------
+    def record_bytes(self) -> int:
+        return N.nomas_kv_frame_record_bytes(self.dims)
+
+    def retained(self):
+        return N.nomas_kv_retained(self.handle)
+
+    def evicted_by(self, n_frames: int):
+        return N.nomas_kv_evicted_by(self.handle, n_frames)
+
+    def archive(self, frame: int, record: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Copy retained `frame` into a host record (a pinned uint8 tensor, allocated when not given)."""
+        if record is None:
+            record = torch.empty(self.record_bytes(), dtype=torch.uint8).pin_memory()
+        N._check(N.nomas_kv_archive(self.handle, frame, record.data_ptr(), _stream_handle(stream)), "nomas_kv_archive")
+        return record
+
+    def select(self, frames, records: Optional[dict] = None, stream=None):
+        """Make `frames` the retained history (age order); records: frame -> host record for frames that
+        are not retained now."""
+        recs = None if records is None else [records[f].data_ptr() if f in records else 0 for f in frames]
+        N._check(N.nomas_kv_select(self.handle, list(frames), recs, _stream_handle(stream)), "nomas_kv_select")
 
     def dequant(self, stream=None):
         st = self.state()

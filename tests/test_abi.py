@@ -82,3 +82,10 @@ def test_prompt_times_to_latent_windows():
         g = json.load(f)
     assert [segment_frames(s) for s in g["segments"]] == g["_expected_n_frames"]
     assert [[list(w) for w in action_windows(s)] for s in g["segments"]] == g["_expected_windows"]
+
+
+def test_frame_record_bytes(N):
+    # one archived frame: K and V codes (H*T*D int8 each) then K and V scales (H*T fp32 each)
+    d = N.make_dims(16, 128, 880, 18, 18, 768)
+    assert N.nomas_kv_frame_record_bytes(d) == 2 * 16 * 880 * 128 + 2 * 16 * 880 * 4
+    assert N.nomas_kv_frame_record_bytes(N.make_dims(16, 96, 880, 18, 18, 768)) == 0   # invalid head_dim

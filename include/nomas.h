@@ -343,7 +343,8 @@ const char *nomas_status_string(int status);
 const char *nomas_last_error(void);
 
 /* Test and diagnostic hook: the limit, in nanoseconds, of every bounded wait inside the attention
- * and append kernels (process-wide, default 2 000 000 000 = 2 s; it applies to later calls).  A
+ * and append kernels and the sparse selection's pooling kernel (process-wide, default
+ * 2 000 000 000 = 2 s; it applies to later calls).  A
  * wait that runs out records NOMAS_ETIMEOUT in the cache's device error word, and every role of the
  * CTA then leaves its loop, lets its in-flight copies and MMAs complete and releases TMEM, so the
  * device stays usable; the call's output is then undefined.  A limit of 0 makes a wait that its

@@ -60,7 +60,11 @@ def test_class_map_and_dense_lists(cfg):
 SPARSE = [small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), window=4),
           small_config(tokens_per_frame=97, n_frames=5, prior_frames=(4, 4), window=5, head_dim=64),
           small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), window=4, keep_frac=1.0),
-          CONFIGS["C3r"], CONFIGS["C3"]]
+          CONFIGS["C3r"], CONFIGS["C3"],
+          # 548 and 1173 candidates: the selection's register paths for up to 1024 keys and its
+          # shared-memory path beyond
+          small_config("wide", tokens_per_frame=100, n_frames=300, prior_frames=(400,), window=400),
+          small_config("wider", tokens_per_frame=100, n_frames=300, prior_frames=(700, 500), window=1200, heads=1)]
 
 
 @pytest.mark.parametrize("cfg", SPARSE, ids=lambda c: c.name + f"_T{c.tokens_per_frame}_k{c.keep_frac}")

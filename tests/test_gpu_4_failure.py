@@ -70,3 +70,35 @@ def test_forced_wait_limit_in_append_reports_timeout_and_the_next_append_is_exac
         s = slice((g % oc.C) * T, (g % oc.C + 1) * T)
         assert np.array_equal(fresh.ring_k8().cpu().numpy()[:, s], oc.k8[:, s])
         assert np.array_equal(fresh.ring_vs().cpu().numpy()[:, s].view(np.uint32), oc.vs[:, s].view(np.uint32))
+
+
+def test_forced_wait_limit_in_sparse_pooling_reports_timeout_and_the_next_build_is_exact():
+    # The sparse selection's pooling kernel waits for its TMA and bulk copies with the same bounded
+    # wait; with the limit at 0 the build records NOMAS_ETIMEOUT, its producer lets the copies land,
+    # and a rebuild on the same context reproduces the first build's selection and lists bit for bit.
+    from int8_kv_cache_action_b200.runtime import mask_views, segment_text_of
+    cfg = small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), window=4)
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    d = to_device(inp)
+    seg = segment_text_of(cfg.current)
+    buf, lay = gc.build_mask(seg, N.NOMAS_MODE_SPARSE, 0.25, d["q"], d["k_cur"])
+    torch.cuda.synchronize()
+    assert gc.status() == N.NOMAS_OK
+    ref = {k: v.clone() for k, v in mask_views(buf, lay).items() if k in ("sel", "score", "count", "list")}
+    prev = N.nomas_set_wait_limit_ns(0)
+    try:
+        gc.build_mask(seg, N.NOMAS_MODE_SPARSE, 0.25, d["q"], d["k_cur"])
+        torch.cuda.synchronize()
+        st = gc.status()
+    finally:
+        N.nomas_set_wait_limit_ns(prev)
+    assert st == N.NOMAS_ETIMEOUT
+    buf2, lay2 = gc.build_mask(seg, N.NOMAS_MODE_SPARSE, 0.25, d["q"], d["k_cur"])
+    torch.cuda.synchronize()
+    assert gc.status() == N.NOMAS_OK
+    mv = mask_views(buf2, lay2)
+    for k in ("sel", "score", "count"):
+        assert torch.equal(mv[k], ref[k]), k
+    for i, n in enumerate(ref["count"].tolist()):     # list entries past a list's count are unused
+        assert torch.equal(mv["list"][i, :n], ref["list"][i, :n])

@@ -16,22 +16,20 @@
 
 namespace nomas {
 
-// max.u16x2: per 16-bit half, the larger unsigned value.
-__device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
+template <int LPV>
+__device__ __forceinline__ float group_max(float a) {
+#pragma unroll
+    for (int off = LPV / 2; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+    return a;
 }
 
-// Absmax of the 16 bf16 values packed in w0, w1, as an fp32 bit pattern.  With the sign bit cleared a
-// bf16 bit pattern orders like its magnitude (an infinity above every finite value, a NaN above an
-// infinity), so the maximum is taken on the integers, as a tree; a NaN element makes the absmax NaN.
-__device__ __forceinline__ uint32_t absmax_bits(const uint4 &w0, const uint4 &w1) {
-    constexpr uint32_t M = 0x7FFF7FFFu;
-    const uint32_t a = umax16x2(w0.x & M, w0.y & M), b = umax16x2(w0.z & M, w0.w & M);
-    const uint32_t c = umax16x2(w1.x & M, w1.y & M), d = umax16x2(w1.z & M, w1.w & M);
-    const uint32_t m = umax16x2(umax16x2(a, b), umax16x2(c, d));
-    return max(m << 16, m & 0xFFFF0000u);
+__device__ __forceinline__ void unpack16(const uint4 &w0, const uint4 &w1, float (&x)[16]) {
+    const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        x[2 * i] = __uint_as_float(u[i] << 16);
+        x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    }
 }
 
 // s = RN(a / 127) for a = absmax of bf16 values, without the division routine: q0 = RN(a c) with
@@ -57,72 +55,56 @@ __device__ __forceinline__ float recip_nr(float s) {
     return __fmaf_rn(r0, __fmaf_rn(-s, r0, 1.0f), r0);
 }
 
-// Scale and codes rint(x / s) (fp32 IEEE division, round-half-even) for the 16 channels one lane holds
-// of one (token, head) vector, given the group's absmax a; s = RN(a / 127), so |x / s| <= 127 (1 + 2^-23)
-// and every code lies in [-127, 127].
+// Codes rint(x / s) in fp32 with IEEE division and round-half-even for the 16 channels this lane
+// holds; s = RN(absmax / 127) over the group's D channels, so |x / s| <= 127 (1 + 2^-23) and every
+// code lies in [-127, 127].
 // With r = 1/s to relative 2^-24 + 2^-40, the exact product x r is within 127 (2^-24 + 2^-40) (1 + 2^-23)
 // < 2^-17 of x / s, which is within 2^-18 of RN(x / s).  t = RN(x r + 1.5 * 2^23) (one FMA) holds the
-// integer q nearest x r, and d = RN(x r - q) (one FMA, |x r - q| <= 1/2, rounding error <= 2^-26).  When
-// |d| < 1/2 - 2^-15, RN(x / s) is within 1/2 - 2^-15 + 2^-26 + 2^-17 + 2^-18 < 1/2 of q, so rint(RN(x / s))
-// = q.  Otherwise (rarely; always for s below 2^-125, where r is a NaN) the exact quotient decides, on a
-// branch the warp takes only when one of its lanes needs it.  The fp32 add of 1.5 * 2^23 leaves q, as a
-// two's-complement byte, in the low byte of t's bit pattern.
-struct QuantOut {
-    uint4 codes;
-    bool slow;        // some element of this lane needs the exact quotient
-};
-
-__device__ __forceinline__ QuantOut quant_fast(const uint4 &w0, const uint4 &w1, float r) {
+// integer q nearest x r, and d = RN(x r - q) (one FMA; |x r - q| <= 1/2, rounding error <= 2^-26).  When
+// |d| < 1/2 - 2^-15, RN(x / s) is within 1/2 - 2^-15 + 2^-26 + 2^-17 + 2^-18 < 1/2 of q, so
+// rint(RN(x / s)) = q.  Otherwise the exact quotient decides: rarely, and always for s below 2^-125,
+// where r is a NaN.  The warp takes that branch only when one of its lanes needs it.  The fp32 add of
+// 1.5 * 2^23 leaves q, as a two's-complement byte, in the low byte of t's bit pattern.
+template <int LPV>
+__device__ __forceinline__ uint4 quant16(const float (&x)[16], float &s_out) {
     constexpr float kMagic = 12582912.0f;                 // 1.5 * 2^23
-    constexpr float kFar = 0.5f - 0x1p-15f;
-    const float2 r2 = make_float2(r, r), m2 = make_float2(kMagic, kMagic), neg1 = make_float2(-1.0f, -1.0f);
-    const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    uint32_t tb[8][2];
+    constexpr float kFar = 0.5f - 0x1p-15f;               // |y - rint(y)| below this: not near a tie
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
+    a = group_max<LPV>(a);
+    const float s = div127(a);
+    s_out = s;
+    const bool nz = s > 0.0f;
+    const float r = s >= 0x1p-125f ? recip_nr(s) : (nz ? __int_as_float(0x7fffffff) : 0.0f);
+    const float2 r2 = make_float2(r, r), m2 = make_float2(kMagic, kMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+    uint32_t tb[16];
     bool slow = false;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float2 x = make_float2(__uint_as_float(u[i] << 16), __uint_as_float(u[i] & 0xFFFF0000u));
-        const float2 t = __ffma2_rn(x, r2, m2);
-        const float2 nq = __ffma2_rn(t, neg1, m2);        // -q, exact
-        const float2 d = __ffma2_rn(x, r2, nq);
-        slow |= !(fabsf(d.x) < kFar) || !(fabsf(d.y) < kFar);   // NaN counts as near
-        tb[i][0] = __float_as_uint(t.x);
-        tb[i][1] = __float_as_uint(t.y);
+        const float2 xx = make_float2(x[2 * i], x[2 * i + 1]);
+        const float2 t = __ffma2_rn(xx, r2, m2);
+        const float2 nq = __ffma2_rn(t, neg1, m2);
+        const float2 d = __ffma2_rn(xx, r2, nq);
+        slow |= !(fabsf(d.x) < kFar) || !(fabsf(d.y) < kFar);   // NaN (tiny s) counts as near
+        tb[2 * i] = __float_as_uint(t.x);
+        tb[2 * i + 1] = __float_as_uint(t.y);
+    }
+    if (__any_sync(0xffffffffu, slow && nz)) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float t = __fmaf_rn(x[i], r, kMagic);
+            const float d = __fmaf_rn(x[i], r, -__fsub_rn(t, kMagic));
+            if (nz && !(fabsf(d) < kFar)) tb[i] = __float_as_uint(__fadd_rn(rintf(__fdiv_rn(x[i], s)), kMagic));
+        }
     }
     uint32_t w[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)   // low bytes of the 4 t of words 2i, 2i+1
-        w[i] = __byte_perm(__byte_perm(tb[2 * i][0], tb[2 * i][1], 0x0040),
-                           __byte_perm(tb[2 * i + 1][0], tb[2 * i + 1][1], 0x0040), 0x5410);
-    return QuantOut{make_uint4(w[0], w[1], w[2], w[3]), slow};
-}
-
-// The same codes with every element near a rounding tie taken from the exact quotient.
-__device__ __noinline__ uint4 quant_exact(const uint4 &w0, const uint4 &w1, float s, float r) {
-    constexpr float kMagic = 12582912.0f;
-    constexpr float kFar = 0.5f - 0x1p-15f;
-    const uint32_t u[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-    uint32_t tb[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float x = __uint_as_float((i & 1) ? (u[i >> 1] & 0xFFFF0000u) : (u[i >> 1] << 16));
-        const float t = __fmaf_rn(x, r, kMagic);
-        const float d = __fmaf_rn(x, r, -__fsub_rn(t, kMagic));
-        tb[i] = __float_as_uint(fabsf(d) < kFar ? t : __fadd_rn(rintf(__fdiv_rn(x, s)), kMagic));
-    }
-    uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)   // low bytes of t[4i .. 4i+3]
         w[i] = __byte_perm(__byte_perm(tb[4 * i], tb[4 * i + 1], 0x0040), __byte_perm(tb[4 * i + 2], tb[4 * i + 3], 0x0040),
                            0x5410);
     return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Reciprocal of a scale for the fast path: 1/s for s >= 2^-125, a NaN for smaller nonzero s (every
-// element then takes the exact path), 0 for s = 0 (all codes 0) or a non-finite s.
-__device__ __forceinline__ float scale_recip(float s) {
-    if (s >= 0x1p-125f && s <= 0x1.fffffep127f) return recip_nr(s);
-    return (s > 0.0f && s < 0x1p-125f) ? __int_as_float(0x7fffffff) : 0.0f;
 }
 
 template <int D>
@@ -239,23 +221,14 @@ __global__ void __launch_bounds__(kAppendThreads, 3)
         const int t = tb * C::TC + row_in_chunk;       // token within the job
         const uint4 *sk = reinterpret_cast<const uint4 *>(sm + st * C::STAGE + row_in_chunk * D * 2 + sub * 32);
         const uint4 *sv = reinterpret_cast<const uint4 *>(sm + st * C::STAGE + C::TILE + row_in_chunk * D * 2 + sub * 32);
-        // K and V of the token side by side: absmax trees, group reductions, scales, codes
-        const uint4 k0 = sk[0], k1 = sk[1], v0 = sv[0], v1 = sv[1];
-        uint32_t ak = absmax_bits(k0, k1), av = absmax_bits(v0, v1);
-#pragma unroll
-        for (int off = LPV / 2; off > 0; off >>= 1) {
-            ak = max(ak, __shfl_xor_sync(0xffffffffu, ak, off));
-            av = max(av, __shfl_xor_sync(0xffffffffu, av, off));
-        }
-        // every lane's loads of the stage have been consumed by the reductions above
-        if (lane == 0) mbar_arrive(&empty[st]);
-        const float skale = div127(__uint_as_float(ak)), svale = div127(__uint_as_float(av));
-        const float rk = scale_recip(skale), rv = scale_recip(svale);
-        QuantOut qk = quant_fast(k0, k1, rk), qv = quant_fast(v0, v1, rv);
-        if (__any_sync(0xffffffffu, (qk.slow && skale > 0.0f) || (qv.slow && svale > 0.0f))) {
-            if (qk.slow && skale > 0.0f) qk.codes = quant_exact(k0, k1, skale, rk);
-            if (qv.slow && svale > 0.0f) qv.codes = quant_exact(v0, v1, svale, rv);
-        }
+        float x[16];
+        float skale, svale;
+        unpack16(sk[0], sk[1], x);
+        const uint4 qk = quant16<LPV>(x, skale);
+        unpack16(sv[0], sv[1], x);
+        const uint4 qv = quant16<LPV>(x, svale);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);    // this warp's reads of the stage are done
         if (t < J.n_tok) {
             int64_t row;
             if (J.head_mode) {
@@ -274,8 +247,8 @@ __global__ void __launch_bounds__(kAppendThreads, 3)
                 row = (int64_t)slot * T + (t - f * T);
             }
             const int64_t di = (int64_t)h * J.rows_per_head + row;
-            *reinterpret_cast<uint4 *>(J.k8 + di * D + sub * 16) = qk.codes;
-            *reinterpret_cast<uint4 *>(J.v8 + di * D + sub * 16) = qv.codes;
+            *reinterpret_cast<uint4 *>(J.k8 + di * D + sub * 16) = qk;
+            *reinterpret_cast<uint4 *>(J.v8 + di * D + sub * 16) = qv;
             if (sub == 0) {
                 J.ks[di] = skale;
                 J.vs[di] = svale;

@@ -391,9 +391,55 @@ def run_ours(args, rank, world, local_rank):
     c4 = KVCache.for_config(big, dev)
     ws_bytes["full_history_7th_of_7"] = int(N.nomas_attn_workspace_bytes(c4.handle, segment_text_of(big.current)))
     del c4
+    linear = measure_linear(dev)
     return dict(ms=ms, phases=ph, flops_dense=flops_dense, flops_text=flops_text, flops_sparse=flops_sparse,
-                append_bytes=append_bytes,
+                append_bytes=append_bytes, linear=linear,
                 prep_bytes=prep_bytes, ws_bytes=ws_bytes, clocks=clk.summary(), e2e=e2e, cfg=cfg)
+
+
+def measure_linear(dev, reps=10):
+    """The INT8-weight linear layer on the DiT's production shapes (tokens of one 30-frame 1280x704 segment
+    plus its 1280 text tokens; hidden 2048, FFN 8192), synthetic bf16 activations and weights: the GEMM
+    alone (nomas_linear_bf16 on the dequantised weights) and the whole call (dequantise + GEMM)."""
+    import torch
+    from int8_kv_cache_action_b200 import _nomas as N
+    from int8_kv_cache_action_b200.runtime import Int8Linear
+    out = {}
+    for name, (m, k, n) in {"qkv_27680x2048x6144": (27680, 2048, 6144),
+                            "ffn_down_27680x8192x2048": (27680, 8192, 2048)}.items():
+        g = torch.Generator().manual_seed(77)
+        x = (torch.randn(m, k, generator=g)).to(torch.bfloat16).to(dev)
+        lin = Int8Linear.from_weights((torch.randn(n, k, generator=g) * 0.02).to(torch.bfloat16).to(dev))
+        w = lin.dequantized()
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        st = torch.cuda.current_stream().cuda_stream
+
+        def gemm():
+            N._check(N.nomas_linear_bf16(x.data_ptr(), m, k, k, w.data_ptr(), n, k, y.data_ptr(), n,
+                                         N.NOMAS_DTYPE_BF16, lin.status_word.data_ptr(), st), "nomas_linear_bf16")
+
+        def full():
+            lin(x, out=y)
+
+        res = {}
+        for label, fn in (("gemm", gemm), ("w8a16", full)):
+            for _ in range(3):
+                fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(reps):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / reps
+            res[label] = {"ms": ms, "tflops": 2.0 * m * n * k / (ms * 1e-3) / 1e12}
+        if lin.status() != N.NOMAS_OK:
+            raise RuntimeError("linear layer reported a device error")
+        res["dequant_bytes"] = n * k * (1 + 2) + 4 * n
+        out[name] = res
+        del x, w, y, lin
+    return out
 
 
 def per_config(args):
@@ -619,6 +665,14 @@ def main():
         "attn_dense_tflops": dense_tflops, "attn_sparse_tflops": sparse_tflops,
         "attn_dense_call_tflops": dense_call_tflops, "attn_sparse_call_tflops": sparse_call_tflops,
         "attn_workspace_bytes": r["ws_bytes"],
+        "roofline_linear": {
+            "bound": "tensor", "kernel": "gemm_bf16_kernel (nomas_linear_bf16; nomas_w8a16_linear adds the dequantise "
+                                        "pre-pass)",
+            "peak": peak_burst, "unit": "TFLOP/s", "peak_kind": f"bf16 dense, burst ({pk_kind})",
+            "shapes": {k: {"gemm_tflops": v["gemm"]["tflops"], "gemm_frac": v["gemm"]["tflops"] / peak_burst,
+                           "gemm_ms": v["gemm"]["ms"], "w8a16_ms": v["w8a16"]["ms"],
+                           "w8a16_tflops": v["w8a16"]["tflops"]} for k, v in r["linear"].items()},
+            "timed": "outside the step (the step is the attention path)"},
         "flops_per_step": {"dense": r["flops_dense"], "text": r["flops_text"], "sparse": r["flops_sparse"]},
         "kv_tokens_per_s_append": (cfg.window_frames * cfg.tokens_per_frame) * cfg.heads / (ph[0] * 1e-3),
         "cpu_baseline": cpu_base,

@@ -332,6 +332,42 @@ int nomas_attn_run(const nomas_kv_cache *cache, const nomas_segment_text *seg, i
  *   k_out, v_out  fp32 [history_tokens][H][D] */
 int nomas_kv_dequant(const nomas_kv_cache *cache, float *k_out, float *v_out, nomas_stream stream);
 
+/* ------------------------------------------------------------------------------------------
+ * INT8-weight / BF16-compute linear layer of the DiT (fluxbbs.com "单卡 4090 怎么做到的", first
+ * technique: model weights are stored as INT8 with float scale factors and dequantised back to BF16
+ * at compute time; the DiT's linear layers compute in BF16).  The pages give no formula; reading:
+ *   - one scale per output channel: row n of W [N][K] is quantised as one vector with the K/V
+ *     quantiser above (s_n = RN(absmax / 127), codes rint(w / s_n) half-even);
+ *   - dequantised weight w_nk = bf16(RN(fp32(q_nk * s_n)));
+ *   - y = x W^T with bf16 x, fp32 accumulation.
+ * Layouts: x bf16 [M][K] row pitch ldx elements, W (bf16 or codes) [N][K] row pitch ldw (codes: K),
+ * y [M][N] row pitch ldy >= N elements, fp32 (NOMAS_DTYPE_F32) or bf16 (NOMAS_DTYPE_BF16).  Every
+ * pointer is device memory, caller-owned, 16-byte aligned; K, ldx and ldw are multiples of 8.
+ * `status` is a caller-owned device int32[4] error word (same format as a cache's): a bounded wait
+ * that runs out records NOMAS_ETIMEOUT there; read and clear it with nomas_status_read.
+ * Errors (returned before anything is enqueued): NOMAS_EINVAL for a null or misaligned pointer,
+ * a size below 1 or a pitch that breaks the rules above; NOMAS_ECUDA for a failed launch. */
+#define NOMAS_DTYPE_F32 0
+#define NOMAS_DTYPE_BF16 1
+
+/* Quantise bf16 weights w [N][K] (row pitch ldw) into codes int8 [N][K] and scales fp32 [N]. */
+int nomas_w8_quantize(const void *w, int64_t n_out, int64_t k_in, int64_t ldw, int8_t *codes, float *scales,
+                      nomas_stream stream);
+/* Dequantise codes int8 [N][K] with scales fp32 [N] into bf16 weights w [N][K] (dense). */
+int nomas_w8_dequant(const int8_t *codes, const float *scales, int64_t n_out, int64_t k_in, void *w,
+                     nomas_stream stream);
+/* y = x W^T for bf16 x [M][K] and bf16 W [N][K]: tcgen05 tiles of 128 x 256, fp32 accumulation in TMEM. */
+int nomas_linear_bf16(const void *x, int64_t m, int64_t k_in, int64_t ldx, const void *w, int64_t n_out,
+                      int64_t ldw, void *y, int64_t ldy, int y_dtype, int32_t *status, nomas_stream stream);
+/* Bytes of the transient bf16 weights nomas_w8a16_linear dequantises into: N * K * 2. */
+size_t nomas_w8a16_workspace_bytes(int64_t n_out, int64_t k_in);
+/* nomas_w8_dequant into `workspace`, then nomas_linear_bf16 with those weights. */
+int nomas_w8a16_linear(const void *x, int64_t m, int64_t k_in, int64_t ldx, const int8_t *codes,
+                       const float *scales, int64_t n_out, void *y, int64_t ldy, int y_dtype, void *workspace,
+                       int32_t *status, nomas_stream stream);
+/* Synchronise `stream`, read and clear a linear layer's device error word. */
+int nomas_status_read(int32_t *status, nomas_stream stream);
+
 /* Synchronise `stream`, read and clear the device error word.  Returns NOMAS_OK
  * or the first device-side error recorded since the last call. */
 int nomas_device_status(const nomas_kv_cache *cache, nomas_stream stream);
@@ -343,7 +379,7 @@ const char *nomas_status_string(int status);
 const char *nomas_last_error(void);
 
 /* Test and diagnostic hook: the limit, in nanoseconds, of every bounded wait inside the attention
- * and append kernels and the sparse selection's pooling kernel (process-wide, default
+ * and append kernels, the sparse selection's pooling kernel and the linear layer (process-wide, default
  * 2 000 000 000 = 2 s; it applies to later calls).  A
  * wait that runs out records NOMAS_ETIMEOUT in the cache's device error word, and every role of the
  * CTA then leaves its loop, lets its in-flight copies and MMAs complete and releases TMEM, so the

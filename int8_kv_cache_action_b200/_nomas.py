@@ -24,13 +24,16 @@ NOMAS_MAX_TAILS = 64
 NOMAS_STATIC_POOL_FLOATS = 2 << 20
 NOMAS_MAX_SPARSE_CANDIDATES = 8192
 NOMAS_MAX_SELECT_FRAMES = 64
+NOMAS_DTYPE_F32, NOMAS_DTYPE_BF16 = 0, 1
 
 EXPORTED = ["nomas_kv_cache_bytes", "nomas_kv_cache_init", "nomas_kv_cache_destroy", "nomas_kv_cache_state",
             "nomas_kv_append", "nomas_mask_layout_query", "nomas_mask_bytes", "nomas_mask_build",
             "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string",
             "nomas_last_error", "nomas_mask_build_static", "nomas_attn_workspace_bytes",
             "nomas_set_wait_limit_ns", "nomas_attn_prepare", "nomas_attn_run", "nomas_kv_frame_record_bytes",
-            "nomas_kv_retained", "nomas_kv_evicted_by", "nomas_kv_archive", "nomas_kv_select"]
+            "nomas_kv_retained", "nomas_kv_evicted_by", "nomas_kv_archive", "nomas_kv_select",
+            "nomas_w8_quantize", "nomas_w8_dequant", "nomas_linear_bf16", "nomas_w8a16_workspace_bytes",
+            "nomas_w8a16_linear", "nomas_status_read"]
 
 
 class nomas_cache_dims(ctypes.Structure):
@@ -96,6 +99,13 @@ _sigs = {
     "nomas_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "nomas_last_error": (ctypes.c_char_p, []),
     "nomas_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
+    "nomas_w8_quantize": (ctypes.c_int, [_p, _i64, _i64, _i64, _p, _p, _p]),
+    "nomas_w8_dequant": (ctypes.c_int, [_p, _p, _i64, _i64, _p, _p]),
+    "nomas_linear_bf16": (ctypes.c_int, [_p, _i64, _i64, _i64, _p, _i64, _i64, _p, _i64, ctypes.c_int, _p, _p]),
+    "nomas_w8a16_workspace_bytes": (_sz, [_i64, _i64]),
+    "nomas_w8a16_linear": (ctypes.c_int, [_p, _i64, _i64, _i64, _p, _p, _i64, _p, _i64, ctypes.c_int, _p, _p,
+                                          _p]),
+    "nomas_status_read": (ctypes.c_int, [_p, _p]),
 }
 for _name, (_res, _args) in _sigs.items():
     _f = getattr(lib, _name)
@@ -251,3 +261,32 @@ def nomas_kv_dequant(handle, k_out, v_out, stream=0):
 
 def nomas_device_status(handle, stream=0):
     return lib.nomas_device_status(handle, stream or None)
+
+
+# ------------------------------------------------------------------------------------------------
+# INT8-weight / BF16-compute linear layer
+# ------------------------------------------------------------------------------------------------
+
+def nomas_w8_quantize(w, n_out, k_in, ldw, codes, scales, stream=0):
+    return lib.nomas_w8_quantize(w, n_out, k_in, ldw, codes, scales, stream or None)
+
+
+def nomas_w8_dequant(codes, scales, n_out, k_in, w, stream=0):
+    return lib.nomas_w8_dequant(codes, scales, n_out, k_in, w, stream or None)
+
+
+def nomas_linear_bf16(x, m, k_in, ldx, w, n_out, ldw, y, ldy, y_dtype, status, stream=0):
+    return lib.nomas_linear_bf16(x, m, k_in, ldx, w, n_out, ldw, y, ldy, y_dtype, status, stream or None)
+
+
+def nomas_w8a16_workspace_bytes(n_out, k_in):
+    return lib.nomas_w8a16_workspace_bytes(n_out, k_in)
+
+
+def nomas_w8a16_linear(x, m, k_in, ldx, codes, scales, n_out, y, ldy, y_dtype, workspace, status, stream=0):
+    return lib.nomas_w8a16_linear(x, m, k_in, ldx, codes, scales, n_out, y, ldy, y_dtype, workspace, status,
+                                  stream or None)
+
+
+def nomas_status_read(status, stream=0):
+    return lib.nomas_status_read(status, stream or None)

@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "quant.cuh"
 
 namespace nomas {
 
@@ -30,29 +31,6 @@ __device__ __forceinline__ void unpack16(const uint4 &w0, const uint4 &w1, float
         x[2 * i] = __uint_as_float(u[i] << 16);
         x[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
     }
-}
-
-// s = RN(a / 127) for a = absmax of bf16 values, without the division routine: q0 = RN(a c) with
-// c = RN(1/127), the remainder a - 127 q0 is exact by FMA, and s = RN(q0 + (a - 127 q0) c) is
-// Markstein's correction step ("Computation of elementary functions on the IBM RISC System/6000
-// processor", 1990).  Checked by exact rational arithmetic against RN(a / 127) for every bf16 a in
-// [2^-110, max finite], where q0 and s are normals and the remainder (a subnormal at the low end) is
-// exact; zero gives zero, and subnormal or non-finite a take the IEEE division.
-__device__ __forceinline__ float div127(float a) {
-    constexpr float c = 0x1.020408p-7f;                   // RN(1/127)
-    const float q0 = __fmul_rn(a, c);
-    const float s = __fmaf_rn(__fmaf_rn(-q0, 127.0f, a), c, q0);
-    if (!(a >= 0x1p-110f && a <= 0x1.fffffep127f) && a != 0.0f) return __fdiv_rn(a, 127.0f);
-    return s;
-}
-
-// 1/s for normal s: the hardware approximation (PTX rcp.approx.f32, relative error about 2^-23)
-// refined by one Newton-Raphson step r = r0 + r0 (1 - s r0), both by FMA, leaves a relative error
-// below 2^-24 + 2^-40.
-__device__ __forceinline__ float recip_nr(float s) {
-    float r0;
-    asm("rcp.approx.f32 %0, %1;" : "=f"(r0) : "f"(s));
-    return __fmaf_rn(r0, __fmaf_rn(-s, r0, 1.0f), r0);
 }
 
 // Codes rint(x / s) in fp32 with IEEE division and round-half-even for the 16 channels this lane

@@ -208,3 +208,55 @@ def mask_views(mask_buf: torch.Tensor, lay: dict):
     out["count"] = mask_buf[lay["off_count"]:lay["off_count"] + nl * 4].view(torch.int32)
     out["list"] = mask_buf[lay["off_list"]:lay["off_list"] + nl * cap * 16].view(torch.int32).view(nl, cap, 4)
     return out
+
+
+class Int8Linear:
+    """A DiT linear layer with INT8 weights and float scales per output channel, computed in BF16
+    (include/nomas.h): codes int8 [N][K] and scales fp32 [N] stay resident; every call dequantises the
+    codes into a transient bf16 workspace and runs the tensor-core GEMM y = x W^T."""
+
+    def __init__(self, codes: torch.Tensor, scales: torch.Tensor):
+        if codes.dtype != torch.int8 or codes.dim() != 2 or not codes.is_contiguous():
+            raise ValueError("codes: contiguous int8 [N, K]")
+        if scales.dtype != torch.float32 or scales.shape != (codes.shape[0],):
+            raise ValueError("scales: float32 [N]")
+        self.codes, self.scales = codes, scales
+        self.n_out, self.k_in = codes.shape
+        self.workspace = torch.empty(N.nomas_w8a16_workspace_bytes(self.n_out, self.k_in), dtype=torch.uint8,
+                                     device=codes.device)
+        self.status_word = torch.zeros(4, dtype=torch.int32, device=codes.device)
+
+    @classmethod
+    def from_weights(cls, w: torch.Tensor, stream=None) -> "Int8Linear":
+        """Quantise bf16 weights [N, K] on the device."""
+        if w.dtype != torch.bfloat16 or w.dim() != 2 or w.stride(1) != 1:
+            raise ValueError("w: bf16 [N, K] with contiguous rows")
+        n, k = w.shape
+        codes = torch.empty((n, k), dtype=torch.int8, device=w.device)
+        scales = torch.empty(n, dtype=torch.float32, device=w.device)
+        N._check(N.nomas_w8_quantize(w.data_ptr(), n, k, w.stride(0), codes.data_ptr(), scales.data_ptr(),
+                                     _stream_handle(stream)), "nomas_w8_quantize")
+        return cls(codes, scales)
+
+    def dequantized(self, stream=None) -> torch.Tensor:
+        w = torch.empty((self.n_out, self.k_in), dtype=torch.bfloat16, device=self.codes.device)
+        N._check(N.nomas_w8_dequant(self.codes.data_ptr(), self.scales.data_ptr(), self.n_out, self.k_in,
+                                    w.data_ptr(), _stream_handle(stream)), "nomas_w8_dequant")
+        return w
+
+    def __call__(self, x: torch.Tensor, out_dtype=torch.bfloat16, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+        if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1 or x.shape[1] != self.k_in:
+            raise ValueError("x: bf16 [M, K] with contiguous rows")
+        m = x.shape[0]
+        if out is None:
+            out = torch.empty((m, self.n_out), dtype=out_dtype, device=x.device)
+        dt = N.NOMAS_DTYPE_BF16 if out.dtype == torch.bfloat16 else N.NOMAS_DTYPE_F32
+        N._check(N.nomas_w8a16_linear(x.data_ptr(), m, self.k_in, x.stride(0), self.codes.data_ptr(),
+                                      self.scales.data_ptr(), self.n_out, out.data_ptr(), out.stride(0), dt,
+                                      self.workspace.data_ptr(), self.status_word.data_ptr(),
+                                      _stream_handle(stream)), "nomas_w8a16_linear")
+        return out
+
+    def status(self, stream=None) -> int:
+        return N.nomas_status_read(self.status_word.data_ptr(), _stream_handle(stream))

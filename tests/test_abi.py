@@ -89,3 +89,24 @@ def test_frame_record_bytes(N):
     d = N.make_dims(16, 128, 880, 18, 18, 768)
     assert N.nomas_kv_frame_record_bytes(d) == 2 * 16 * 880 * 128 + 2 * 16 * 880 * 4
     assert N.nomas_kv_frame_record_bytes(N.make_dims(16, 96, 880, 18, 18, 768)) == 0   # invalid head_dim
+
+
+def test_linear_host_checks_without_a_device(N):
+    # every rejected argument returns before any CUDA call, so this runs without a GPU
+    assert N.nomas_w8a16_workspace_bytes(2048, 6144) == 2048 * 6144 * 2
+    assert N.nomas_w8a16_workspace_bytes(0, 8) == 0
+    a = 0x10000                                          # 16-byte aligned stand-in addresses (never read)
+    ok = dict(x=a, m=4, k_in=32, ldx=32, codes=a, scales=a, n_out=16, y=a, ldy=16, y_dtype=N.NOMAS_DTYPE_F32,
+              workspace=a, status=a)
+
+    def call(**kw):
+        v = dict(ok, **kw)
+        return N.nomas_w8a16_linear(v["x"], v["m"], v["k_in"], v["ldx"], v["codes"], v["scales"], v["n_out"],
+                                    v["y"], v["ldy"], v["y_dtype"], v["workspace"], v["status"])
+    for bad in (dict(k_in=30, ldx=30), dict(ldx=16), dict(m=0), dict(n_out=0), dict(x=a + 4), dict(y=0),
+                dict(y_dtype=2), dict(status=0), dict(ldy=12), dict(codes=0), dict(workspace=a + 8)):
+        assert call(**bad) == N.NOMAS_EINVAL, bad
+    assert N.nomas_linear_bf16(a, 4, 32, 32, a, 16, 24, a, 16, 0, a) == N.NOMAS_EINVAL   # W pitch not a multiple of 8
+    assert N.nomas_w8_dequant(a, a, 16, 12, a) == N.NOMAS_EINVAL                         # K not a multiple of 8
+    assert N.nomas_w8_quantize(0, 16, 32, 32, a, a) == N.NOMAS_EINVAL
+    assert N.nomas_status_read(0) == N.NOMAS_EINVAL

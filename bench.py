@@ -56,7 +56,9 @@ TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose 
     "attn": (os.path.join(ROOT, "profiles", "attn_dense_production_traffic.json"),
              (os.path.join(CSRC, "attn.cu"), COMMON)),
     "append": (os.path.join(ROOT, "profiles", "append_production_traffic.json"),
-               (os.path.join(CSRC, "append.cu"), COMMON)),
+               (os.path.join(CSRC, "append.cu"), os.path.join(CSRC, "quant.cuh"), COMMON)),
+    "linear": (os.path.join(ROOT, "profiles", "gemm_dit_qkv_traffic.json"),
+               (os.path.join(CSRC, "linear.cu"), os.path.join(CSRC, "quant.cuh"), COMMON)),
 }
 
 
@@ -575,6 +577,8 @@ def main():
                     help="print one line per config (attention call and append) instead of the step line")
     ap.add_argument("--only", default="", help="with --per-config: comma-separated config names (C0..C4, C3r)")
     ap.add_argument("--reps", type=int, default=0, help="with --per-config: timed calls per config")
+    ap.add_argument("--linear-only", action="store_true",
+                    help="print one line with the INT8-weight linear layer on the DiT shapes only")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
@@ -603,6 +607,13 @@ def main():
 
     if args.per_config:
         per_config(args)
+        return
+    if args.linear_only:
+        import torch
+        lin = measure_linear(torch.device("cuda", 0), reps=args.reps or 10)
+        peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        print(json.dumps({"linear": lin, "peak_bf16_tflops": peak, "peak_kind": pk_kind,
+                          "frac": {k: v["gemm"]["tflops"] / peak for k, v in lin.items()}}))
         return
 
     import torch
@@ -672,6 +683,7 @@ def main():
             "shapes": {k: {"gemm_tflops": v["gemm"]["tflops"], "gemm_frac": v["gemm"]["tflops"] / peak_burst,
                            "gemm_ms": v["gemm"]["ms"], "w8a16_ms": v["w8a16"]["ms"],
                            "w8a16_tflops": v["w8a16"]["tflops"]} for k, v in r["linear"].items()},
+            "traffic_qkv": measured_traffic("linear"),
             "timed": "outside the step (the step is the attention path)"},
         "flops_per_step": {"dense": r["flops_dense"], "text": r["flops_text"], "sparse": r["flops_sparse"]},
         "kv_tokens_per_s_append": (cfg.window_frames * cfg.tokens_per_frame) * cfg.heads / (ph[0] * 1e-3),

@@ -10,7 +10,8 @@ tails of 64):
   a4" nomas_mask_build + nomas_attn_run (NOMAS_MODE_TEXT)   the text query rows of the same joint
       attention (the text stream), over the workspace the video call prepared (same K/V and cache)
   a3  nomas_mask_build    sparse selection (25 % of candidate video blocks)
-  a4' nomas_attn_prepare + nomas_attn_run   block-sparse attention (steps 3-8)
+  a4' nomas_attn_run      block-sparse attention (steps 3-8) over the same prepared workspace: one
+      pre-pass serves every call of one cache state and one segment's K/V
 (nomas_attn_fwd is exactly prepare + run; they are called separately so each is timed.)
 `value` = algorithmic attention FLOPs of the step (visible / selected keys only) / step time, on the
 device, inputs resident in HBM.  Inputs (324 MB of bf16 q/k/v per step) exceed the 126 MB L2.
@@ -47,9 +48,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # Kernel launches of one step: append 1; dense mask 3; prepare 3 (key copy, transposed values, history
-# widening); dense attention 1; text mask 3; text attention 1; sparse mask 5; prepare 3; sparse
-# attention 1.
-LAUNCHES_PER_STEP = 21
+# widening); dense attention 1; text mask 3; text attention 1; sparse mask 5; sparse attention 1.
+LAUNCHES_PER_STEP = 18
 CSRC = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc")
 COMMON = os.path.join(CSRC, "common.cuh")
 TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose digest it was taken with)
@@ -286,11 +286,9 @@ def run_ours(args, rank, world, local_rank):
         check(N.nomas_mask_build(cache.handle, seg, 1, 0.25, b["q"].data_ptr(), b["kc"].data_ptr(), ts, hs,
                                  mbuf_s.data_ptr(), sh), "mask sparse")
         mark(7)
-        prepare()
-        mark(8)
         check(N.nomas_attn_run(cache.handle, seg, 1, 0.25, mbuf_s.data_ptr(), b["q"].data_ptr(), ts, hs, scale,
                                b["out_s"].data_ptr(), 0, ws.data_ptr(), sh), "attn sparse")
-        mark(9)
+        mark(8)
 
     for _ in range(args.warmup):
         step()
@@ -330,11 +328,11 @@ def run_ours(args, rank, world, local_rank):
     # per-phase breakdown: a separate pass of steps issued back to back with events between the
     # phases (no host synchronisation inside the pass, so no phase includes host launch latency)
     n_ph = max(3, min(args.steps, 10))
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(n_ph)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(9)] for _ in range(n_ph)]
     for k in range(n_ph):
         step(evs[k])
     torch.cuda.synchronize()
-    ph = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(n_ph)) for i in range(9)]
+    ph = [statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(n_ph)) for i in range(8)]
 
     # end to end: every step copies its inputs from pinned host memory, runs the same C-ABI calls and
     # copies both outputs back.  Like a serving loop, the copies of one step overlap the compute of
@@ -635,15 +633,15 @@ def main():
     flops = r["flops_dense"] + r["flops_text"] + r["flops_sparse"]
     _, value = aggregate_ranks(ms_step, flops, world)
     value /= 1e12
-    # append, mask dense, prepare, run dense, mask text, run text, mask sparse, prepare, run sparse
+    # append, mask dense, prepare, run dense, mask text, run text, mask sparse, run sparse
     ph = r["phases"]
     dense_tflops = r["flops_dense"] / (ph[3] * 1e-3) / 1e12
     text_tflops = r["flops_text"] / (ph[5] * 1e-3) / 1e12
-    sparse_tflops = r["flops_sparse"] / (ph[8] * 1e-3) / 1e12
+    sparse_tflops = r["flops_sparse"] / (ph[7] * 1e-3) / 1e12
     dense_call_tflops = r["flops_dense"] / ((ph[2] + ph[3]) * 1e-3) / 1e12
-    sparse_call_tflops = r["flops_sparse"] / ((ph[7] + ph[8]) * 1e-3) / 1e12
+    sparse_call_tflops = r["flops_sparse"] / (ph[7] * 1e-3) / 1e12   # the workspace is already prepared
     append_gbs = r["append_bytes"] / (ph[0] * 1e-3) / 1e9
-    prep_ms = 0.5 * (ph[2] + ph[7])
+    prep_ms = ph[2]
     prep_gbs = r["prep_bytes"] / (prep_ms * 1e-3) / 1e9
     peak_sus = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -670,8 +668,7 @@ def main():
                              "achieved": prep_gbs, "peak": hbm, "unit": "GB/s", "frac": prep_gbs / hbm,
                              "bytes_per_call": r["prep_bytes"], "ms_per_call": prep_ms, "traffic": None},
         "breakdown_ms": {"append": ph[0], "mask_dense": ph[1], "prepare_dense": ph[2], "attn_dense": ph[3],
-                         "mask_text": ph[4], "attn_text": ph[5], "mask_sparse": ph[6], "prepare_sparse": ph[7],
-                         "attn_sparse": ph[8]},
+                         "mask_text": ph[4], "attn_text": ph[5], "mask_sparse": ph[6], "attn_sparse": ph[7]},
         "attn_text_tflops": text_tflops,
         "attn_dense_tflops": dense_tflops, "attn_sparse_tflops": sparse_tflops,
         "attn_dense_call_tflops": dense_call_tflops, "attn_sparse_call_tflops": sparse_call_tflops,

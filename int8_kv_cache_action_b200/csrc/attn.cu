@@ -286,16 +286,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int t = threadIdx.x - 32 * kWarpCi;   // 0..127
         struct ColInfo {
             float ks, vs;   // raw key / value scale (cached tiles), 1 / 0 otherwise
-            VisCode w;      // visibility code of the key
+            VisCode w;      // visibility code of the key (masked tiles only)
+            bool masked;    // the softmax reads the codes of this tile
         };
         // Column info of a tile (key scale, value scale, visibility code), loaded one tile ahead of its
         // use: only loads happen here, so nothing waits for them until the next tile consumes them.
         auto col_info = [&](const int4 &e, int col) -> ColInfo {
-            ColInfo ci{0.0f, 0.0f, key_none()};
+            ColInfo ci{0.0f, 0.0f, key_none(), (e.x & mask_bit) != 0};
             const int kind = e.x & 3;
             const int64_t start = e.y;
             if (col < e.z) {
-                if (kind == kKindText) {
+                if (!ci.masked) {
+                    // codes unused: the whole tile is visible to every row of the block
+                } else if (kind == kKindText) {
                     if (start + col < p.head_len) {
                         ci.w = key_always();
                     } else {
@@ -332,7 +335,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (!__all_sync(0xffffffffu, mbar_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, wd, 1))) break;
             sCS[ci * 128 + t] = p.scale_log2 * c0.ks;
             sCV[ci * 128 + t] = c0.vs;
-            sCW[ci * 128 + t] = make_int4(c0.w.x, c0.w.y, c0.w.z, c0.w.w);
+            if (c0.masked) sCW[ci * 128 + t] = make_int4(c0.w.x, c0.w.y, c0.w.z, c0.w.w);
             __syncwarp();
             if (lane == 0) mbar_arrive(&ci_full[ci]);
             ++u;

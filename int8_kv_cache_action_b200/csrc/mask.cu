@@ -465,15 +465,13 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
     }
 }
 
-// score[h][b][cand] = fmaf chain over channels in ascending order from +0.0f.  One CTA covers 32 query
-// blocks x 32 candidates of one head (small patches: the work is tiny, so latency, not arithmetic, is
-// what many CTAs hide); each of its 256 threads runs the 4 independent chains of a 2 x 2 patch.  Means
-// are staged channel-major in shared memory, 64 channels at a time, so a thread reads its 2 query means
-// and its 2 candidate means of one channel as two float2.
-constexpr int kScoreTile = 32;
+// score[h][b][cand] = fmaf chain over channels in ascending order from +0.0f.  One CTA covers 64 query
+// blocks x 64 candidates of one head; each of its 256 threads runs the 16 independent chains of a
+// 4 x 4 patch.  Means are staged channel-major in shared memory, 64 channels at a time, so a thread
+// reads its 4 query means and its 4 candidate means of one channel as two float4.
+constexpr int kScoreTile = 64;
 
 __global__ void __launch_bounds__(256) score_kernel(MaskParams p, const float *qmean, const float *kmean) {
-    constexpr int P = kScoreTile / 16;
     __shared__ __align__(16) float sq[64][kScoreTile];   // [channel in chunk][query block]
     __shared__ __align__(16) float sk[64][kScoreTile];   // [channel in chunk][candidate]
     const int D = p.D;
@@ -481,11 +479,11 @@ __global__ void __launch_bounds__(256) score_kernel(MaskParams p, const float *q
     const int n_ct = (p.n_cand + kScoreTile - 1) / kScoreTile;   // candidate tiles; x = qb tile * n_ct + ct
     const int b0 = (int)(blockIdx.x / n_ct) * kScoreTile, c0 = (int)(blockIdx.x % n_ct) * kScoreTile;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[P][P];
+    float acc[4][4];
 #pragma unroll
-    for (int i = 0; i < P; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < P; ++j) acc[i][j] = 0.0f;
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
     const float *qm = qmean + (int64_t)h * p.n_qb * D;
     const float *km = kmean + (int64_t)h * p.n_cand * D;
     for (int ch0 = 0; ch0 < D; ch0 += 64) {
@@ -505,25 +503,25 @@ __global__ void __launch_bounds__(256) score_kernel(MaskParams p, const float *q
             sk[c4 + 3][r] = b.w;
         }
         __syncthreads();
-#pragma unroll 16
+#pragma unroll 8
         for (int c = 0; c < 64; ++c) {
-            const float2 qv = *reinterpret_cast<const float2 *>(&sq[c][ty * P]);
-            const float2 kv = *reinterpret_cast<const float2 *>(&sk[c][tx * P]);
-            const float qa[P] = {qv.x, qv.y}, ka[P] = {kv.x, kv.y};
+            const float4 qv = *reinterpret_cast<const float4 *>(&sq[c][ty * 4]);
+            const float4 kv = *reinterpret_cast<const float4 *>(&sk[c][tx * 4]);
+            const float qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-            for (int i = 0; i < P; ++i)
+            for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < P; ++j) acc[i][j] = __fmaf_rn(qa[i], ka[j], acc[i][j]);
+                for (int j = 0; j < 4; ++j) acc[i][j] = __fmaf_rn(qa[i], ka[j], acc[i][j]);
         }
     }
     float *sc = reinterpret_cast<float *>(p.buf + p.lay.off_score);
 #pragma unroll
-    for (int i = 0; i < P; ++i) {
-        const int b = b0 + ty * P + i;
+    for (int i = 0; i < 4; ++i) {
+        const int b = b0 + ty * 4 + i;
         if (b >= p.n_qb) continue;
 #pragma unroll
-        for (int j = 0; j < P; ++j) {
-            const int cand = c0 + tx * P + j;
+        for (int j = 0; j < 4; ++j) {
+            const int cand = c0 + tx * 4 + j;
             if (cand < p.n_cand) sc[((int64_t)h * p.n_qb + b) * p.n_cand + cand] = acc[i][j];
         }
     }

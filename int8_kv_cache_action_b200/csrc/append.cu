@@ -17,6 +17,13 @@
 
 namespace nomas {
 
+// max(a, b, c); a NaN operand is ignored unless all three are NaN (PTX max.f32 semantics).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 template <int LPV>
 __device__ __forceinline__ float group_max(float a) {
 #pragma unroll
@@ -42,14 +49,16 @@ __device__ __forceinline__ void unpack16(const uint4 &w0, const uint4 &w1, float
 // |d| < 1/2 - 2^-15, RN(x / s) is within 1/2 - 2^-15 + 2^-26 + 2^-17 + 2^-18 < 1/2 of q, so
 // rint(RN(x / s)) = q.  Otherwise the exact quotient decides: rarely, and always for s below 2^-125,
 // where r is a NaN.  The warp takes that branch only when one of its lanes needs it.  The fp32 add of
-// 1.5 * 2^23 leaves q, as a two's-complement byte, in the low byte of t's bit pattern.
+// 1.5 * 2^23 leaves q, as a two's-complement byte, in the low byte of t's bit pattern.  The absmax
+// and the largest |d| of the lane are taken with three-input maxima (which return a NaN only when every
+// operand is one, so a NaN start value drops out and an all-NaN d -- the tiny-s case -- stays NaN).
 template <int LPV>
 __device__ __forceinline__ uint4 quant16(const float (&x)[16], float &s_out) {
     constexpr float kMagic = 12582912.0f;                 // 1.5 * 2^23
     constexpr float kFar = 0.5f - 0x1p-15f;               // |y - rint(y)| below this: not near a tie
     float a = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(x[i]));
+    for (int i = 0; i < 16; i += 2) a = max3f(a, fabsf(x[i]), fabsf(x[i + 1]));
     a = group_max<LPV>(a);
     const float s = div127(a);
     s_out = s;
@@ -58,17 +67,18 @@ __device__ __forceinline__ uint4 quant16(const float (&x)[16], float &s_out) {
     const float2 r2 = make_float2(r, r), m2 = make_float2(kMagic, kMagic);
     const float2 neg1 = make_float2(-1.0f, -1.0f);
     uint32_t tb[16];
-    bool slow = false;
+    float dmax = __int_as_float(0x7fffffff);             // NaN: max.f32 keeps the other operands
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
         const float2 xx = make_float2(x[2 * i], x[2 * i + 1]);
         const float2 t = __ffma2_rn(xx, r2, m2);
         const float2 nq = __ffma2_rn(t, neg1, m2);
         const float2 d = __ffma2_rn(xx, r2, nq);
-        slow |= !(fabsf(d.x) < kFar) || !(fabsf(d.y) < kFar);   // NaN (tiny s) counts as near
+        dmax = max3f(dmax, fabsf(d.x), fabsf(d.y));
         tb[2 * i] = __float_as_uint(t.x);
         tb[2 * i + 1] = __float_as_uint(t.y);
     }
+    const bool slow = !(dmax < kFar);                     // NaN (tiny s: every d is NaN) counts as near
     if (__any_sync(0xffffffffu, slow && nz)) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {

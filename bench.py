@@ -48,8 +48,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # Kernel launches of one step: append 1; dense mask 3; prepare 3 (key copy, transposed values, history
-# widening); dense attention 1; text mask 3; text attention 1; sparse mask 5; sparse attention 1.
-LAUNCHES_PER_STEP = 18
+# widening); dense attention 1; text mask 3; text attention 2 (the list shares, their merge); sparse
+# mask 5; sparse attention 1.
+LAUNCHES_PER_STEP = 19
 CSRC = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc")
 COMMON = os.path.join(CSRC, "common.cuh")
 TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose digest it was taken with)

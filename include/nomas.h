@@ -388,6 +388,16 @@ const char *nomas_last_error(void);
  * limit. */
 uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns);
 
+/* Tuning and test hook: the number of shares a NOMAS_MODE_TEXT call cuts each key list into.  The
+ * text query rows fill only ceil(text_tokens / 128) x heads CTAs and their lists differ in length, so
+ * each list is cut into shares of ceil(list capacity / shares) entries, one CTA each; a CTA writes its
+ * output without normalisation plus (running maximum, row sum) per row to the workspace, and a merge
+ * kernel forms out and lse from the shares (the softmax merge of disjoint key sets, exact up to
+ * rounding order).  By default (shares = 0) the call picks the count from the CTA count, the SM
+ * count and the list capacity; 1 to 16 forces that count (1: one CTA per list, no merge); other
+ * values select the default.  Process-wide, applies to later calls; returns the previous setting. */
+int nomas_set_text_split(int shares);
+
 #ifdef __cplusplus
 }
 #endif

@@ -42,6 +42,7 @@
 // moves only when the row maximum grows by more than 6 (log2 units), so p <= 64 and p * scale stays
 // inside fp16 for every input in the supported range (absmax <= 65504 gives scale <= 516); O is
 // then rescaled in TMEM once the previous PV has completed.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cuda_fp16.h>
@@ -110,6 +111,12 @@ struct AttnParams {
     float *lse;
     int *err;
     uint64_t timeout_ns;
+    // text query rows: each list cut into shares of share_len entries, share blockIdx.z per CTA, which
+    // writes its O without normalisation and (offset, row sum) per row for attn_combine_kernel;
+    // share_len == 0: the whole list, normalised output
+    int32_t share_len;
+    float *part_o;              // [share][Nq][H][D]
+    float2 *part_ml;            // [share][H][Nq]
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -219,7 +226,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int use_bit = (qb & 1) ? kUse1 : kUse0;
     const int mask_bit = (qb & 1) ? kMask1 : kMask0;
     const int list_id = p.sparse ? h * p.n_pairs + (qb >> 1) : (qb >> 1);
-    const int4 *list = p.lists + (int64_t)list_id * p.expect.list_cap;
+    const int4 *list = p.lists + (int64_t)list_id * p.expect.list_cap;   // advanced to this split's share below
 
     // header check (every thread reads the same words; all take the same branch)
     const MaskHeader *hd = reinterpret_cast<const MaskHeader *>(p.mask);
@@ -238,7 +245,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (threadIdx.x == 0) set_device_error(p.err, NOMAS_EDEVICE, hdr_ok ? 2 : 1);
         return;
     }
-    const int n_tiles = p.counts[list_id];
+    // this CTA's share of the list (a share past the list's end has nothing to do: the merge skips it)
+    const int n_all = p.counts[list_id];
+    const bool partial = p.share_len > 0;
+    const int lo = partial ? (int)blockIdx.z * p.share_len : 0;
+    if (partial && lo >= n_all) return;
+    const int n_tiles = partial ? min(p.share_len, n_all - lo) : n_all;
+    list += lo;
 
     if (threadIdx.x == 0) {
         mbar_init(q_ready, 8);
@@ -613,8 +626,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (ok) {
             tc_fence_after();
             const float lt = l + sXL[(half ^ 1) * 128 + r];
-            const float inv = lt > 0.0f ? 1.0f / lt : 0.0f;
-            float *dst = p.out + (row * p.H + h) * (int64_t)D + half * DH;
+            const float inv = partial ? 1.0f : (lt > 0.0f ? 1.0f / lt : 0.0f);
+            float *dst = (partial ? p.part_o + (int64_t)blockIdx.z * p.Nq * p.H * D : p.out) +
+                         (row * p.H + h) * (int64_t)D + half * DH;
             const uint32_t tO = tmem + lane_base + kTmO + (uint32_t)(half * DH);
 #pragma unroll 1
             for (int c0 = 0; c0 < DH; c0 += 32) {
@@ -625,12 +639,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int i = 0; i < 32; i += 4) {
                         float4 v = make_float4(__uint_as_float(rr[i]) * inv, __uint_as_float(rr[i + 1]) * inv,
                                                __uint_as_float(rr[i + 2]) * inv, __uint_as_float(rr[i + 3]) * inv);
-                        if (lt == 0.0f) v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);   // no visible key at all
+                        if (lt == 0.0f) v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);   // no visible key (in this share)
                         *reinterpret_cast<float4 *>(dst + c0 + i) = v;
                     }
                 }
             }
-            if (p.lse && row_ok && half == 0)
+            if (partial && row_ok && half == 0)
+                p.part_ml[((int64_t)blockIdx.z * p.H + h) * p.Nq + row] = make_float2(m_used, lt);
+            else if (p.lse && row_ok && half == 0)
                 p.lse[(int64_t)h * p.Nq + row] = (m_used + log2f(lt)) * 0.69314718055994530942f;
         }
     }
@@ -643,6 +659,48 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
 }
 
+}  // namespace nomas
+
+// Merge of the list shares of a text-row call: per (row, head), over the shares that saw a visible key,
+// with M the largest offset, O = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M) and lse = (M + log2 of
+// the denominator) ln 2 (the kernel's log2 domain).  Shares past the end of the row's list were not
+// run and are not read.  One warp per (row, head), D / 32 channels per lane.
+namespace nomas {
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float *part_o, const float2 *part_ml,
+                                                           const int32_t *counts, int share_len, int64_t Nq,
+                                                           int H, float *out, float *lse) {
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= Nq * H) return;                       // warp-uniform
+    const int64_t row = w / H;
+    const int h = (int)(w - row * H);
+    const int n_share = (counts[row >> 8] + share_len - 1) / share_len;   // list of the block pair
+    float M = -INFINITY;
+    for (int s = 0; s < n_share; ++s) {
+        const float2 ml = part_ml[((int64_t)s * H + h) * Nq + row];
+        if (ml.y > 0.0f) M = fmaxf(M, ml.x);
+    }
+    constexpr int PL = D / 32;
+    float acc[PL];
+#pragma unroll
+    for (int i = 0; i < PL; ++i) acc[i] = 0.0f;
+    float L = 0.0f;
+    for (int s = 0; s < n_share; ++s) {
+        const float2 ml = part_ml[((int64_t)s * H + h) * Nq + row];
+        if (!(ml.y > 0.0f)) continue;
+        const float wgt = exp2f(ml.x - M);
+        L += ml.y * wgt;
+        const float *src = part_o + (((int64_t)s * Nq + row) * H + h) * D;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) acc[i] += src[lane + 32 * i] * wgt;
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    float *dst = out + (row * H + h) * (int64_t)D;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) dst[lane + 32 * i] = acc[i] * inv;
+    if (lse && lane == 0) lse[(int64_t)h * Nq + row] = (M + log2f(L)) * 0.69314718055994530942f;
+}
 }  // namespace nomas
 
 // ------------------------------------------------------------------------------------------------
@@ -667,8 +725,10 @@ static int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 //   ksl, vsl fp32 [H][lhp]        their scales
 //   kp       fp16 [H][Lp][D]      description-head key codes
 //   vpt      fp16 [H][D][lpp]     description-head value codes, transposed
+constexpr int kTextSplitMax = 16;   // list shares of a text-row call (nomas_set_text_split bounds it too)
+
 struct WsLayout {
-    size_t kc, kt, vc, vt, kh, vht, ksl, vsl, kp, vpt, total;
+    size_t kc, kt, vc, vt, kh, vht, ksl, vsl, kp, vpt, part_o, part_ml, total;
 };
 static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
     const auto &d = c->d;
@@ -693,6 +753,8 @@ static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
     w.vsl = take((size_t)H * lhp * 4);
     w.kp = take((size_t)H * d.head_store_tokens * D * 2);
     w.vpt = take((size_t)H * D * lpp * 2);
+    w.part_o = take((size_t)kTextSplitMax * lt * H * D * 4);    // text-row partials (split calls)
+    w.part_ml = take((size_t)kTextSplitMax * H * lt * 8);
     w.total = off;
     return w;
 }
@@ -899,8 +961,36 @@ static int enqueue_run(const nomas_kv_cache *c, const nomas_segment_text *seg, c
     p.lse = lse;
     p.err = static_cast<int *>(c->buf[NOMAS_BUF_ERR]);
     p.timeout_ns = wait_limit_ns();
-    dim3 grid((unsigned)lay.n_qblocks, (unsigned)H);
-    return D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
+    // Text query rows fill few CTAs (ceil(Lt / 128) x H) and their lists differ in length (head rows see
+    // all current video, tail rows one window): each list is cut into S shares of equal length, one CTA
+    // each, merged by attn_combine_kernel.  S minimises waves x (share length + 24 tiles of fixed CTA
+    // cost) + 2 tiles of merge traffic per share, with the list capacity standing in for the length
+    // (production segment: 10 x 16 CTAs, 341 entries, S = 4; S = 3 to 5 measured within 1 %, 16 at +19 %).
+    int S = 1;
+    if (mode == NOMAS_MODE_TEXT && Lt > 0 && lay.list_cap > 0) {
+        const int64_t ctas = (int64_t)lay.n_qblocks * H, sms = sm_count(), cap = lay.list_cap;
+        int64_t best = 0;
+        for (int s = 1; s <= kTextSplitMax && s <= cap; ++s) {
+            const int64_t cost = (ctas * s + sms - 1) / sms * ((cap + s - 1) / s + 24) + 2 * s;
+            if (s == 1 || cost < best) best = cost, S = s;
+        }
+        if (text_split_setting() > 0) S = text_split_setting();
+    }
+    const int share_len = S > 1 ? (int)((lay.list_cap + S - 1) / S) : 0;
+    p.share_len = share_len;
+    p.part_o = reinterpret_cast<float *>(wsb + ws.part_o);
+    p.part_ml = reinterpret_cast<float2 *>(wsb + ws.part_ml);
+    const unsigned nz = share_len > 0 ? (unsigned)((lay.list_cap + share_len - 1) / share_len) : 1u;
+    dim3 grid((unsigned)lay.n_qblocks, (unsigned)H, nz);
+    int rc = D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
+    if (rc || share_len == 0) return rc;
+    const int64_t warps = Lt * H;
+    const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
+    if (D == 128)
+        attn_combine_kernel<128><<<blocks, 256, 0, st>>>(p.part_o, p.part_ml, p.counts, share_len, Lt, H, out, lse);
+    else
+        attn_combine_kernel<64><<<blocks, 256, 0, st>>>(p.part_o, p.part_ml, p.counts, share_len, Lt, H, out, lse);
+    return check_launch("attn_combine_kernel launch");
 }
 
 }  // namespace nomas

@@ -28,6 +28,10 @@ static std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};   // 2 s per wait
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
+static std::atomic<int> g_text_split{0};   // 0: chosen per call
+
+int text_split_setting() { return g_text_split.load(std::memory_order_relaxed); }
+
 int bind_device(const nomas_kv_cache *c) {
     int cur = -1;
     if (cudaGetDevice(&cur) == cudaSuccess && cur == c->device) return NOMAS_OK;
@@ -265,6 +269,10 @@ extern "C" const char *nomas_last_error(void) { return g_last_error; }
 
 extern "C" uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns) {
     return g_wait_limit_ns.exchange(limit_ns, std::memory_order_relaxed);
+}
+
+extern "C" int nomas_set_text_split(int shares) {
+    return g_text_split.exchange(shares >= 1 && shares <= 16 ? shares : 0, std::memory_order_relaxed);
 }
 
 extern "C" const char *nomas_status_string(int s) {

@@ -110,3 +110,14 @@ def test_linear_host_checks_without_a_device(N):
     assert N.nomas_w8_dequant(a, a, 16, 12, a) == N.NOMAS_EINVAL                         # K not a multiple of 8
     assert N.nomas_w8_quantize(0, 16, 32, 32, a, a) == N.NOMAS_EINVAL
     assert N.nomas_status_read(0) == N.NOMAS_EINVAL
+
+
+def test_text_split_setting_round_trips(N):
+    # host-side setting only: 0 = chosen per call, 1..16 forced, anything else back to 0
+    prev = N.nomas_set_text_split(3)
+    try:
+        assert N.nomas_set_text_split(17) == 3
+        assert N.nomas_set_text_split(16) == 0
+        assert N.nomas_set_text_split(-1) == 16
+    finally:
+        N.nomas_set_text_split(prev)

@@ -85,6 +85,18 @@ def test_text_rows_full_size_sampled(name):
     _run(cfg, np.asarray(sorted(rows), np.int64))
 
 
+@pytest.mark.parametrize("shares", [2, 3, 8])
+@pytest.mark.parametrize("cfg", SMALL[:2], ids=lambda c: f"T{c.tokens_per_frame}_h{c.current.head_len}")
+def test_text_rows_split_lists(cfg, shares):
+    # each key list cut into 2, 3 or 8 shares (some of them empty at this size) and merged
+    from int8_kv_cache_action_b200 import _nomas as N
+    prev = N.nomas_set_text_split(shares)
+    try:
+        _run(cfg)
+    finally:
+        N.nomas_set_text_split(prev)
+
+
 def test_video_rows_unchanged_by_a_text_call():
     # a text-mode call between two video calls leaves the video output bitwise identical
     from int8_kv_cache_action_b200.runtime import segment_text_of

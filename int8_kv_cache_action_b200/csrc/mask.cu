@@ -582,29 +582,11 @@ __device__ void write_pair_list(const MaskParams &p, int h, int pr, const uint32
     if (lane == 0) reinterpret_cast<int32_t *>(p.buf + p.lay.off_count)[hp] = n;
 }
 
-// Selection with the keys in registers: one warp per query block (eight per CTA, four CTA pairs), up to
-// 32 M candidates, M keys per lane.  Lane l starts with candidates i * 32 + l (the order does not matter:
-// every key carries its index) and the bitonic network runs on element e = l M + i, exchanging across
-// lanes by shuffles when the partner distance is M or more and inside the lane otherwise.  The first
-// `keep` elements of the ascending order are the kept candidates in rank order; then warps 0..3 write
-// the lists of the CTA's pairs.
+// Bitonic networks over the 32 M keys of a warp, element e = lane * M + i (lane l holds elements
+// l M .. l M + M - 1): partners at distance j >= M are exchanged across lanes by shuffles, closer ones
+// inside the lane.  warp_sort_up sorts ascending; warp_merge_up sorts a bitonic sequence ascending.
 template <int M>
-__global__ void __launch_bounds__(256, M >= 32 ? 1 : 2) select_lists_warp_kernel(MaskParams p) {
-    __shared__ uint32_t bits[8][M];            // kept-candidate bit mask per query block (32 M bits)
-    const int n_pairs = (p.n_qb + 1) / 2;
-    const int groups = (n_pairs + 3) / 4;
-    const int h = blockIdx.x / groups, g = blockIdx.x - h * groups;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = 8 * g + warp;                  // = 2 * (4 g + warp / 2) + warp % 2
-    const bool valid = b < p.n_qb;
-    if (lane < M) bits[warp][lane] = 0;
-    unsigned long long a[M];
-    const float *sc = reinterpret_cast<const float *>(p.buf + p.lay.off_score) + ((int64_t)h * p.n_qb + b) * p.n_cand;
-#pragma unroll
-    for (int i = 0; i < M; ++i) {
-        const int c = i * 32 + lane;
-        a[i] = (valid && c < p.n_cand) ? rank_key(sc[c], c) : ~0ull;
-    }
+__device__ __forceinline__ void warp_sort_up(unsigned long long (&a)[M], int lane) {
     for (int k = 2; k <= 32 * M; k <<= 1) {
         for (int j = k >> 1; j >= M; j >>= 1) {            // partner in lane ^ (j / M), same register
             const int lm = j / M;
@@ -629,6 +611,115 @@ __global__ void __launch_bounds__(256, M >= 32 ? 1 : 2) select_lists_warp_kernel
             }
         }
     }
+}
+
+template <int M>
+__device__ __forceinline__ void warp_merge_up(unsigned long long (&a)[M], int lane) {
+#pragma unroll
+    for (int j = 16 * M; j >= M; j >>= 1) {
+        const int lm = j / M;
+        const bool take_min = (lane & lm) == 0;
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, a[i], lm);
+            a[i] = take_min ? (o < a[i] ? o : a[i]) : (o > a[i] ? o : a[i]);
+        }
+    }
+#pragma unroll
+    for (int j = M / 2; j > 0; j >>= 1) {
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            if (i & j) continue;
+            const unsigned long long x = a[i], y = a[i ^ j];
+            a[i] = x < y ? x : y;
+            a[i ^ j] = x < y ? y : x;
+        }
+    }
+}
+
+// Selection when keep <= 128: one warp per query block keeps the 128 smallest keys (ascending) of the
+// candidates seen so far.  Candidates arrive in chunks of 128 (4 per lane, padded with the largest key);
+// a chunk is sorted, and with B its sorted keys the 128 smallest of A and B are min(A[e], B[127 - e]),
+// a bitonic sequence that one merge network sorts.  The first `keep` keys are the kept candidates in
+// rank order -- the same result as sorting every key.  Then warps 0..3 write the CTA's pair lists.
+__global__ void __launch_bounds__(256, 4) select_lists_top128_kernel(MaskParams p) {
+    __shared__ uint32_t bits[8][32];             // kept-candidate bit mask per query block (1024 bits)
+    const int n_pairs = (p.n_qb + 1) / 2;
+    const int groups = (n_pairs + 3) / 4;
+    const int h = blockIdx.x / groups, g = blockIdx.x - h * groups;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = 8 * g + warp;
+    const bool valid = b < p.n_qb;
+    uint32_t *bw = bits[warp];
+    unsigned long long a[4];
+    const float *sc = reinterpret_cast<const float *>(p.buf + p.lay.off_score) + ((int64_t)h * p.n_qb + b) * p.n_cand;
+    for (int c0 = 0; c0 < p.n_cand; c0 += 128) {
+        unsigned long long t[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int c = c0 + lane * 4 + i;
+            t[i] = (valid && c < p.n_cand) ? rank_key(sc[c], c) : ~0ull;
+        }
+        warp_sort_up<4>(t, lane);
+        if (c0 == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = t[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const unsigned long long o = __shfl_xor_sync(0xffffffffu, t[3 - i], 31);   // B[127 - e]
+                a[i] = o < a[i] ? o : a[i];
+            }
+            warp_merge_up<4>(a, lane);
+        }
+    }
+    bw[lane] = 0;
+    __syncwarp();
+    if (valid) {
+        int32_t *sel = reinterpret_cast<int32_t *>(p.buf + p.lay.off_sel) + ((int64_t)h * p.n_qb + b) * p.keep;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = lane * 4 + i;
+            if (r >= p.keep) continue;
+            const uint32_t c = (uint32_t)a[i];
+            if (c >= (uint32_t)p.n_cand) {                  // cannot happen (keep <= n_cand): record and skip
+                set_device_error(p.err, NOMAS_EDEVICE, 20);
+                continue;
+            }
+            sel[r] = (int32_t)c;
+            atomicOr(&bw[c >> 5], 1u << (c & 31));
+        }
+    }
+    __syncthreads();
+    const int pr = 4 * g + warp;
+    if (warp < 4 && pr < n_pairs)
+        write_pair_list(p, h, pr, bits[2 * warp], 2 * pr + 1 < p.n_qb ? bits[2 * warp + 1] : nullptr, lane);
+}
+
+// Selection with the keys in registers: one warp per query block (eight per CTA, four CTA pairs), up to
+// 32 M candidates, M keys per lane.  Lane l starts with candidates i * 32 + l (the order does not matter:
+// every key carries its index) and the bitonic network runs on element e = l M + i, exchanging across
+// lanes by shuffles when the partner distance is M or more and inside the lane otherwise.  The first
+// `keep` elements of the ascending order are the kept candidates in rank order; then warps 0..3 write
+// the lists of the CTA's pairs.
+template <int M>
+__global__ void __launch_bounds__(256, M >= 32 ? 1 : 2) select_lists_warp_kernel(MaskParams p) {
+    __shared__ uint32_t bits[8][M];            // kept-candidate bit mask per query block (32 M bits)
+    const int n_pairs = (p.n_qb + 1) / 2;
+    const int groups = (n_pairs + 3) / 4;
+    const int h = blockIdx.x / groups, g = blockIdx.x - h * groups;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = 8 * g + warp;                  // = 2 * (4 g + warp / 2) + warp % 2
+    const bool valid = b < p.n_qb;
+    if (lane < M) bits[warp][lane] = 0;
+    unsigned long long a[M];
+    const float *sc = reinterpret_cast<const float *>(p.buf + p.lay.off_score) + ((int64_t)h * p.n_qb + b) * p.n_cand;
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+        const int c = i * 32 + lane;
+        a[i] = (valid && c < p.n_cand) ? rank_key(sc[c], c) : ~0ull;
+    }
+    warp_sort_up<M>(a, lane);
     __syncwarp();
     if (valid) {
         int32_t *sel = reinterpret_cast<int32_t *>(p.buf + p.lay.off_sel) + ((int64_t)h * p.n_qb + b) * p.keep;
@@ -845,7 +936,8 @@ static int enqueue_mask(const MaskParams &p, float *qmean, float *kmean, cudaStr
         score_kernel<<<sg, 256, 0, st>>>(p, qmean, kmean);
         const int npow2 = pow2_at_least(p.n_cand);
         const unsigned groups = (unsigned)(((p.n_qb + 1) / 2 + 3) / 4);
-        if (npow2 <= 256) select_lists_warp_kernel<8><<<p.H * groups, 256, 0, st>>>(p);
+        if (p.keep <= 128 && p.n_cand <= 1024) select_lists_top128_kernel<<<p.H * groups, 256, 0, st>>>(p);
+        else if (npow2 <= 256) select_lists_warp_kernel<8><<<p.H * groups, 256, 0, st>>>(p);
         else if (npow2 <= 512) select_lists_warp_kernel<16><<<p.H * groups, 256, 0, st>>>(p);
         else if (npow2 <= 1024) select_lists_warp_kernel<32><<<p.H * groups, 256, 0, st>>>(p);
         else select_lists_kernel<<<p.H * ((p.n_qb + 1) / 2), 256, select_smem(npow2, p.n_cand), st>>>(p, npow2);

@@ -1,5 +1,6 @@
 """GPU parity of nomas_mask_build: tile classes (exact), sparse scores and kept blocks (bit-exact), and
 the per-CTA tile lists derived from them."""
+import dataclasses
 import numpy as np
 import pytest
 import torch
@@ -61,8 +62,14 @@ SPARSE = [small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), wi
           small_config(tokens_per_frame=97, n_frames=5, prior_frames=(4, 4), window=5, head_dim=64),
           small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), window=4, keep_frac=1.0),
           CONFIGS["C3r"], CONFIGS["C3"],
-          # 548 and 1173 candidates: the selection's register paths for up to 1024 keys and its
-          # shared-memory path beyond
+          # keep <= 128 takes the chunked top-128 selection (C3r, C3, the small shapes, and 548
+          # candidates in five chunks, the last one ragged); larger keeps the full sorts: 158
+          # candidates (keys in registers, 8 per lane), C3 at half keep (16 per lane), 548 (32 per
+          # lane) and 1173 candidates (shared memory)
+          small_config("wide", tokens_per_frame=100, n_frames=300, prior_frames=(400,), window=400, keep_frac=0.2),
+          small_config("k158", tokens_per_frame=100, n_frames=100, prior_frames=(100,), window=100, heads=2,
+                       keep_frac=0.9),
+          dataclasses.replace(CONFIGS["C3"], keep_frac=0.5, name="C3half"),
           small_config("wide", tokens_per_frame=100, n_frames=300, prior_frames=(400,), window=400),
           small_config("wider", tokens_per_frame=100, n_frames=300, prior_frames=(700, 500), window=1200, heads=1)]
 

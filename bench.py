@@ -675,7 +675,7 @@ def main():
         "attn_dense_call_tflops": dense_call_tflops, "attn_sparse_call_tflops": sparse_call_tflops,
         "attn_workspace_bytes": r["ws_bytes"],
         "roofline_linear": {
-            "bound": "tensor", "kernel": "gemm_bf16_kernel (nomas_linear_bf16; nomas_w8a16_linear adds the dequantise "
+            "bound": "tensor", "kernel": "gemm2_bf16_kernel (nomas_linear_bf16; nomas_w8a16_linear adds the dequantise "
                                         "pre-pass)",
             "peak": peak_burst, "unit": "TFLOP/s", "peak_kind": f"bf16 dense, burst ({pk_kind})",
             "shapes": {k: {"gemm_tflops": v["gemm"]["tflops"], "gemm_frac": v["gemm"]["tflops"] / peak_burst,

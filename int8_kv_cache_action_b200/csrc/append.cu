@@ -4,7 +4,7 @@
 //
 // HBM-bound: per (token, head) 2*D bf16 read, 2*D int8 + 2 fp32 written.  A persistent kernel: in
 // every CTA a producer warp keeps TMA copies of (one head x TC tokens) chunks of K and V in flight
-// through a four-stage shared-memory ring while eight consumer warps quantise the chunks already
+// through a three-stage shared-memory ring while eight consumer warps quantise the chunks already
 // landed, so loads overlap the arithmetic.  One group of D/16 lanes handles one (token, head): each
 // lane holds 16 channels of K and 16 of V, the absmax is reduced with xor-shuffles inside the group,
 // and each lane stores 16 codes.  The ring rows of the video frames and the description-head rows
@@ -100,7 +100,7 @@ constexpr int kTokBlock = 32 / (D / 16);    // tokens per warp: one token per gr
 
 constexpr int kAppendConsumers = 8;         // consumer warps; warp 8 is the producer
 constexpr int kAppendThreads = 32 * (kAppendConsumers + 1);
-constexpr int kAppendStages = 4;
+constexpr int kAppendStages = 3;          // with four CTAs per SM: 192 KB of chunks in flight per SM
 
 template <int D>
 struct AppendCfg {
@@ -144,7 +144,7 @@ __device__ __forceinline__ void chunk_of(const AppendParams &a, uint32_t c, int 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAppendThreads, 3)
+__global__ void __launch_bounds__(kAppendThreads, 4)
     quant_append_kernel(const __grid_constant__ CUtensorMap tk0, const __grid_constant__ CUtensorMap tv0,
                         const __grid_constant__ CUtensorMap tk1, const __grid_constant__ CUtensorMap tv1,
                         const AppendParams a) {
@@ -304,7 +304,7 @@ static int launch_append(const CUtensorMap *maps, const AppendParams &a, cudaStr
     if (attr != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(append smem)", (int)attr, cudaGetErrorString(attr));
     const int64_t total = a.job[0].n_chunks + a.job[1].n_chunks;
     if (total >= ((int64_t)1 << 31)) return NOMAS_EINVAL;   // chunk ids are 32-bit
-    int64_t blocks = (int64_t)sm_count() * 3;
+    int64_t blocks = (int64_t)sm_count() * 4;
     if (blocks > total) blocks = total;
     quant_append_kernel<D><<<(unsigned)blocks, kAppendThreads, C::SMEM, st>>>(maps[0], maps[1], maps[2], maps[3], a);
     return check_launch("quant_append_kernel launch");

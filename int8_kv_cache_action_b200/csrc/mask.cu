@@ -223,7 +223,7 @@ __global__ void lists_dense_kernel(MaskParams p) {
 // scale, one rounding), then divided once by the number of valid rows.  Units are dealt to CTAs
 // round-robin, blocks of q and current keys first.
 constexpr int kPoolRows = 16;       // rows per stage (bf16 stages: min(16, query rows))
-constexpr int kPoolStages = 3;
+constexpr int kPoolStages = 2;     // with three CTAs per SM (measured best of 1-3 CTAs x 2-6 stages)
 constexpr int kPoolConsumers = 4;   // warps; warp 4 is the producer
 constexpr int kPoolThreads = 32 * (kPoolConsumers + 1);
 
@@ -928,7 +928,7 @@ static int enqueue_mask(const MaskParams &p, float *qmean, float *kmean, cudaStr
     if (!sp) {
         lists_dense_kernel<<<nblk((int64_t)p.n_lists * 32, 128), 128, 0, st>>>(p);
     } else {
-        int64_t blocks = (int64_t)2 * sm_count();     // two CTAs per SM (shared memory)
+        int64_t blocks = (int64_t)3 * sm_count();     // three CTAs per SM (shared memory)
         if (blocks > pp.n_units) blocks = pp.n_units;
         if (p.D == 128) pool_kernel<128><<<(unsigned)blocks, kPoolThreads, PoolCfg<128>::SMEM, st>>>(tq, tk, p, pp);
         else pool_kernel<64><<<(unsigned)blocks, kPoolThreads, PoolCfg<64>::SMEM, st>>>(tq, tk, p, pp);

@@ -60,6 +60,8 @@ TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose 
                (os.path.join(CSRC, "append.cu"), os.path.join(CSRC, "quant.cuh"), COMMON)),
     "linear": (os.path.join(ROOT, "profiles", "gemm_dit_qkv_traffic.json"),
                (os.path.join(CSRC, "linear.cu"), os.path.join(CSRC, "quant.cuh"), COMMON)),
+    "prepare": (os.path.join(ROOT, "profiles", "prepare_production_traffic.json"),
+                (os.path.join(CSRC, "prep.cu"), os.path.join(CSRC, "prep.cuh"), COMMON)),
 }
 
 
@@ -667,7 +669,8 @@ def main():
                              "kernel": "nomas_attn_prepare (keys_f16 + values_t16 + hist_prep: INT8 history codes "
                                        "and bf16 current/text K,V widened to fp16)",
                              "achieved": prep_gbs, "peak": hbm, "unit": "GB/s", "frac": prep_gbs / hbm,
-                             "bytes_per_call": r["prep_bytes"], "ms_per_call": prep_ms, "traffic": None},
+                             "bytes_per_call": r["prep_bytes"], "ms_per_call": prep_ms,
+                             "traffic": measured_traffic("prepare")},
         "breakdown_ms": {"append": ph[0], "mask_dense": ph[1], "prepare_dense": ph[2], "attn_dense": ph[3],
                          "mask_text": ph[4], "attn_text": ph[5], "mask_sparse": ph[6], "attn_sparse": ph[7]},
         "attn_text_tflops": text_tflops,

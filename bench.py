@@ -47,10 +47,10 @@ def step_config(cfg, world):
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# Kernel launches of one step: append 1; dense mask 3; prepare 3 (key copy, transposed values, history
-# widening); dense attention 1; text mask 3; text attention 2 (the list shares, their merge); sparse
-# mask 5; sparse attention 1.
-LAUNCHES_PER_STEP = 19
+# Kernel launches of one step: append 1; dense mask 3; prepare 1 (key copy, transposed values and history
+# widening in one launch); dense attention 1; text mask 3; text attention 2 (the list shares, their
+# merge); sparse mask 5; sparse attention 1.
+LAUNCHES_PER_STEP = 17
 CSRC = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc")
 COMMON = os.path.join(CSRC, "common.cuh")
 TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose digest it was taken with)
@@ -666,7 +666,7 @@ def main():
                             "peak": hbm, "unit": "GB/s", "frac": append_gbs / hbm, "traffic": append_traffic,
                             "peak_kind": f"HBM copy ({pk_kind})"},
         "roofline_dequant": {"bound": "hbm",
-                             "kernel": "nomas_attn_prepare (keys_f16 + values_t16 + hist_prep: INT8 history codes "
+                             "kernel": "nomas_attn_prepare (prepare_kernel: INT8 history codes "
                                        "and bf16 current/text K,V widened to fp16)",
                              "achieved": prep_gbs, "peak": hbm, "unit": "GB/s", "frac": prep_gbs / hbm,
                              "bytes_per_call": r["prep_bytes"], "ms_per_call": prep_ms,

@@ -830,7 +830,6 @@ static int enqueue_prepare(const nomas_kv_cache *c, const nomas_mask_layout &lay
     const WsLayout ws = ws_layout(c, Nq, Lt);
     uint8_t *wsb = static_cast<uint8_t *>(workspace);
     int *err = static_cast<int *>(c->buf[NOMAS_BUF_ERR]);
-    int rc;
     F16Jobs jobs{};
     jobs.H = H;
     jobs.D = D;
@@ -843,7 +842,6 @@ static int enqueue_prepare(const nomas_kv_cache *c, const nomas_mask_layout &lay
     if (Lt > 0)
         jobs.job[jobs.n_jobs++] =
             F16Job{static_cast<const __nv_bfloat16 *>(ktxt), reinterpret_cast<__half *>(wsb + ws.kt), Lt};
-    if ((rc = launch_keys_f16(jobs, st))) return rc;
 
     VtJobs vj{};
     vj.H = H;
@@ -854,7 +852,6 @@ static int enqueue_prepare(const nomas_kv_cache *c, const nomas_mask_layout &lay
     vj.job[0] = VtJob{static_cast<const __nv_bfloat16 *>(vcur), reinterpret_cast<__half *>(wsb + ws.vc), Nq, nqp};
     vj.job[1] = VtJob{static_cast<const __nv_bfloat16 *>(Lt > 0 ? vtxt : vcur), reinterpret_cast<__half *>(wsb + ws.vt),
                       Lt, ltp};
-    if ((rc = launch_values_t16(vj, Lt > 0, nqp > ltp ? nqp : ltp, st))) return rc;
 
     if (Lh > 0 || Lp > 0) {
         const HistView hv = hist_view(c);
@@ -882,9 +879,9 @@ static int enqueue_prepare(const nomas_kv_cache *c, const nomas_mask_layout &lay
         hp.head_rows = d.head_store_tokens;
         hp.H = H;
         hp.D = D;
-        if ((rc = launch_hist_prep(hp, st))) return rc;
+        return launch_prepare(jobs, vj, Lt > 0, nqp > ltp ? nqp : ltp, &hp, st);
     }
-    return NOMAS_OK;
+    return launch_prepare(jobs, vj, Lt > 0, nqp > ltp ? nqp : ltp, nullptr, st);
 }
 
 // The attention kernel over a prepared workspace.

@@ -26,11 +26,11 @@ __device__ __forceinline__ void i8x16_to_f16(const uint4 &w, uint4 &lo, uint4 &h
 
 // bf16 [n][H][D] (token / head strides in elements) -> fp16 [H][n][D], for up to two tensors.  One
 // block converts 64 tokens x D of one head (a contiguous 64 x D run of the destination).
-__global__ void __launch_bounds__(256) keys_f16_kernel(F16Jobs jobs) {
-    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *jobs.hdr_dst = jobs.hdr;
-    const F16Job J = blockIdx.z ? jobs.job[1] : jobs.job[0];
-    const int h = blockIdx.y;
-    const int64_t t0 = (int64_t)blockIdx.x * 64;
+__device__ __forceinline__ void keys_f16_block(const F16Jobs &jobs, const uint3 blk) {
+    if (blk.x == 0 && blk.y == 0 && blk.z == 0 && threadIdx.x == 0) *jobs.hdr_dst = jobs.hdr;
+    const F16Job J = blk.z ? jobs.job[1] : jobs.job[0];
+    const int h = blk.y;
+    const int64_t t0 = (int64_t)blk.x * 64;
     if (t0 >= J.n) return;
     const int cpr = jobs.D / 8;   // 16-byte chunks per row
     const int rows = J.n - t0 < 64 ? (int)(J.n - t0) : 64;
@@ -53,11 +53,11 @@ __global__ void __launch_bounds__(256) keys_f16_kernel(F16Jobs jobs) {
 // row writes stay contiguous, and a warp reading one word of 8 tokens spaced 8 apart for 4
 // adjacent words hits 32 distinct banks.  Each thread then emits 8 tokens of two channel rows.
 
-__global__ void __launch_bounds__(256) values_t16_kernel(VtJobs jobs) {
-    __shared__ __align__(16) uint32_t tile[64 * 64];   // [token][word], D / 2 words per token used
-    const VtJob J = blockIdx.z ? jobs.job[1] : jobs.job[0];
-    const int h = blockIdx.y;
-    const int64_t t0 = (int64_t)blockIdx.x * 64;
+__device__ __forceinline__ void values_t16_block(const VtJobs &jobs, const uint3 blk, uint32_t *tile) {
+    // tile: [token][word] (64 x 64 words), D / 2 words per token used
+    const VtJob J = blk.z ? jobs.job[1] : jobs.job[0];
+    const int h = blk.y;
+    const int64_t t0 = (int64_t)blk.x * 64;
     if (t0 >= J.np) return;
     const int D = jobs.D;
     const int W = D / 2;                  // words per token row
@@ -101,12 +101,11 @@ __global__ void __launch_bounds__(256) values_t16_kernel(VtJobs jobs) {
 //          read in place).
 // One block converts 64 tokens x D of one head; values are transposed through shared memory.
 
-__global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
-    __shared__ __align__(16) int8_t tile[64][128 + 16];
-    const bool heads = blockIdx.z == 1;
-    const int h = blockIdx.y;
+__device__ __forceinline__ void hist_prep_block(const HistPrep &P, const uint3 blk, int8_t (*tile)[128 + 16]) {
+    const bool heads = blk.z == 1;
+    const int h = blk.y;
     const int64_t n = heads ? P.Lp : P.Lh, np = heads ? P.lpp : P.lhp;
-    const int64_t t0 = (int64_t)blockIdx.x * 64;
+    const int64_t t0 = (int64_t)blk.x * 64;
     if (t0 >= np) return;
     const int D = P.D;
     const int cpr = D / 16;
@@ -169,28 +168,48 @@ __global__ void __launch_bounds__(256) hist_prep_kernel(HistPrep P) {
     }
 }
 
-int launch_keys_f16(const F16Jobs &jobs, cudaStream_t st) {
+// The three copies of a call in one launch: blocks [0, n_k) convert keys, [n_k, n_k + n_v) transpose
+// values, the rest widen the history and the description heads; every block is independent, so the
+// block scheduler interleaves them and no copy waits for another's tail.
+struct PrepGrid {
+    dim3 k, v, h;       // the grid of each part (zero blocks: part absent)
+    uint32_t n_k, n_v;  // blocks of the first two parts
+};
+
+__device__ __forceinline__ uint3 block_of(uint32_t b, const dim3 &g) {
+    return make_uint3(b % g.x, (b / g.x) % g.y, b / (g.x * g.y));
+}
+
+__global__ void __launch_bounds__(256) prepare_kernel(const F16Jobs fj, const VtJobs vj, const HistPrep hp,
+                                                      const PrepGrid g) {
+    __shared__ __align__(16) uint32_t smem[64 * 64];   // the value transpose tile or the history tile
+    const uint32_t b = blockIdx.x;
+    if (b < g.n_k) {
+        keys_f16_block(fj, block_of(b, g.k));
+    } else if (b < g.n_k + g.n_v) {
+        values_t16_block(vj, block_of(b - g.n_k, g.v), smem);
+    } else {
+        static_assert(64 * (128 + 16) <= 64 * 64 * 4, "the history tile fits");
+        hist_prep_block(hp, block_of(b - g.n_k - g.n_v, g.h), reinterpret_cast<int8_t (*)[128 + 16]>(smem));
+    }
+}
+
+int launch_prepare(const F16Jobs &fj, const VtJobs &vj, bool two, int64_t max_np, const HistPrep *hp, cudaStream_t st) {
+    PrepGrid g{};
     int64_t nmax = 0;
-    for (int j = 0; j < jobs.n_jobs; ++j) nmax = jobs.job[j].n > nmax ? jobs.job[j].n : nmax;
-    const dim3 grid((unsigned)((nmax + 63) / 64), (unsigned)jobs.H, (unsigned)jobs.n_jobs);
-    if (grid.x == 0 || grid.z == 0) return NOMAS_OK;
-    keys_f16_kernel<<<grid, 256, 0, st>>>(jobs);
-    return check_launch("keys_f16_kernel launch");
-}
-
-int launch_values_t16(const VtJobs &jobs, bool two, int64_t max_np, cudaStream_t st) {
-    const dim3 grid((unsigned)((max_np + 63) / 64), (unsigned)jobs.H, two ? 2u : 1u);
-    if (grid.x == 0) return NOMAS_OK;
-    values_t16_kernel<<<grid, 256, 0, st>>>(jobs);
-    return check_launch("values_t16_kernel launch");
-}
-
-int launch_hist_prep(const HistPrep &P, cudaStream_t st) {
-    const int64_t nmax = P.lhp > P.lpp ? P.lhp : P.lpp;
-    const dim3 grid((unsigned)((nmax + 63) / 64), (unsigned)P.H, 2u);
-    if (grid.x == 0) return NOMAS_OK;
-    hist_prep_kernel<<<grid, 256, 0, st>>>(P);
-    return check_launch("hist_prep_kernel launch");
+    for (int j = 0; j < fj.n_jobs; ++j) nmax = fj.job[j].n > nmax ? fj.job[j].n : nmax;
+    g.k = dim3((unsigned)((nmax + 63) / 64), (unsigned)fj.H, (unsigned)fj.n_jobs);
+    g.v = dim3((unsigned)((max_np + 63) / 64), (unsigned)vj.H, two ? 2u : 1u);
+    const int64_t hmax = hp ? (hp->lhp > hp->lpp ? hp->lhp : hp->lpp) : 0;
+    g.h = dim3((unsigned)((hmax + 63) / 64), hp ? (unsigned)hp->H : 0u, 2u);
+    const int64_t nk = (int64_t)g.k.x * g.k.y * g.k.z, nv = (int64_t)g.v.x * g.v.y * g.v.z;
+    const int64_t nh = (int64_t)g.h.x * g.h.y * g.h.z;
+    if (nk + nv + nh >= ((int64_t)1 << 31)) return NOMAS_EINVAL;
+    g.n_k = (uint32_t)nk;
+    g.n_v = (uint32_t)nv;
+    if (nk + nv + nh == 0) return NOMAS_OK;
+    prepare_kernel<<<(unsigned)(nk + nv + nh), 256, 0, st>>>(fj, vj, hp ? *hp : HistPrep{}, g);
+    return check_launch("prepare_kernel launch");
 }
 
 }  // namespace nomas

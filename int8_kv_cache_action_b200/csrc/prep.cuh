@@ -38,7 +38,7 @@ struct VtJobs {
 };
 
 // INT8 ring rows of the retained history (age order) and description-head rows -> fp16 codes; see
-// hist_prep_kernel.
+// the history part of prepare_kernel.
 struct HistPrep {
     const int8_t *k8, *v8, *hk8, *hv8;
     const float *ks, *vs;
@@ -51,9 +51,8 @@ struct HistPrep {
     int *err;                 // device error word: NOMAS_ERANGE for a value scale above kMaxValueScale
 };
 
-// Each enqueues one kernel on `st` and returns NOMAS_OK or the launch error.
-int launch_keys_f16(const F16Jobs &jobs, cudaStream_t st);
-int launch_values_t16(const VtJobs &jobs, bool two, int64_t max_np, cudaStream_t st);
-int launch_hist_prep(const HistPrep &P, cudaStream_t st);
+// One launch for the three copies of a call (keys, transposed values, and -- when hp is not null -- the
+// retained history and the description heads); returns NOMAS_OK or the launch error.
+int launch_prepare(const F16Jobs &fj, const VtJobs &vj, bool two, int64_t max_np, const HistPrep *hp, cudaStream_t st);
 
 }  // namespace nomas

@@ -55,7 +55,7 @@ CSRC = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc")
 COMMON = os.path.join(CSRC, "common.cuh")
 TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose digest it was taken with)
     "attn": (os.path.join(ROOT, "profiles", "attn_dense_production_traffic.json"),
-             (os.path.join(CSRC, "attn.cu"), COMMON)),
+             (os.path.join(CSRC, "attn_pair.cu"), os.path.join(CSRC, "attn.cuh"), COMMON)),
     "append": (os.path.join(ROOT, "profiles", "append_production_traffic.json"),
                (os.path.join(CSRC, "append.cu"), os.path.join(CSRC, "quant.cuh"), COMMON)),
     "linear": (os.path.join(ROOT, "profiles", "gemm_dit_qkv_traffic.json"),
@@ -578,6 +578,8 @@ def main():
                     help="print one line per config (attention call and append) instead of the step line")
     ap.add_argument("--only", default="", help="with --per-config: comma-separated config names (C0..C4, C3r)")
     ap.add_argument("--reps", type=int, default=0, help="with --per-config: timed calls per config")
+    ap.add_argument("--attn-kernel", type=int, default=0,
+                    help="head_dim-128 attention kernel: 0 chosen per call, 1 one query block per CTA, 2 block pairs")
     ap.add_argument("--linear-only", action="store_true",
                     help="print one line with the INT8-weight linear layer on the DiT shapes only")
     args = ap.parse_args()
@@ -606,6 +608,9 @@ def main():
         print(json.dumps(line))
         return
 
+    if args.attn_kernel:
+        from int8_kv_cache_action_b200 import _nomas as N
+        N.nomas_set_attn_kernel(args.attn_kernel)
     if args.per_config:
         per_config(args)
         return
@@ -657,7 +662,7 @@ def main():
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": step_config(cfg, world),
         "roofline": {"bound": "tensor",
-                     "kernel": "attn_fwd_kernel<128> (nomas_attn_run, dense)",
+                     "kernel": "attn_pair_kernel (nomas_attn_run, dense: one CTA per query-block pair)",
                      "achieved": dense_tflops,
                      "peak": peak_burst, "unit": "TFLOP/s", "frac": dense_tflops / peak_burst,
                      "peak_kind": f"bf16 dense, burst ({pk_kind}): the kernel runs {ph[3]:.2f} ms at a time",

@@ -398,6 +398,17 @@ uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns);
  * values select the default.  Process-wide, applies to later calls; returns the previous setting. */
 int nomas_set_text_split(int shares);
 
+/* Tuning and test hook: which attention kernel nomas_attn_run uses at head_dim 128.  0 (default): one
+ * CTA per pair of 128-row query blocks that share a tile list for NOMAS_MODE_DENSE when the pairs fill
+ * the SMs in fewer waves of work (the two blocks' softmax warps alternate on the tensor pipe, and each
+ * K / V^T tile is staged once for both), else and for the sparse and text-row modes (whose two blocks
+ * share fewer tiles) one CTA per query block; 1: one CTA per
+ * query block in every mode (the kernel head_dim 64 always uses); 2: block pairs in every mode.  All
+ * compute the same function (same operand precision and softmax arithmetic; results agree up to the
+ * order of the fp32 row-sum additions).  Other values select 0.  Process-wide, applies to later
+ * calls; returns the previous setting. */
+int nomas_set_attn_kernel(int which);
+
 #ifdef __cplusplus
 }
 #endif

@@ -30,7 +30,7 @@ EXPORTED = ["nomas_kv_cache_bytes", "nomas_kv_cache_init", "nomas_kv_cache_destr
             "nomas_kv_append", "nomas_mask_layout_query", "nomas_mask_bytes", "nomas_mask_build",
             "nomas_attn_fwd", "nomas_kv_dequant", "nomas_device_status", "nomas_status_string",
             "nomas_last_error", "nomas_mask_build_static", "nomas_attn_workspace_bytes",
-            "nomas_set_wait_limit_ns", "nomas_set_text_split", "nomas_attn_prepare", "nomas_attn_run", "nomas_kv_frame_record_bytes",
+            "nomas_set_wait_limit_ns", "nomas_set_text_split", "nomas_set_attn_kernel", "nomas_attn_prepare", "nomas_attn_run", "nomas_kv_frame_record_bytes",
             "nomas_kv_retained", "nomas_kv_evicted_by", "nomas_kv_archive", "nomas_kv_select",
             "nomas_w8_quantize", "nomas_w8_dequant", "nomas_linear_bf16", "nomas_w8a16_workspace_bytes",
             "nomas_w8a16_linear", "nomas_status_read"]
@@ -100,6 +100,7 @@ _sigs = {
     "nomas_last_error": (ctypes.c_char_p, []),
     "nomas_set_wait_limit_ns": (ctypes.c_uint64, [ctypes.c_uint64]),
     "nomas_set_text_split": (ctypes.c_int, [ctypes.c_int]),
+    "nomas_set_attn_kernel": (ctypes.c_int, [ctypes.c_int]),
     "nomas_w8_quantize": (ctypes.c_int, [_p, _i64, _i64, _i64, _p, _p, _p]),
     "nomas_w8_dequant": (ctypes.c_int, [_p, _p, _i64, _i64, _p, _p]),
     "nomas_linear_bf16": (ctypes.c_int, [_p, _i64, _i64, _i64, _p, _i64, _i64, _p, _i64, ctypes.c_int, _p, _p]),
@@ -142,6 +143,12 @@ def nomas_set_wait_limit_ns(limit_ns: int) -> int:
 def nomas_set_text_split(shares: int) -> int:
     """Set the share count of text-row calls (0 = chosen per call, 1..16 forced); returns the previous one."""
     return int(lib.nomas_set_text_split(int(shares)))
+
+
+def nomas_set_attn_kernel(which: int) -> int:
+    """Choose the head_dim-128 attention kernel (0 = per call: block pairs for dense video rows, 1 = one
+    block per CTA, 2 = block pairs); returns the previous choice."""
+    return int(lib.nomas_set_attn_kernel(int(which)))
 
 
 def make_dims(heads, head_dim, tokens_per_frame, window_frames, capacity_frames, head_store_tokens):

@@ -47,6 +47,7 @@
 #include <cstdio>
 #include <cuda_fp16.h>
 
+#include "attn.cuh"
 #include "common.cuh"
 #include "prep.cuh"
 
@@ -57,7 +58,6 @@ constexpr int kWarpCi = 8, kWarpMma = 12, kWarpTma = 13;  // column info: warps 
 constexpr int kRegSoftmax = 168, kRegLoader = 112, kRegMma = 64;
 static_assert(2 * kRegSoftmax + kRegLoader + kRegMma == 4 * 128, "register split must equal the launch total");
 constexpr int kNCI = 4;                     // column-info ring depth
-constexpr float kRescaleThreshold = 6.0f;   // log2 units: P <= 64
 constexpr uint32_t kTmQ = 0, kTmS = 128, kTmO = 384;
 
 template <int D>
@@ -82,113 +82,6 @@ struct AttnCfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int SMEM = BYTES + 1024;              // slack for 1024-byte alignment
-};
-
-struct AttnParams {
-    const float *ksl, *vsl;     // retained-history scales in age order, [H][hist_stride]
-    const float *hks, *hvs;     // description-head scales, [H][head_rows]
-    int64_t hist_stride, head_rows;
-    // mask buffer
-    const uint8_t *mask;
-    const int4 *lists;
-    const int32_t *counts;
-    const int2 *txtwin;         // per text token: frame window (tails) or [0, kAlwaysHi) (head)
-    MaskHeader expect;
-    const WsHeader *ws_hdr;     // written by nomas_attn_prepare
-    WsHeader ws_expect;
-    int32_t sparse;
-    int32_t text_rows;          // query rows are the current text (NOMAS_MODE_TEXT), else the video
-    int32_t head_len;           // description-head tokens at the front of the current text
-    int32_t n_pairs;
-    // queries and shapes
-    const __nv_bfloat16 *q;
-    int64_t tok_stride, head_stride;
-    int32_t H, T;
-    FastDiv divT;               // token -> frame (every token index here is below 2^31)
-    int64_t Nq;
-    float scale_log2;           // softmax_scale * log2(e)
-    float *out;
-    float *lse;
-    int *err;
-    uint64_t timeout_ns;
-    // text query rows: each list cut into shares of share_len entries, share blockIdx.z per CTA, which
-    // writes its O without normalisation and (offset, row sum) per row for attn_combine_kernel;
-    // share_len == 0: the whole list, normalised output
-    int32_t share_len;
-    float *part_o;              // [share][Nq][H][D]
-    float2 *part_ml;            // [share][H][Nq]
-};
-
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// 2^x for x <= 6 on the FMA pipe (the MUFU unit's exponential throughput equals the tensor pipe's
-// rate per score at head_dim 128, so part of the exponentials are taken off it): x is clamped at -125,
-// n = rint(x) by the 1.5 * 2^23 add, f = x - n lies in [-1/2, 1/2], 2^f comes from a degree-3
-// polynomial fitted by weighted least squares to the relative error on Chebyshev nodes (maximum
-// relative error 7.5e-5, below fp16's half unit in the last place, 2^-12), and n is added to the
-// exponent field.
-__device__ __forceinline__ float2 exp2_poly(float2 x) {
-    x.x = fmaxf(x.x, -125.0f);
-    x.y = fmaxf(x.y, -125.0f);
-    const float2 t = __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
-    const float2 n = __fadd2_rn(t, make_float2(-12582912.0f, -12582912.0f));
-    const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
-    float2 q = __ffma2_rn(make_float2(0.055171605f, 0.055171605f), f, make_float2(0.24261111f, 0.24261111f));
-    q = __ffma2_rn(q, f, make_float2(0.69326097f, 0.69326097f));
-    q = __ffma2_rn(q, f, make_float2(0.99992806f, 0.99992806f));
-    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
-                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
-}
-
-#ifndef NOMAS_POLY_PAIRS
-#define NOMAS_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = NOMAS_POLY_PAIRS;   // of every 16 column pairs, this many take exp2_poly
-
-__device__ __forceinline__ float max3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-template <int N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
-__device__ __forceinline__ bool is_cached(int kind) { return kind == kKindHist || kind == kKindPriorHead; }
-
-// Walks a CTA's tile list, each entry loaded two entries ahead of its use.
-struct ListCursor {
-    const int4 *list;
-    int n, j;
-    int4 a, b;
-    __device__ __forceinline__ ListCursor(const int4 *l, int n_) : list(l), n(n_), j(0) {
-        a = n > 0 ? list[0] : make_int4(0, 0, 0, 0);
-        b = n > 1 ? list[1] : make_int4(0, 0, 0, 0);
-    }
-    // the next entry carrying `bit`; false at the end of the list
-    __device__ __forceinline__ bool next(int bit, int4 &e) {
-        while (j < n) {
-            const int4 c = a;
-            a = b;
-            b = (j + 2 < n) ? list[j + 2] : make_int4(0, 0, 0, 0);
-            ++j;
-            if (c.x & bit) {
-                e = c;
-                return true;
-            }
-        }
-        return false;
-    }
 };
 
 template <int D>
@@ -297,53 +190,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         setmaxnreg_dec<kRegLoader>();
         wd.where = 3;
         const int t = threadIdx.x - 32 * kWarpCi;   // 0..127
-        struct ColInfo {
-            float ks, vs;   // raw key / value scale (cached tiles), 1 / 0 otherwise
-            VisCode w;      // visibility code of the key (masked tiles only)
-            bool masked;    // the softmax reads the codes of this tile
-        };
-        // Column info of a tile (key scale, value scale, visibility code), loaded one tile ahead of its
-        // use: only loads happen here, so nothing waits for them until the next tile consumes them.
-        auto col_info = [&](const int4 &e, int col) -> ColInfo {
-            ColInfo ci{0.0f, 0.0f, key_none(), (e.x & mask_bit) != 0};
-            const int kind = e.x & 3;
-            const int64_t start = e.y;
-            if (col < e.z) {
-                if (!ci.masked) {
-                    // codes unused: the whole tile is visible to every row of the block
-                } else if (kind == kKindText) {
-                    if (start + col < p.head_len) {
-                        ci.w = key_always();
-                    } else {
-                        const int2 w = p.txtwin[start + col];
-                        ci.w = key_tail(w.x, w.y);
-                    }
-                } else if (kind == kKindCur) {
-                    ci.w = key_video((int)fdiv((uint32_t)(start + col), p.divT));
-                } else {
-                    ci.w = key_always();
-                }
-                if (is_cached(kind)) {
-                    const bool hist = kind == kKindHist;
-                    const int64_t i = (int64_t)h * (hist ? p.hist_stride : p.head_rows) + start + col;
-                    ci.ks = __ldg((hist ? p.ksl : p.hks) + i);
-                    ci.vs = __ldg((hist ? p.vsl : p.hvs) + i);
-                } else {
-                    ci.ks = 1.0f;
-                }
-            }
-            return ci;
-        };
         ListCursor cursor(list, n_tiles);
         int u = 0;                          // index among this block's tiles
         int4 en;
         bool have = cursor.next(use_bit, en);
         ColInfo nxt0;
-        if (have) nxt0 = col_info(en, t);
+        if (have) nxt0 = column_info(p, h, en, t, (en.x & mask_bit) != 0);
         while (have) {
             const ColInfo c0 = nxt0;
             have = cursor.next(use_bit, en);
-            if (have) nxt0 = col_info(en, t);
+            if (have) nxt0 = column_info(p, h, en, t, (en.x & mask_bit) != 0);
             const int ci = u % kNCI;
             if (!__all_sync(0xffffffffu, mbar_wait(&ci_empty[ci], ((u / kNCI) & 1) ^ 1, wd, 1))) break;
             sCS[ci * 128 + t] = p.scale_log2 * c0.ks;
@@ -978,8 +834,23 @@ static int enqueue_run(const nomas_kv_cache *c, const nomas_segment_text *seg, c
     p.part_o = reinterpret_cast<float *>(wsb + ws.part_o);
     p.part_ml = reinterpret_cast<float2 *>(wsb + ws.part_ml);
     const unsigned nz = share_len > 0 ? (unsigned)((lay.list_cap + share_len - 1) / share_len) : 1u;
-    dim3 grid((unsigned)lay.n_qblocks, (unsigned)H, nz);
-    int rc = D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
+    // head_dim 128 video rows (dense mode): one CTA per query-block pair (attn_pair_kernel) when that takes
+    // fewer SM-waves of work: a pair CTA runs about 1.6 times as long as a block CTA on the same list
+    // (measured per list entry: 4570 cycles for the pair's two blocks, 2900 for one block), so few,
+    // partly filled waves favour blocks (480 x 832: 3 block waves against 2 pair waves).  The sparse
+    // and text-row lists of a pair's two blocks overlap less (each block keeps its own candidates, and
+    // text lists are cut into shares): one CTA per block.  nomas_set_attn_kernel overrides the choice.
+    const int choice = attn_kernel_setting();
+    bool pair = D == 128 && choice == 2;
+    if (D == 128 && choice == 0 && mode == NOMAS_MODE_DENSE) {
+        const int64_t sms = sm_count();
+        const int64_t wb = ((int64_t)lay.n_qblocks * H + sms - 1) / sms;
+        const int64_t wp = ((int64_t)p.n_pairs * H + sms - 1) / sms;
+        pair = 16 * wp < 10 * wb;
+    }
+    dim3 grid(pair ? (unsigned)p.n_pairs : (unsigned)lay.n_qblocks, (unsigned)H, nz);
+    int rc = pair ? launch_attn_pair(p, grid, maps, st)
+             : D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
     if (rc || share_len == 0) return rc;
     const int64_t warps = Lt * H;
     const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);

@@ -31,6 +31,8 @@ uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed
 static std::atomic<int> g_text_split{0};   // 0: chosen per call
 
 int text_split_setting() { return g_text_split.load(std::memory_order_relaxed); }
+static std::atomic<int> g_attn_kernel{0};   // 0: chosen per call, 1: one block per CTA, 2: block pairs
+int attn_kernel_setting() { return g_attn_kernel.load(std::memory_order_relaxed); }
 
 int bind_device(const nomas_kv_cache *c) {
     int cur = -1;
@@ -273,6 +275,10 @@ extern "C" uint64_t nomas_set_wait_limit_ns(uint64_t limit_ns) {
 
 extern "C" int nomas_set_text_split(int shares) {
     return g_text_split.exchange(shares >= 1 && shares <= 16 ? shares : 0, std::memory_order_relaxed);
+}
+
+extern "C" int nomas_set_attn_kernel(int which) {
+    return g_attn_kernel.exchange(which == 1 || which == 2 ? which : 0, std::memory_order_relaxed);
 }
 
 extern "C" const char *nomas_status_string(int s) {

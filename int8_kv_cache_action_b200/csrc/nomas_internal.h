@@ -178,5 +178,6 @@ bool make_tensor_map_3d(CUtensorMap *m, CUtensorMapDataType dt, const void *base
 // Number of SMs of the current device (queried once per device).
 int sm_count();
 int text_split_setting();   // nomas_set_text_split: 0 = chosen per call, else 1..16
+int attn_kernel_setting();  // nomas_set_attn_kernel: 0 = chosen per call, 1 = one block per CTA, 2 = block pairs
 
 }  // namespace nomas

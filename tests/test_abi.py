@@ -121,3 +121,15 @@ def test_text_split_setting_round_trips(N):
         assert N.nomas_set_text_split(-1) == 16
     finally:
         N.nomas_set_text_split(prev)
+
+
+def test_attn_kernel_setting_round_trips(N):
+    # host-only setter: no GPU needed
+    prev = N.nomas_set_attn_kernel(1)
+    try:
+        assert N.nomas_set_attn_kernel(2) == 1
+        assert N.nomas_set_attn_kernel(7) == 2
+        assert N.nomas_set_attn_kernel(0) == 0
+        assert N.nomas_set_attn_kernel(-3) == 0
+    finally:
+        N.nomas_set_attn_kernel(prev)

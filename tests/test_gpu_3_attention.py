@@ -67,7 +67,7 @@ SMALL_DENSE = [
 
 
 @pytest.mark.parametrize("cfg", SMALL_DENSE, ids=lambda c: f"{c.name}_d{c.head_dim}_T{c.tokens_per_frame}_F{c.current.n_frames}")
-def test_dense_small_all_rows(cfg):
+def test_dense_small_all_rows(cfg, attn_kernel):
     _check(cfg)
 
 
@@ -76,11 +76,11 @@ SMALL_SPARSE = [small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 
 
 
 @pytest.mark.parametrize("cfg", SMALL_SPARSE, ids=lambda c: f"{c.name}_d{c.head_dim}_T{c.tokens_per_frame}")
-def test_sparse_small_all_rows(cfg):
+def test_sparse_small_all_rows(cfg, attn_kernel):
     _check(cfg, mode=1)
 
 
-def test_sparse_full_keep_equals_dense_bitwise():
+def test_sparse_full_keep_equals_dense_bitwise(attn_kernel):
     cfg = small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), window=4)
     inp = make_inputs(cfg)
     gc = gpu_cache(cfg, inp)
@@ -89,7 +89,7 @@ def test_sparse_full_keep_equals_dense_bitwise():
     assert torch.equal(dense, full) and torch.equal(dl, fl)
 
 
-def test_masked_tail_keys_contribute_exactly_nothing():
+def test_masked_tail_keys_contribute_exactly_nothing(attn_kernel):
     # rows outside a tail's window must not change at all when that tail's K/V change
     cfg = small_config(tokens_per_frame=70, n_frames=5, tails=((64, 0, 1), (100, 1, 4), (5, 4, 5), (130, 2, 3)))
     inp = make_inputs(cfg)
@@ -105,7 +105,7 @@ def test_masked_tail_keys_contribute_exactly_nothing():
     assert (base[~outside] - pert[~outside]).abs().max() > 1e-3
 
 
-def test_deterministic():
+def test_deterministic(attn_kernel):
     cfg = small_config()
     inp = make_inputs(cfg)
     gc = gpu_cache(cfg, inp)
@@ -173,3 +173,24 @@ def test_prepare_then_run_equals_fwd_and_a_stale_workspace_is_reported():
     fresh, _ = gc.build_mask(seg)
     out = run(ws, fresh)                                            # prepared before the append
     assert gc.status() == N.NOMAS_EDEVICE and bool((out == -7.0).all())
+
+
+@pytest.mark.parametrize("name,mode", [("C1", 0), ("C3r", 1), ("C2", 0)])
+def test_pair_and_block_kernels_agree(name, mode):
+    # the two head_dim-128 kernels compute the same function: same fp16 operands and softmax arithmetic,
+    # only the order of the row sum's fp32 additions differs (one rounding per tile and partial sum:
+    # a few hundred tiles x 2^-24 relative bounds the difference of ln l near 1e-4)
+    from int8_kv_cache_action_b200 import _nomas as N
+    cfg = CONFIGS[name]
+    inp = make_inputs(cfg)
+    gc = gpu_cache(cfg, inp)
+    prev = N.nomas_set_attn_kernel(2)
+    try:
+        a, la, _, _ = _run(cfg, inp, gc, mode)
+        N.nomas_set_attn_kernel(1)
+        b, lb, _, _ = _run(cfg, inp, gc, mode)
+    finally:
+        N.nomas_set_attn_kernel(prev)
+    assert gc.status() == 0
+    assert (a - b).abs().max().item() <= 1e-5 * max(1.0, b.abs().max().item())
+    assert (la - lb).abs().max().item() <= 1e-4

@@ -71,7 +71,7 @@ def _run(cfg, rows=None):
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: f"T{c.tokens_per_frame}_d{c.head_dim}_h{c.current.head_len}")
-def test_text_rows_small_all_rows(cfg):
+def test_text_rows_small_all_rows(cfg, attn_kernel):
     _run(cfg)
 
 
@@ -87,7 +87,7 @@ def test_text_rows_full_size_sampled(name):
 
 @pytest.mark.parametrize("shares", [2, 3, 8])
 @pytest.mark.parametrize("cfg", SMALL[:2], ids=lambda c: f"T{c.tokens_per_frame}_h{c.current.head_len}")
-def test_text_rows_split_lists(cfg, shares):
+def test_text_rows_split_lists(cfg, shares, attn_kernel):
     # each key list cut into 2, 3 or 8 shares (some of them empty at this size) and merged
     from int8_kv_cache_action_b200 import _nomas as N
     prev = N.nomas_set_text_split(shares)

@@ -532,30 +532,9 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const float *part_o, 
     const int64_t row = w / H;
     const int h = (int)(w - row * H);
     const int n_share = (counts[row >> 8] + share_len - 1) / share_len;   // list of the block pair
-    float M = -INFINITY;
-    for (int s = 0; s < n_share; ++s) {
-        const float2 ml = part_ml[((int64_t)s * H + h) * Nq + row];
-        if (ml.y > 0.0f) M = fmaxf(M, ml.x);
-    }
-    constexpr int PL = D / 32;
-    float acc[PL];
-#pragma unroll
-    for (int i = 0; i < PL; ++i) acc[i] = 0.0f;
-    float L = 0.0f;
-    for (int s = 0; s < n_share; ++s) {
-        const float2 ml = part_ml[((int64_t)s * H + h) * Nq + row];
-        if (!(ml.y > 0.0f)) continue;
-        const float wgt = exp2f(ml.x - M);
-        L += ml.y * wgt;
-        const float *src = part_o + (((int64_t)s * Nq + row) * H + h) * D;
-#pragma unroll
-        for (int i = 0; i < PL; ++i) acc[i] += src[lane + 32 * i] * wgt;
-    }
-    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-    float *dst = out + (row * H + h) * (int64_t)D;
-#pragma unroll
-    for (int i = 0; i < PL; ++i) dst[lane + 32 * i] = acc[i] * inv;
-    if (lse && lane == 0) lse[(int64_t)h * Nq + row] = (M + log2f(L)) * 0.69314718055994530942f;
+    merge_shares<D>(part_o + (row * H + h) * (int64_t)D, Nq * H * (int64_t)D, part_ml + (int64_t)h * Nq + row,
+                    (int64_t)H * Nq, n_share, out + (row * H + h) * (int64_t)D, lse ? lse + (int64_t)h * Nq + row : nullptr,
+                    lane);
 }
 }  // namespace nomas
 
@@ -582,9 +561,10 @@ static int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 //   kp       fp16 [H][Lp][D]      description-head key codes
 //   vpt      fp16 [H][D][lpp]     description-head value codes, transposed
 constexpr int kTextSplitMax = 16;   // list shares of a text-row call (nomas_set_text_split bounds it too)
+constexpr int kTailCtasMax = 256;   // CTAs of the split last wave of a dense pair-kernel call
 
 struct WsLayout {
-    size_t kc, kt, vc, vt, kh, vht, ksl, vsl, kp, vpt, part_o, part_ml, total;
+    size_t kc, kt, vc, vt, kh, vht, ksl, vsl, kp, vpt, part_o, part_ml, tail_o, tail_ml, total;
 };
 static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
     const auto &d = c->d;
@@ -611,6 +591,8 @@ static WsLayout ws_layout(const nomas_kv_cache *c, int64_t nq, int64_t lt) {
     w.vpt = take((size_t)H * D * lpp * 2);
     w.part_o = take((size_t)kTextSplitMax * lt * H * D * 4);    // text-row partials (split calls)
     w.part_ml = take((size_t)kTextSplitMax * H * lt * 8);
+    w.tail_o = take((size_t)kTailCtasMax * 2 * kTile * D * 4);    // split last wave (dense pair kernel)
+    w.tail_ml = take((size_t)kTailCtasMax * 2 * kTile * 8);
     w.total = off;
     return w;
 }
@@ -848,10 +830,36 @@ static int enqueue_run(const nomas_kv_cache *c, const nomas_segment_text *seg, c
         const int64_t wp = ((int64_t)p.n_pairs * H + sms - 1) / sms;
         pair = 16 * wp < 10 * wb;
     }
-    dim3 grid(pair ? (unsigned)p.n_pairs : (unsigned)lay.n_qblocks, (unsigned)H, nz);
+    // The pair kernel walks units (head, pair) head-major.  A dense call whose units leave a partial last
+    // wave (production segment: 1664 units on 148 SMs, 36 left over) runs each left-over unit as S
+    // shares of its list (S = SMs / left-over units, at most 16), so that the last wave is one wave of
+    // short CTAs; attn_combine_tail_kernel merges them (measured: whole lists in the last wave cost
+    // about 5 % of the call).
+    const int64_t units = (int64_t)p.n_pairs * H;
+    p.n_full = (int)units;
+    p.n_tail = p.tail_shares = p.tail_len = 0;
+    p.tail_o = reinterpret_cast<float *>(wsb + ws.tail_o);
+    p.tail_ml = reinterpret_cast<float2 *>(wsb + ws.tail_ml);
+    if (pair && mode == NOMAS_MODE_DENSE && share_len == 0) {
+        const int64_t sms = sm_count(), rem = units % sms;
+        if (units > sms && rem > 0) {
+            const int64_t S = std::min<int64_t>(std::min<int64_t>(16, sms / rem),
+                                                std::min<int64_t>(kTailCtasMax / rem, lay.list_cap));
+            if (S >= 2) {
+                p.n_full = (int)(units - rem);
+                p.n_tail = (int)rem;
+                p.tail_shares = (int)S;
+                p.tail_len = (int)((lay.list_cap + S - 1) / S);
+            }
+        }
+    }
+    const unsigned pair_ctas = (unsigned)(p.n_full + (int64_t)p.n_tail * p.tail_shares);
+    dim3 grid(pair ? pair_ctas : (unsigned)lay.n_qblocks, pair ? 1u : (unsigned)H, nz);
     int rc = pair ? launch_attn_pair(p, grid, maps, st)
              : D == 128 ? launch_attn<128>(p, grid, maps, st) : launch_attn<64>(p, grid, maps, st);
-    if (rc || share_len == 0) return rc;
+    if (rc) return rc;
+    if (p.tail_len > 0) return launch_combine_tail(p, D, st);
+    if (share_len == 0) return rc;
     const int64_t warps = Lt * H;
     const unsigned blocks = (unsigned)((warps * 32 + 255) / 256);
     if (D == 128)

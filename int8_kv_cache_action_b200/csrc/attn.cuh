@@ -44,6 +44,13 @@ struct AttnParams {
     int32_t share_len;
     float *part_o;              // [share][Nq][H][D]
     float2 *part_ml;            // [share][H][Nq]
+    // dense calls of the pair kernel (grid x = work units, unit = head * n_pairs + pair): units
+    // [0, n_full) run whole lists; each of the n_tail units after them runs as tail_shares CTAs of
+    // tail_len entries that write unnormalised partials for attn_combine_tail_kernel, so that the
+    // partial last wave of whole lists becomes one wave of short shares (tail_len == 0: no split)
+    int32_t n_full, n_tail, tail_shares, tail_len;
+    float *tail_o;              // [tail_shares][n_tail][2 * 128 rows][D]
+    float2 *tail_ml;            // [tail_shares][n_tail][2 * 128 rows]
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -157,7 +164,42 @@ __device__ __forceinline__ ColInfo column_info(const AttnParams &p, int h, const
     return ci;
 }
 
-// The pair kernel (head_dim 128): grid (query-block pairs, heads, list shares).
+// Softmax merge of one (row, head) over list shares: with M the largest offset among the shares that saw
+// a visible key, O = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M) and lse = (M + log2 of the
+// denominator) ln 2 (the kernels' log2 domain).  One warp, D / 32 channels per lane; share s of the
+// row's partial output starts at o + s * o_stride, its (offset, row sum) at ml[s * ml_stride].
+template <int D>
+__device__ __forceinline__ void merge_shares(const float *o, int64_t o_stride, const float2 *ml, int64_t ml_stride,
+                                             int n_share, float *dst, float *lse, int lane) {
+    float M = -INFINITY;
+    for (int s = 0; s < n_share; ++s) {
+        const float2 v = ml[s * ml_stride];
+        if (v.y > 0.0f) M = fmaxf(M, v.x);
+    }
+    constexpr int PL = D / 32;
+    float acc[PL];
+#pragma unroll
+    for (int i = 0; i < PL; ++i) acc[i] = 0.0f;
+    float L = 0.0f;
+    for (int s = 0; s < n_share; ++s) {
+        const float2 v = ml[s * ml_stride];
+        if (!(v.y > 0.0f)) continue;
+        const float wgt = exp2f(v.x - M);
+        L += v.y * wgt;
+        const float *src = o + s * o_stride;
+#pragma unroll
+        for (int i = 0; i < PL; ++i) acc[i] += src[lane + 32 * i] * wgt;
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+#pragma unroll
+    for (int i = 0; i < PL; ++i) dst[lane + 32 * i] = acc[i] * inv;
+    if (lse && lane == 0) *lse = (M + log2f(L)) * 0.69314718055994530942f;
+}
+
+// The pair kernel (head_dim 128): grid (work units, 1, list shares); with a tail split, grid x =
+// n_full + n_tail * tail_shares.
 int launch_attn_pair(const AttnParams &p, dim3 grid, const CUtensorMap *maps, cudaStream_t st);
+// Merge of the tail shares of a pair-kernel call into out / lse.
+int launch_combine_tail(const AttnParams &p, int D, cudaStream_t st);
 
 }  // namespace nomas

@@ -93,8 +93,17 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int pair = blockIdx.x;
-    const int h = blockIdx.y;
+    // work unit (head-major: the CTAs of one head run close together and share its K / V^T in L2) and,
+    // for a unit of the split tail, its share
+    int unit = blockIdx.x, tshare = 0;
+    const bool tail = p.tail_len > 0 && unit >= p.n_full;
+    if (tail) {
+        const int t = unit - p.n_full;
+        unit = p.n_full + t / p.tail_shares;
+        tshare = t - (t / p.tail_shares) * p.tail_shares;
+    }
+    const int h = unit / p.n_pairs;
+    const int pair = unit - h * p.n_pairs;
     constexpr int kBoth = kUse0 | kUse1;
     const int list_id = p.sparse ? h * p.n_pairs + pair : pair;
     const int4 *list = p.lists + (int64_t)list_id * p.expect.list_cap;   // advanced to this CTA's share below
@@ -118,10 +127,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     // this CTA's share of the list (a share past the list's end has nothing to do: the merge skips it)
     const int n_all = p.counts[list_id];
-    const bool partial = p.share_len > 0;
-    const int lo = partial ? (int)blockIdx.z * p.share_len : 0;
+    const bool partial = p.share_len > 0 || tail;
+    const int slen = tail ? p.tail_len : p.share_len;
+    const int lo = partial ? (tail ? tshare : (int)blockIdx.z) * slen : 0;
     if (partial && lo >= n_all) return;
-    const int n_tiles = partial ? min(p.share_len, n_all - lo) : n_all;
+    const int n_tiles = partial ? min(slen, n_all - lo) : n_all;
     list += lo;
 
     if (threadIdx.x == 0) {
@@ -477,8 +487,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (ok) {
             tc_fence_after();
             const float inv = partial ? 1.0f : (l > 0.0f ? 1.0f / l : 0.0f);
-            float *dst = (partial ? p.part_o + (int64_t)blockIdx.z * p.Nq * p.H * D : p.out) +
-                         (row * p.H + h) * (int64_t)D;
+            const int64_t trow = ((int64_t)tshare * p.n_tail + (unit - p.n_full)) * (2 * kTile) + qt * kTile + r;
+            float *dst = tail      ? p.tail_o + trow * D
+                         : partial ? p.part_o + ((int64_t)blockIdx.z * p.Nq * p.H + row * p.H + h) * D
+                                   : p.out + (row * p.H + h) * (int64_t)D;
 #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t rr[32];
@@ -493,7 +505,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     }
                 }
             }
-            if (partial && row_ok)
+            if (tail && row_ok)
+                p.tail_ml[trow] = make_float2(m_used, l);
+            else if (partial && row_ok)
                 p.part_ml[((int64_t)blockIdx.z * p.H + h) * p.Nq + row] = make_float2(m_used, l);
             else if (p.lse && row_ok)
                 p.lse[(int64_t)h * p.Nq + row] = (m_used + log2f(l)) * 0.69314718055994530942f;
@@ -506,6 +520,31 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// Merge of the split tail of a dense pair-kernel call: one warp per (tail unit, row of its query-block
+// pair); the unit's list of the block pair gives how many shares ran.
+template <int D>
+__global__ void __launch_bounds__(256) attn_combine_tail_kernel(const AttnParams p) {
+    const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (w >= (int64_t)p.n_tail * 2 * kTile) return;          // warp-uniform
+    const int tu = (int)(w / (2 * kTile)), rr = (int)(w - (int64_t)tu * 2 * kTile);
+    const int unit = p.n_full + tu;
+    const int h = unit / p.n_pairs, pair = unit - h * p.n_pairs;
+    const int64_t row = (int64_t)pair * 2 * kTile + rr;
+    if (row >= p.Nq) return;
+    const int n_share = min(p.tail_shares, (p.counts[pair] + p.tail_len - 1) / p.tail_len);
+    const int64_t t0 = (int64_t)tu * 2 * kTile + rr, stride = (int64_t)p.n_tail * 2 * kTile;
+    merge_shares<D>(p.tail_o + t0 * D, stride * D, p.tail_ml + t0, stride, n_share, p.out + (row * p.H + h) * (int64_t)D,
+                    p.lse ? p.lse + (int64_t)h * p.Nq + row : nullptr, lane);
+}
+
+int launch_combine_tail(const AttnParams &p, int D, cudaStream_t st) {
+    if (D != 128) return NOMAS_EUNSUPPORTED;
+    const int64_t warps = (int64_t)p.n_tail * 2 * kTile;
+    attn_combine_tail_kernel<128><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(p);
+    return check_launch("attn_combine_tail_kernel launch");
 }
 
 int launch_attn_pair(const AttnParams &p, dim3 grid, const CUtensorMap *maps, cudaStream_t st) {

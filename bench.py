@@ -48,9 +48,24 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # Kernel launches of one step: append 1; dense mask 3; prepare 1 (key copy, transposed values and history
-# widening in one launch); dense attention 1; text mask 3; text attention 2 (the list shares, their
-# merge); sparse mask 5; sparse attention 1.
+# widening in one launch); dense attention 1, plus 1 when the pair kernel splits its partial last wave
+# (dense_attention_launches); text mask 3; text attention 2 (the list shares, their merge); sparse mask
+# 5; sparse attention 1.
 LAUNCHES_PER_STEP = 17
+
+
+def dense_attention_launches(n_query, heads, sms):
+    """Launches of a dense nomas_attn_run at head_dim 128: the library's per-call choice of the pair
+    kernel (1.6 x its waves < the block kernel's) and its last-wave split (left-over units run as
+    min(16, SMs / left-over, 256 / left-over) >= 2 shares, merged by one more launch)."""
+    blocks = (n_query + 127) // 128
+    pairs = (blocks + 1) // 2
+    wb, wp = -(-blocks * heads // sms), -(-pairs * heads // sms)
+    if not 16 * wp < 10 * wb:
+        return 1
+    units = pairs * heads
+    rem = units % sms
+    return 2 if units > sms and rem > 0 and min(16, sms // rem, 256 // rem) >= 2 else 1
 CSRC = os.path.join(ROOT, "int8_kv_cache_action_b200", "csrc")
 COMMON = os.path.join(CSRC, "common.cuh")
 TRAFFIC = {  # kernel -> (ncu summary with DRAM bytes per launch, sources whose digest it was taken with)
@@ -695,7 +710,8 @@ def main():
         "kv_tokens_per_s_append": (cfg.window_frames * cfg.tokens_per_frame) * cfg.heads / (ph[0] * 1e-3),
         "cpu_baseline": cpu_base,
         "e2e": r["e2e"],
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP - 1 + dense_attention_launches(
+            cfg.n_query, cfg.heads, torch.cuda.get_device_properties(local_rank).multi_processor_count)) * args.steps,
         "clocks": r["clocks"],
     }
     print(json.dumps(line))

@@ -218,7 +218,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             bool acc_on[2] = {false, false}; // O_t holds a product
             // PV_t of entry `ent` once query tile t's P is stored and V^T has landed
             auto issue_pv = [&](int t, int ent) -> bool {
-                if (!mbar_wait(&p_full[t], (cnt[t] - 1) & 1, wd, 3)) return false;
+                // the P hand-off is on the critical path of each query tile: poll without suspending
+                if (!mbar_wait_spin(&p_full[t], (cnt[t] - 1) & 1, wd, 3)) return false;
                 const int sv = ent % C::NV;
                 if (!mbar_wait(&v_full[sv], (ent / C::NV) & 1, wd, 4)) return false;
                 tc_fence_after();

@@ -107,6 +107,29 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
     }
 }
 
+// The same wait polling with test_wait (never suspending the thread): for a single thread on the
+// critical path of a short hand-off, where a suspended try_wait wakes late.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, const Watchdog &wd, int site) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if (wd.limit_ns == 0) {
+        set_device_error(wd.err, NOMAS_ETIMEOUT, wd.where * 100 + site);
+        *wd.abort = 1;
+        return false;
+    }
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_test_wait(bar, parity)) return true;
+        if (*wd.abort) return false;
+        if (globaltimer_ns() - t0 > wd.limit_ns) {
+            set_device_error(wd.err, NOMAS_ETIMEOUT, wd.where * 100 + site);
+            *wd.abort = 1;
+            return false;
+        }
+    }
+}
+
 // Drain wait used on the abort path: ignores the abort flag, gives up after limit_ns.
 __device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
     const uint64_t t0 = globaltimer_ns();

@@ -18,7 +18,7 @@ def _attention(gc, cfg, d, seg):
     return out
 
 
-def test_forced_wait_limit_reports_timeout_and_context_stays_usable():
+def test_forced_wait_limit_reports_timeout_and_context_stays_usable(attn_kernel):
     from int8_kv_cache_action_b200.runtime import segment_text_of
     cfg = small_config(tokens_per_frame=150, n_frames=3, prior_frames=(3, 3), window=4)
     inp = make_inputs(cfg)

@@ -162,6 +162,33 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch: a grid launched by launch_pdl is launched as the previous grid of the
+// stream retires its CTAs (no explicit trigger: each CTA's exit is its trigger), instead of after that
+// grid's completion has been processed; griddep_wait then blocks until the previous grid has completed
+// and its memory operations are visible (a no-op for a grid launched without the attribute).  Every
+// kernel launched this way calls griddep_wait before it touches global memory, so the stream order of
+// reads and writes is kept.  (Triggering at the start of each CTA instead let the next grid's CTAs
+// take SM slots early: the sparse mask build went from 0.108 to 0.131 ms; without it, 0.099.)
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+static inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                     Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// ---------------------------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y, int z) {

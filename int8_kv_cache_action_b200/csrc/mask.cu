@@ -69,6 +69,7 @@ __device__ __forceinline__ TileInfo tile_info(const MaskParams &p, int j) {
 
 // Header + per-text-token visibility window [lo, hi) in segment-local latent frames.
 __global__ void mask_prep_kernel(MaskParams p) {
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (i == 0) *reinterpret_cast<MaskHeader *>(p.buf) = p.hdr;
     if (i >= p.Lt) return;
@@ -93,6 +94,7 @@ __global__ void mask_prep_kernel(MaskParams p) {
 // each (query block, text tile): lanes hold the windows of 4 keys each and, frame by frame over the
 // block's rows, count the keys visible to that frame.
 __global__ void class_map_kernel(MaskParams p, int plain_blocks) {
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     int8_t *cls = reinterpret_cast<int8_t *>(p.buf + p.lay.off_class);
     const int n_plain = p.n_tiles - p.n_text_tiles;      // text tiles come last in tile order
     if ((int)blockIdx.x < plain_blocks) {
@@ -143,6 +145,7 @@ __device__ __forceinline__ VisCode text_key_code(const MaskParams &p, int64_t i)
 
 __global__ void __launch_bounds__(128) class_map_text_kernel(MaskParams p) {
     __shared__ VisCode skey[kTile];
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     const int b = blockIdx.x / p.n_tiles, j = blockIdx.x % p.n_tiles;
     const TileInfo ti = tile_info(p, j);
     int8_t *cls = reinterpret_cast<int8_t *>(p.buf + p.lay.off_class) + (int64_t)b * p.n_tiles + j;
@@ -181,6 +184,7 @@ __device__ __forceinline__ int mask_flag(int8_t cls, int32_t count) { return (cl
 // Dense lists: one warp per pair of query blocks (one attention CTA pair); lists are head-independent.
 // Lanes test 32 tiles at a time and kept tiles are compacted in index order.
 __global__ void lists_dense_kernel(MaskParams p) {
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     const int pr = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
     const int lane = threadIdx.x & 31;
     if (pr >= p.n_lists) return;   // warp-uniform
@@ -346,6 +350,7 @@ __global__ void __launch_bounds__(kPoolThreads) pool_kernel(const __grid_constan
                                                             const __grid_constant__ CUtensorMap tk,
                                                             const __grid_constant__ MaskParams p,
                                                             const PoolParams pp) {
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     using C = PoolCfg<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -474,6 +479,7 @@ constexpr int kScoreTile = 64;
 __global__ void __launch_bounds__(256) score_kernel(MaskParams p, const float *qmean, const float *kmean) {
     __shared__ __align__(16) float sq[64][kScoreTile];   // [channel in chunk][query block]
     __shared__ __align__(16) float sk[64][kScoreTile];   // [channel in chunk][candidate]
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     const int D = p.D;
     const int h = blockIdx.y;
     const int n_ct = (p.n_cand + kScoreTile - 1) / kScoreTile;   // candidate tiles; x = qb tile * n_ct + ct
@@ -644,6 +650,7 @@ __device__ __forceinline__ void warp_merge_up(unsigned long long (&a)[M], int la
 // rank order -- the same result as sorting every key.  Then warps 0..3 write the CTA's pair lists.
 __global__ void __launch_bounds__(256, 4) select_lists_top128_kernel(MaskParams p) {
     __shared__ uint32_t bits[8][32];             // kept-candidate bit mask per query block (1024 bits)
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     const int n_pairs = (p.n_qb + 1) / 2;
     const int groups = (n_pairs + 3) / 4;
     const int h = blockIdx.x / groups, g = blockIdx.x - h * groups;
@@ -705,6 +712,7 @@ __global__ void __launch_bounds__(256, 4) select_lists_top128_kernel(MaskParams 
 template <int M>
 __global__ void __launch_bounds__(256, M >= 32 ? 1 : 2) select_lists_warp_kernel(MaskParams p) {
     __shared__ uint32_t bits[8][M];            // kept-candidate bit mask per query block (32 M bits)
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     const int n_pairs = (p.n_qb + 1) / 2;
     const int groups = (n_pairs + 3) / 4;
     const int h = blockIdx.x / groups, g = blockIdx.x - h * groups;
@@ -750,6 +758,7 @@ __global__ void __launch_bounds__(256, M >= 32 ? 1 : 2) select_lists_warp_kernel
 __global__ void __launch_bounds__(256) select_lists_kernel(MaskParams p, int npow2) {
     extern __shared__ unsigned long long keys[];                 // [2][npow2]
     uint32_t *bits = reinterpret_cast<uint32_t *>(keys + 2 * npow2);   // [2][words]
+    griddep_wait();   // the previous grid of the stream has completed (programmatic launch)
     const int n_pairs = (p.n_qb + 1) / 2;
     const int hp = blockIdx.x;           // h * n_pairs + pair
     const int h = hp / n_pairs, pr = hp % n_pairs;
@@ -914,33 +923,33 @@ static int enqueue_mask(const MaskParams &p, float *qmean, float *kmean, cudaStr
                                 CU_TENSOR_MAP_SWIZZLE_NONE))
             return NOMAS_ECUDA;
     }
-    mask_prep_kernel<<<nblk(p.Lt > 0 ? p.Lt : 1, 256), 256, 0, st>>>(p);
+    launch_pdl(mask_prep_kernel, nblk(p.Lt > 0 ? p.Lt : 1, 256), 256, 0, st, p);
     if (p.hdr.mode == NOMAS_MODE_TEXT) {
-        class_map_text_kernel<<<(unsigned)((int64_t)p.n_qb * p.n_tiles), 128, 0, st>>>(p);
-        lists_dense_kernel<<<nblk((int64_t)p.n_lists * 32, 128), 128, 0, st>>>(p);
+        launch_pdl(class_map_text_kernel, (unsigned)((int64_t)p.n_qb * p.n_tiles), 128, 0, st, p);
+        launch_pdl(lists_dense_kernel, nblk((int64_t)p.n_lists * 32, 128), 128, 0, st, p);
         return check_launch("mask_build kernels launch");
     }
     {
         const unsigned plain = nblk((int64_t)p.n_qb * (p.n_tiles - p.n_text_tiles), 256);
         const unsigned text = nblk((int64_t)p.n_qb * p.n_text_tiles * 32, 256);
-        if (plain + text > 0) class_map_kernel<<<plain + text, 256, 0, st>>>(p, (int)plain);
+        if (plain + text > 0) launch_pdl(class_map_kernel, plain + text, 256, 0, st, p, (int)plain);
     }
     if (!sp) {
-        lists_dense_kernel<<<nblk((int64_t)p.n_lists * 32, 128), 128, 0, st>>>(p);
+        launch_pdl(lists_dense_kernel, nblk((int64_t)p.n_lists * 32, 128), 128, 0, st, p);
     } else {
         int64_t blocks = (int64_t)3 * sm_count();     // three CTAs per SM (shared memory)
         if (blocks > pp.n_units) blocks = pp.n_units;
-        if (p.D == 128) pool_kernel<128><<<(unsigned)blocks, kPoolThreads, PoolCfg<128>::SMEM, st>>>(tq, tk, p, pp);
-        else pool_kernel<64><<<(unsigned)blocks, kPoolThreads, PoolCfg<64>::SMEM, st>>>(tq, tk, p, pp);
+        if (p.D == 128) launch_pdl(pool_kernel<128>, (unsigned)blocks, kPoolThreads, PoolCfg<128>::SMEM, st, tq, tk, p, pp);
+        else launch_pdl(pool_kernel<64>, (unsigned)blocks, kPoolThreads, PoolCfg<64>::SMEM, st, tq, tk, p, pp);
         const dim3 sg(nblk(p.n_cand, kScoreTile) * nblk(p.n_qb, kScoreTile), (unsigned)p.H);
-        score_kernel<<<sg, 256, 0, st>>>(p, qmean, kmean);
+        launch_pdl(score_kernel, sg, 256, 0, st, p, (const float *)qmean, (const float *)kmean);
         const int npow2 = pow2_at_least(p.n_cand);
         const unsigned groups = (unsigned)(((p.n_qb + 1) / 2 + 3) / 4);
-        if (p.keep <= 128 && p.n_cand <= 1024) select_lists_top128_kernel<<<p.H * groups, 256, 0, st>>>(p);
-        else if (npow2 <= 256) select_lists_warp_kernel<8><<<p.H * groups, 256, 0, st>>>(p);
-        else if (npow2 <= 512) select_lists_warp_kernel<16><<<p.H * groups, 256, 0, st>>>(p);
-        else if (npow2 <= 1024) select_lists_warp_kernel<32><<<p.H * groups, 256, 0, st>>>(p);
-        else select_lists_kernel<<<p.H * ((p.n_qb + 1) / 2), 256, select_smem(npow2, p.n_cand), st>>>(p, npow2);
+        if (p.keep <= 128 && p.n_cand <= 1024) launch_pdl(select_lists_top128_kernel, p.H * groups, 256, 0, st, p);
+        else if (npow2 <= 256) launch_pdl(select_lists_warp_kernel<8>, p.H * groups, 256, 0, st, p);
+        else if (npow2 <= 512) launch_pdl(select_lists_warp_kernel<16>, p.H * groups, 256, 0, st, p);
+        else if (npow2 <= 1024) launch_pdl(select_lists_warp_kernel<32>, p.H * groups, 256, 0, st, p);
+        else launch_pdl(select_lists_kernel, p.H * ((p.n_qb + 1) / 2), 256, select_smem(npow2, p.n_cand), st, p, npow2);
     }
     return check_launch("mask_build kernels launch");
 }

@@ -114,3 +114,14 @@ def test_text_row_key_count_matches_the_oracle_mask(name):
     lp = sum(p.head_len for p in cfg.prior)
     m = vis.text_query_mask(lh, lp, cfg.n_query, cfg.tokens_per_frame, cfg.current)
     assert bench.text_key_sum(cfg, lh, lp) == int(m.sum())
+
+
+def test_dense_attention_launch_count_follows_the_kernel_choice():
+    # the bench's launch claim: the production segment runs the pair kernel with a split last wave (two
+    # launches: the kernel and the merge of the split units); the 480 x 832 shape runs one block per
+    # CTA (one launch); a unit count that is a multiple of the SM count leaves no wave to split
+    from bench import dense_attention_launches
+    assert dense_attention_launches(26400, 16, 148) == 2       # 1664 pair units, 36 left over
+    assert dense_attention_launches(3120, 16, 148) == 1        # pairs take 2 waves against 3 for blocks
+    assert dense_attention_launches(148 * 256, 2, 148) == 1    # 148 x 2 units: whole waves only
+    assert dense_attention_launches(26400, 16, 132) == 1       # 80 left over of 132: no two shares fit

@@ -29,6 +29,10 @@
 // PV_t(j-1) is issued before S_t(j), the completion of S_t(j) implies that of PV_t(j-1): the softmax
 // may rescale O_t as soon as it sees S_t(j), and S_t(j) may overwrite P_t(j-1) (in-order execution).
 // A tile skipped by one query tile costs that tile's warps only the column-info hand-off.
+//
+// Grid: one CTA per work unit (head, pair), head-major.  For a dense call whose units leave a partial
+// last wave, the host splits each left-over unit into list shares (AttnParams::n_full / tail_*): such
+// a CTA runs one share and writes unnormalised partials that attn_combine_tail_kernel merges.
 #include <cmath>
 #include <cuda_fp16.h>
 

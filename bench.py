@@ -461,9 +461,9 @@ def measure_linear(dev, reps=10):
 
 
 def per_config(args):
-    """One JSON line per config: the attention call (its mode: dense, or sparse for C3) timed with CUDA
-    events over back-to-back calls after 3 warm-ups, and the quantise-append of one 30-frame (C0: 2)
-    segment into a fresh cache of the config's dimensions."""
+    """One JSON line per config: the attention call (its mode: dense, or sparse for C3) and the mask
+    build of that mode timed with CUDA events over back-to-back calls after 3 warm-ups, and the
+    quantise-append of one 30-frame (C0: 2) segment into a fresh cache of the config's dimensions."""
     import torch
     from int8_kv_cache_action_b200 import _nomas as N
     from int8_kv_cache_action_b200.runtime import KVCache, mask_views, segment_text_of
@@ -505,6 +505,16 @@ def per_config(args):
         e1.record()
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / reps
+        # the mask build of the call's mode (sparse: block means, scores, ranking and lists)
+        for _ in range(3):
+            cache.build_mask(seg, cfg.mode, cfg.keep_frac, q, kc, mask_buf=buf)
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            cache.build_mask(seg, cfg.mode, cfg.keep_frac, q, kc, mask_buf=buf)
+        e1.record()
+        torch.cuda.synchronize()
+        mask_ms = e0.elapsed_time(e1) / reps
         status = cache.status()
         # append: the config's last prior segment (or the current segment's K/V) into a fresh cache
         src = inp.prior[-1] if cfg.prior else None
@@ -525,6 +535,7 @@ def per_config(args):
         app_bytes = kept * cfg.tokens_per_frame * cfg.heads * APPEND_BYTES_PER_TOKEN_HEAD(cfg.head_dim)
         print(json.dumps({"config": name, "workload": cfg.name, "mode": "sparse" if cfg.mode else "dense",
                           "attn_ms": ms, "attn_tflops": flops / (ms * 1e-3) / 1e12, "attn_flops": flops,
+                          "mask_ms": mask_ms,
                           "append_ms": app_ms, "append_gbs": app_bytes / (app_ms * 1e-3) / 1e9,
                           "append_kv_tokens_per_s": kept * cfg.tokens_per_frame * cfg.heads / (app_ms * 1e-3),
                           "status": status}), flush=True)
